@@ -1,0 +1,82 @@
+"""Work accounting for the attention workloads: visible (query, key) pairs, FLOPs and bytes.
+
+Closed forms only (no enumeration), so the benchmark can count work at any size.  The test
+suite pins every closed form against brute-force enumeration of the mask definition.
+
+Mask definitions (the same reading the library implements):
+  FULL     every key is visible;
+  CAUSAL   key j is visible to query row i iff j <= p_i, with p_i = i + Nk - Nq
+           (bottom-right alignment when Nq != Nk);
+  SLIDING  causal, and either p_i - w < j (a left window of w keys including the diagonal,
+           "each token attends to w neighbouring tokens" in "Quadratic Complexity Bottleneck",
+           sparse-attention section) or j < n_sink (always-visible sink tokens, "Attention
+           Research", section 4).
+
+FLOPs count 4*d per visible pair (2*d for Q K^T, 2*d for P V), the standard count for the
+forward pass of "Chapter 3.1 - The Cost of Attention", section 2; masked pairs and tile padding
+are not credited.
+"""
+
+from __future__ import annotations
+
+MASK_FULL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2
+
+
+def _sum_min_w(lo: int, hi: int, w: int) -> int:
+    """sum_{x=lo}^{hi} min(w, x) for integers 0 <= lo, with hi < lo meaning an empty sum."""
+    if hi < lo:
+        return 0
+    total = 0
+    a, b = lo, min(hi, w)
+    if a <= b:
+        total += (a + b) * (b - a + 1) // 2
+    a = max(lo, w + 1)
+    if a <= hi:
+        total += w * (hi - a + 1)
+    return total
+
+
+def visible_pairs(Nq: int, Nk: int, mask_kind: int, window: int = 0, n_sink: int = 0) -> int:
+    """Visible (query, key) pairs of one (b, h) slice."""
+    if Nq <= 0 or Nk <= 0:
+        return 0
+    off = Nk - Nq
+    if mask_kind == MASK_FULL:
+        return Nq * Nk
+    # causal row i sees keys 0..p_i (p_i = i + off) clipped to [0, Nk): count c_i = clip(p_i + 1)
+    p_lo, p_hi = off, Nq - 1 + off  # p ranges over [p_lo, p_hi]; p_hi = Nk - 1
+    lo = max(p_lo, -1)
+    if mask_kind == MASK_CAUSAL:
+        # sum over p of max(0, p + 1), p <= Nk - 1 always
+        a = max(lo, 0)
+        if a > p_hi:
+            return 0
+        return (a + 1 + p_hi + 1) * (p_hi - a + 1) // 2
+    if mask_kind != MASK_SLIDING:
+        raise ValueError("mask_kind")
+    w, s = window, n_sink
+    a = max(lo, 0)
+    if a > p_hi:
+        return 0
+    # window part: min(w, p + 1) keys for each p in [a, p_hi]
+    total = _sum_min_w(a + 1, p_hi + 1, w)
+    # sinks outside the window: keys j < s with j <= p - w  ->  max(0, min(s, p - w + 1))
+    total += _sum_min_w(max(a - w + 1, 0), p_hi - w + 1, s) if s > 0 else 0
+    return total
+
+
+def attn_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int, window: int = 0,
+               n_sink: int = 0) -> int:
+    """Unmasked forward FLOPs: 4*d per visible pair, over every (b, query head)."""
+    return 4 * d * B * Hq * visible_pairs(Nq, Nk, mask_kind, window, n_sink)
+
+
+def attn_fwd_bytes(B: int, Hq: int, Hkv: int, Nq: int, Nk: int, d: int, elem: int = 2) -> int:
+    """Unique HBM bytes of one forward call: Q, K, V read once, O written once, fp32 LSE."""
+    return elem * d * (2 * B * Hq * Nq + 2 * B * Hkv * Nk) + 4 * B * Hq * Nq
+
+
+def decode_bytes(B: int, Hq: int, Hkv: int, Nk: int, d: int, elem: int = 2) -> int:
+    """Algorithmic bytes of one decode call: the K and V cache once (shared by the G query heads
+    of a group), Q read, O written, fp32 LSE written."""
+    return elem * d * 2 * B * Hkv * Nk + elem * d * 2 * B * Hq + 4 * B * Hq

@@ -1,0 +1,198 @@
+/*
+ * Exact attention oracle: plain, slow, fp64 CPU implementation of
+ *
+ *     O = softmax(Q K^T * scale + mask) V,   LSE_i = ln sum_{visible j} exp(scale * q_i . k_j)
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg may load this library.  It shares no code, header or constant with the CUDA
+ * library and includes no CUDA header.
+ *
+ * What it follows:
+ *  - "Chapter 3.1 - The Cost of Attention" (llmis.ru), section 2: Q, K, V of shape (n, d),
+ *    output softmax(Q K^T / sqrt(d)) V.  The caller passes the scale (1/sqrt(d) in every
+ *    workload) so scale = 0 and other finite values can be checked too.
+ *  - Same page, section 5: the tiled method must give this exact result, so the oracle is the
+ *    definition written out with no tiling, no blocking and no online softmax: for each query
+ *    row it materialises the full row of scores over all Nk keys, masks it, takes the
+ *    max-subtracted softmax and forms P V.
+ *  - Masks: sliding window of w neighbouring tokens ("Quadratic Complexity Bottleneck",
+ *    sparse attention and sliding window sections; "Attention Research", section 4), read as
+ *    the causal left window of w keys including the diagonal; always-visible sink tokens
+ *    ("Attention Research", section 4), read as key positions 0..n_sink-1, still causal.
+ *  - GQA ("Quadratic Complexity Bottleneck", grouped-query attention): query heads are
+ *    partitioned into Hkv contiguous groups of G = Hq / Hkv; query head h reads kv head h / G.
+ *  - Causal alignment when Nq != Nk (the pages are silent): bottom-right, query row i sits at
+ *    key position p_i = i + Nk - Nq, so a one-token decode equals the last prefill row.
+ *  - A row with no visible key gets O = 0 and LSE = -inf.
+ *
+ * Layouts (row-major, d innermost): Q, O [B][Hq][Nq][d]; K, V [B][Hkv][Nk][d]; LSE [B][Hq][Nq].
+ * Parallelism: OpenMP over independent query rows; each row's arithmetic is sequential.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_MASK_FULL 0
+#define ORACLE_MASK_CAUSAL 1
+#define ORACLE_MASK_SLIDING 2
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Visibility of key j to the query at absolute key position p (see header comment). */
+int oracle_visible(int64_t p, int64_t j, int mask_kind, int64_t window, int64_t n_sink) {
+    if (mask_kind == ORACLE_MASK_FULL) return 1;
+    if (j > p) return 0; /* causal */
+    if (mask_kind == ORACLE_MASK_CAUSAL) return 1;
+    if (j > p - window) return 1; /* inside the window: p - w < j <= p */
+    if (j < n_sink) return 1;     /* sink tokens */
+    return 0;
+}
+
+static int check_args(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window,
+                      int n_sink) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 0 || d < 1) return -1;
+    if (Hq % Hkv != 0) return -1;
+    if (mask_kind < 0 || mask_kind > 2) return -1;
+    if (mask_kind == ORACLE_MASK_SLIDING && window < 1) return -1;
+    if (n_sink < 0) return -1;
+    return 0;
+}
+
+/*
+ * One query row: scores over every key, mask, softmax, P V.
+ * s and e are caller-provided scratch of Nk doubles each.
+ */
+static void attend_row(const double *q, const double *K, const double *V, int Nk, int d,
+                       int64_t p, int mask_kind, int window, int n_sink, double scale,
+                       double *s, unsigned char *vis, double *o, double *lse) {
+    int64_t j;
+    int t;
+    int any = 0;
+    double m = -INFINITY, l = 0.0;
+    /* 1. the full row of scores s_j = scale * q . k_j */
+    for (j = 0; j < Nk; ++j) {
+        double acc = 0.0;
+        for (t = 0; t < d; ++t) acc += q[t] * K[j * (int64_t)d + t];
+        s[j] = scale * acc;
+        vis[j] = (unsigned char)oracle_visible(p, j, mask_kind, window, n_sink);
+        if (vis[j]) {
+            if (!any || s[j] > m) m = s[j];
+            any = 1;
+        }
+    }
+    for (t = 0; t < d; ++t) o[t] = 0.0;
+    if (!any) {
+        *lse = -INFINITY;
+        return;
+    }
+    /* 2. max-subtracted exponentials and their sum */
+    for (j = 0; j < Nk; ++j) {
+        s[j] = vis[j] ? exp(s[j] - m) : 0.0;
+        l += s[j];
+    }
+    /* 3. O = P V with P = e / l */
+    for (j = 0; j < Nk; ++j) {
+        if (!vis[j]) continue;
+        double pj = s[j] / l;
+        for (t = 0; t < d; ++t) o[t] += pj * V[j * (int64_t)d + t];
+    }
+    *lse = m + log(l);
+}
+
+/* Full forward: every row of every (b, h). Returns 0, or -1 on invalid arguments. */
+int oracle_attn(const double *q, const double *k, const double *v, double *o, double *lse, int B,
+                int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                double scale) {
+    if (check_args(B, Hq, Hkv, Nq, Nk, d, mask_kind, window, n_sink)) return -1;
+    const int G = Hq / Hkv;
+    const int64_t rows = (int64_t)B * Hq * Nq;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        unsigned char *vis = (unsigned char *)malloc((size_t)(Nk > 0 ? Nk : 1));
+        if (!s || !vis) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            int64_t r;
+#pragma omp for schedule(dynamic, 16)
+            for (r = 0; r < rows; ++r) {
+                int64_t i = r % Nq;
+                int64_t bh = r / Nq;
+                int64_t h = bh % Hq, b = bh / Hq;
+                int64_t hk = h / G;
+                const double *Kb = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                double l_out;
+                attend_row(q + r * d, Kb, Vb, Nk, d, i + (int64_t)Nk - Nq, mask_kind, window,
+                           n_sink, scale, s, vis, o + r * d, &l_out);
+                if (lse) lse[r] = l_out;
+            }
+        }
+        free(s);
+        free(vis);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Selected rows only.  rows[] holds flat row indices r = (b * Hq + h) * Nq + i; the results go
+ * to o_rows[n_rows][d] and lse_rows[n_rows].  Same arithmetic as oracle_attn, row by row.
+ */
+int oracle_attn_rows(const double *q, const double *k, const double *v, int B, int Hq, int Hkv,
+                     int Nq, int Nk, int d, int mask_kind, int window, int n_sink, double scale,
+                     const int64_t *rows, int64_t n_rows, double *o_rows, double *lse_rows) {
+    if (check_args(B, Hq, Hkv, Nq, Nk, d, mask_kind, window, n_sink)) return -1;
+    const int G = Hq / Hkv;
+    const int64_t total = (int64_t)B * Hq * Nq;
+    int64_t n;
+    for (n = 0; n < n_rows; ++n)
+        if (rows[n] < 0 || rows[n] >= total) return -1;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        unsigned char *vis = (unsigned char *)malloc((size_t)(Nk > 0 ? Nk : 1));
+        if (!s || !vis) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            int64_t t;
+#pragma omp for schedule(dynamic, 1)
+            for (t = 0; t < n_rows; ++t) {
+                int64_t r = rows[t];
+                int64_t i = r % Nq;
+                int64_t bh = r / Nq;
+                int64_t h = bh % Hq, b = bh / Hq;
+                int64_t hk = h / G;
+                const double *Kb = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                attend_row(q + r * d, Kb, Vb, Nk, d, i + (int64_t)Nk - Nq, mask_kind, window,
+                           n_sink, scale, s, vis, o_rows + t * d, &lse_rows[t]);
+            }
+        }
+        free(s);
+        free(vis);
+    }
+    return failed ? -2 : 0;
+}
+
+/* Number of visible (query, key) pairs of one (b, h) slice: the pair count behind FLOP totals. */
+int64_t oracle_visible_pairs(int Nq, int Nk, int mask_kind, int window, int n_sink) {
+    int64_t i, j, c = 0;
+    for (i = 0; i < Nq; ++i)
+        for (j = 0; j < Nk; ++j)
+            c += oracle_visible(i + (int64_t)Nk - Nq, j, mask_kind, window, n_sink);
+    return c;
+}

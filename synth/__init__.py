@@ -1,0 +1,136 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle harness.
+
+This module only draws numbers; it holds none of the attention arithmetic.
+
+Generator (counter based, so any element can be drawn on its own and any
+device produces the same stream):
+
+    key   = (seed << 40) ^ (tensor_id << 32) ^ idx          (idx < 2**32)
+    x     = splitmix64(key)                                  (Steele, Lea & Flood, 2014)
+    u1    = ((x >> 40) + 0.5) / 2**24                        in (0, 1)
+    u2    = ((x >> 16) & 0xFFFFFF) / 2**24                   in [0, 1)
+    z     = sqrt(-2 ln u1) * cos(2 pi u2)                    Box-Muller, fp64
+    value = fp32(z), then bf16 by round-to-nearest-even for the bf16 workloads
+
+Tensor ids: Q = 0, K = 1, V = 2.  ``idx`` is the flat row-major element index.
+The workloads draw Q, K and V iid N(0, 1), as the configurations of the exact
+attention benchmark state.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+Q_ID, K_ID, V_ID = 0, 1, 2
+
+_GOLDEN = 0x9E3779B97F4A7C15
+_M1 = 0xBF58476D1CE4E5B9
+_M2 = 0x94D049BB133111EB
+_MASK64 = (1 << 64) - 1
+_CHUNK = 1 << 24
+
+
+def splitmix64_np(z: np.ndarray) -> np.ndarray:
+    """SplitMix64 finaliser over a uint64 array (wrapping arithmetic)."""
+    z = z.astype(np.uint64, copy=True)
+    with np.errstate(over="ignore"):
+        z += np.uint64(_GOLDEN)
+        z = (z ^ (z >> np.uint64(30))) * np.uint64(_M1)
+        z = (z ^ (z >> np.uint64(27))) * np.uint64(_M2)
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def _keys(seed: int, tensor_id: int, start: int, count: int) -> np.ndarray:
+    if start + count > (1 << 32):
+        raise ValueError("element index must stay below 2**32")
+    base = ((seed << 40) ^ (tensor_id << 32)) & _MASK64
+    idx = np.arange(start, start + count, dtype=np.uint64)
+    return idx ^ np.uint64(base)
+
+
+def _box_muller(x: np.ndarray) -> np.ndarray:
+    u1 = ((x >> np.uint64(40)).astype(np.float64) + 0.5) * (1.0 / (1 << 24))
+    u2 = ((x >> np.uint64(16)) & np.uint64(0xFFFFFF)).astype(np.float64) * (1.0 / (1 << 24))
+    return np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+
+
+def normal_f32(seed: int, tensor_id: int, shape) -> np.ndarray:
+    """iid N(0,1) drawn in fp64 and rounded once to fp32."""
+    n = int(np.prod(shape, dtype=np.int64))
+    out = np.empty(n, dtype=np.float32)
+    for s in range(0, n, _CHUNK):
+        c = min(_CHUNK, n - s)
+        out[s:s + c] = _box_muller(splitmix64_np(_keys(seed, tensor_id, s, c))).astype(np.float32)
+    return out.reshape(shape)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 to bf16 (round to nearest, ties to even); returns the uint16 bit patterns."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    r = (b + np.uint64(0x7FFF) + ((b >> np.uint64(16)) & np.uint64(1))) >> np.uint64(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to fp32."""
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def normal_bf16_bits(seed: int, tensor_id: int, shape) -> np.ndarray:
+    """iid N(0,1) as bf16 bit patterns (uint16), drawn as in ``normal_f32`` and rounded once."""
+    return f32_to_bf16_bits(normal_f32(seed, tensor_id, shape)).reshape(shape)
+
+
+# --------------------------------------------------------------------------------------------
+# torch implementation of the same counter-based stream (used to fill large device buffers
+# directly on the GPU; equality with the numpy stream is checked on the CPU by the tests).
+# --------------------------------------------------------------------------------------------
+
+def _s64(c: int) -> int:
+    c &= _MASK64
+    return c - (1 << 64) if c >= (1 << 63) else c
+
+
+def _lsr(x, k: int):
+    import torch  # noqa: F401
+
+    return (x >> k) & ((1 << (64 - k)) - 1)
+
+
+def splitmix64_torch(z):
+    """SplitMix64 on an int64 tensor, interpreting the bits as uint64 (wrapping)."""
+    z = z + _s64(_GOLDEN)
+    z = (z ^ _lsr(z, 30)) * _s64(_M1)
+    z = (z ^ _lsr(z, 27)) * _s64(_M2)
+    return z ^ _lsr(z, 31)
+
+
+def normal_torch(seed: int, tensor_id: int, shape, dtype=None, device="cpu"):
+    """Fill a tensor of ``shape`` on ``device`` with the same stream as ``normal_f32``.
+
+    ``dtype`` is torch.float32 or torch.bfloat16 (bf16 by round-to-nearest-even from fp32).
+    """
+    import math
+
+    import torch
+
+    dtype = torch.bfloat16 if dtype is None else dtype
+    n = 1
+    for s in shape:
+        n *= int(s)
+    if n > (1 << 32):
+        raise ValueError("element index must stay below 2**32")
+    out = torch.empty(n, dtype=dtype, device=device)
+    base = _s64((seed << 40) ^ (tensor_id << 32))
+    chunk = 1 << 26
+    for s in range(0, n, chunk):
+        c = min(chunk, n - s)
+        idx = torch.arange(s, s + c, dtype=torch.int64, device=device)
+        x = splitmix64_torch(idx ^ base)
+        u1 = (_lsr(x, 40).to(torch.float64) + 0.5) * (1.0 / (1 << 24))
+        u2 = (_lsr(x, 16) & 0xFFFFFF).to(torch.float64) * (1.0 / (1 << 24))
+        z = torch.sqrt(-2.0 * torch.log(u1)) * torch.cos((2.0 * math.pi) * u2)
+        out[s:s + c] = z.to(torch.float32).to(dtype)
+        del idx, x, u1, u2, z
+    return out.view(*shape)
