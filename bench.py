@@ -1,0 +1,530 @@
+#!/usr/bin/env python3
+"""Benchmark of the exact attention path on B200: one JSON line per run.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME|all] [--impl ours|reference]
+
+A step is one call of the library on one batch of synthetic input (iid N(0,1), seeded,
+counter-based generator in ``synth``), with the inputs resident in HBM.  The headline workload
+is causal self-attention prefill, B=4, Hq=Hkv=16, n=2048, d=128, bf16 (fp32 accumulate); the
+same line carries the split-K decode workload (64 sequences x 1 token, Hq=32, Hkv=8, 32768
+cached keys) under "decode", because the metric names both.
+
+Timing: W warm-up steps, then K timed steps; before every timed step a 256 MiB buffer is
+written (more than the 126 MB L2) and the step itself is bracketed by CUDA events on the
+launching stream; ``ms_per_step`` is the mean of the K event intervals.  With N > 1 (torchrun,
+one process per GPU) every rank runs its own replica of the workload on its own GPU (weak
+scaling: independent batches, no data-path collective), the ranks meet at a barrier before and
+after the timed loop, and the slowest rank's time sets the whole-job throughput.
+
+``--impl reference`` times the fp64 CPU oracle (the repository's reference implementation of
+the same operation) on bounded samples of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s & % BF16 TC peak (prefill); decode HBM GB/s & % peak"
+FULL, CAUSAL, SLIDING = 0, 1, 2
+MASK_NAMES = {FULL: "full", CAUSAL: "causal", SLIDING: "sliding"}
+
+WORKLOADS = {
+    "full_b1_h1_n256_d64_f32": dict(kind="fwd_f32", B=1, Hq=1, Hkv=1, N=256, d=64, mask=FULL,
+                                    window=0, n_sink=0, seed=1),
+    "causal_b4_h16_n2048_d128": dict(kind="fwd", B=4, Hq=16, Hkv=16, N=2048, d=128,
+                                     mask=CAUSAL, window=0, n_sink=0, seed=2),
+    "gqa_causal_b2_h32_kv8_n8192_d128": dict(kind="fwd", B=2, Hq=32, Hkv=8, N=8192, d=128,
+                                             mask=CAUSAL, window=0, n_sink=0, seed=3),
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": dict(kind="fwd", B=1, Hq=32, Hkv=8, N=32768,
+                                                    d=128, mask=SLIDING, window=4096, n_sink=4,
+                                                    seed=4),
+    "decode_b64_h32_kv8_n32768_d128": dict(kind="decode", B=64, Hq=32, Hkv=8, N=32768, d=128,
+                                           mask=FULL, window=0, n_sink=0, seed=5),
+}
+HEADLINE = "causal_b4_h16_n2048_d128"
+DECODE = "decode_b64_h32_kv8_n32768_d128"
+
+# DRAM traffic per launch of each workload's dominant kernel, from one ncu capture
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel sources the
+# capture was taken with; reported as null once the sources differ.
+NCU_TRAFFIC = {}
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_82_b200", "csrc")
+    for dirpath, _, files in sorted(os.walk(csrc)):
+        for f in sorted(files):
+            if f.endswith((".cu", ".cuh")):
+                with open(os.path.join(dirpath, f), "rb") as fh:
+                    h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            p = json.load(fh)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------------------------
+# work accounting
+# ----------------------------------------------------------------------------------------------
+def work_of(w):
+    from exact_io_aware_82_b200 import accounting as acc
+
+    if w["kind"] == "decode":
+        return acc.decode_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"]), "GB/s", 1e9
+    fl = acc.attn_flops(w["B"], w["Hq"], w["N"], w["N"], w["d"], w["mask"], w["window"],
+                        w["n_sink"])
+    return fl, "TFLOP/s", 1e12
+
+
+def config_of(name, w, n_gpus):
+    c = {"workload": name, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "d": w["d"],
+         "mask": MASK_NAMES[w["mask"]]}
+    if w["kind"] == "decode":
+        c.update({"q_tokens": 1, "kv_len": w["N"]})
+    else:
+        c.update({"n": w["N"]})
+    if w["mask"] == SLIDING:
+        c.update({"window": w["window"], "n_sink": w["n_sink"]})
+    c["inputs"] = "fp32" if w["kind"] == "fwd_f32" else "bf16"
+    c["l2"] = "flushed before every timed step (256 MiB write)"
+    c["parallelism"] = "replicas x%d (independent batch per GPU, no collective)" % n_gpus
+    return c
+
+
+# ----------------------------------------------------------------------------------------------
+# clock sampling (NVML, read-only) during the timed region
+# ----------------------------------------------------------------------------------------------
+_REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index, interval_s=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.interval = interval_s
+        self.ok = False
+        try:
+            import pynvml
+
+            import torch
+
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    handle = h
+            if handle is None:
+                handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.h = pynvml, handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = repr(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nvml.nvmlDeviceGetClockInfo(self.h, self.nvml.NVML_CLOCK_SM))
+                bits = self.nvml.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, n in _REASON_BITS.items():
+                    if bits & b:
+                        self.reasons.add(n)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.interval)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t is not None:
+            self._stop.set()
+            self._t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+                "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------------------------
+class Workload:
+    """Device buffers and the step function of one workload on the current GPU."""
+
+    def __init__(self, name, rank):
+        import torch
+
+        import synth
+        from exact_io_aware_82_b200 import attn as A
+
+        self.name, self.w = name, WORKLOADS[name]
+        w = self.w
+        self.A = A
+        seed = w["seed"] + 1000 * rank
+        dt = torch.float32 if w["kind"] == "fwd_f32" else torch.bfloat16
+        nq = 1 if w["kind"] == "decode" else w["N"]
+        self.q = synth.normal_torch(seed, synth.Q_ID, (w["B"], w["Hq"], nq, w["d"]), dt, "cuda")
+        self.k = synth.normal_torch(seed, synth.K_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
+        self.v = synth.normal_torch(seed, synth.V_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
+        self.o = torch.empty_like(self.q)
+        lse_shape = (w["B"], w["Hq"]) if w["kind"] == "decode" else (w["B"], w["Hq"], nq)
+        self.lse = torch.empty(lse_shape, dtype=torch.float32, device="cuda")
+        self.ws = None
+        if w["kind"] == "decode":
+            nb = A.attn_decode_workspace_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], 0)
+            self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
+        self.launches_per_step = 2 if w["kind"] == "decode" else 1
+
+    def run(self, q=None, k=None, v=None, o=None, lse=None):
+        w, A = self.w, self.A
+        q = self.q if q is None else q
+        k = self.k if k is None else k
+        v = self.v if v is None else v
+        o = self.o if o is None else o
+        lse = self.lse if lse is None else lse
+        if w["kind"] == "decode":
+            A.attn_decode(q, k, v, o=o, lse=lse, workspace=self.ws)
+        elif w["kind"] == "fwd_f32":
+            A.attn_fwd_f32(q, k, v, o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
+                           n_sink=w["n_sink"])
+        else:
+            A.attn_fwd(q, k, v, o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
+                       n_sink=w["n_sink"])
+
+
+def timed_loop(fn, steps, warmup, flush, dist_on, sampler=None):
+    """W warm-ups, then K steps each bracketed by CUDA events, with an L2 flush before each."""
+    import torch
+
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    ctx = sampler if sampler is not None else _Null()
+    with ctx:
+        for s, e in ev:
+            flush.zero_()
+            s.record(stream)
+            fn()
+            e.record(stream)
+        torch.cuda.synchronize()
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+    return [s.elapsed_time(e) for s, e in ev]
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def max_over_ranks(x, dist_on):
+    if not dist_on:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_kind):
+    import torch
+
+    wl = Workload(name, rank)
+    w = wl.w
+    work, unit, scale = work_of(w)
+    A = wl.A
+    sampler = ClockSampler(torch.cuda.current_device())
+    times = timed_loop(wl.run, steps, warmup, flush, dist_on, sampler)
+    err = A.attn_get_device_error()
+    if err != 0:
+        raise RuntimeError("device error flag set after the timed loop: %d" % err)
+    total_ms = max_over_ranks(sum(times), dist_on)
+    ms_per_step = total_ms / steps
+    value = world * work * steps / (total_ms * 1e-3) / scale
+
+    # roofline of the dominant kernel: algorithmic work per launch / mean launch duration
+    mean_ms = sum(times) / len(times)
+    achieved = work / (mean_ms * 1e-3) / scale
+    if w["kind"] == "decode":
+        bound, peak, punit = "hbm", peaks["hbm_gbs"], "GB/s"
+    else:
+        bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        if w["kind"] == "fwd_f32":
+            bound, peak = "fp32-fma", None
+    tr = NCU_TRAFFIC.get(name)
+    traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash() else None
+    roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
+            "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic,
+            "peak_source": peak_kind + (" burst" if bound == "tensor" else "")}
+
+    # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
+    qh = wl.q.cpu().pin_memory()
+    kh = wl.k.cpu().pin_memory()
+    vh = wl.v.cpu().pin_memory()
+    oh = torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory()
+    lh = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+    qd, kd, vd = torch.empty_like(wl.q), torch.empty_like(wl.k), torch.empty_like(wl.v)
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        wl.run(qd, kd, vd)
+        oh.copy_(wl.o, non_blocking=True)
+        lh.copy_(wl.lse, non_blocking=True)
+
+    e2e_times = timed_loop(e2e_step, max(3, min(steps, 20)), 2, flush, dist_on)
+    e2e_ms = max_over_ranks(sum(e2e_times), dist_on) / len(e2e_times)
+    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    e2e = {"value": round(world * work / (e2e_ms * 1e-3) / scale, 3), "unit": unit,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": round(e2e_ms, 4)}
+    del qh, kh, vh, qd, kd, vd
+    return dict(wl=wl, work=work, unit=unit, value=value, ms_per_step=ms_per_step,
+                roofline=roof, e2e=e2e, clocks=sampler.report(),
+                launches=wl.launches_per_step * steps)
+
+
+# ----------------------------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and the reference arm)
+# ----------------------------------------------------------------------------------------------
+def oracle_sample(name, budget_s, seed=0, host=None):
+    """Time the fp64 oracle on a random sample of the workload's output rows (prefill) or
+    sequences (decode), growing the sample until it has run for about ``budget_s`` seconds.
+    Returns (work units done, seconds, cores, description)."""
+    import numpy as np
+
+    import synth
+    from exact_io_aware_82_b200 import accounting as acc
+    from oracle import oracle as O
+
+    w = WORKLOADS[name]
+    rng = np.random.default_rng(seed)
+    cores = O.num_threads()
+    d = w["d"]
+    scale = 1 / math.sqrt(d)
+    B, Hq, Hkv, N = w["B"], w["Hq"], w["Hkv"], w["N"]
+    G = Hq // Hkv
+
+    def draw(tid, shape):
+        if w["kind"] == "fwd_f32":
+            return synth.normal_f32(w["seed"], tid, shape).astype(np.float64)
+        return synth.bf16_bits_to_f32(synth.normal_bf16_bits(w["seed"], tid, shape)).astype(np.float64)
+
+    if w["kind"] == "decode":
+        # one sequence at a time: its query (Hq x d) against its own Hkv heads of the cache
+        done, secs, seqs = 0, 0.0, 0
+        qall = draw(synth.Q_ID, (B, Hq, 1, d))
+        while secs < budget_s and seqs < B:
+            b = int(rng.integers(0, B))
+            # draw only this sequence's cache slice: element indices of [b][:][:][:]
+            kk = _draw_slice(w, synth.K_ID, b, Hkv * N * d).reshape(1, Hkv, N, d)
+            vv = _draw_slice(w, synth.V_ID, b, Hkv * N * d).reshape(1, Hkv, N, d)
+            t0 = time.perf_counter()
+            O.attention(qall[b:b + 1], kk, vv, FULL, scale=scale)
+            secs += time.perf_counter() - t0
+            done += acc.decode_bytes(1, Hq, Hkv, N, d)
+            seqs += 1
+        return done, secs, cores, "%d of %d sequences (all %d heads, %d cached keys each)" % (
+            seqs, B, Hq, N)
+
+    q = draw(synth.Q_ID, (B, Hq, N, d)) if host is None else host[0]
+    k = draw(synth.K_ID, (B, Hkv, N, d)) if host is None else host[1]
+    v = draw(synth.V_ID, (B, Hkv, N, d)) if host is None else host[2]
+    total_rows = B * Hq * N
+    done_rows, secs, work = 0, 0.0, 0
+    batch = 64
+    while secs < budget_s and done_rows < total_rows:
+        rows = rng.integers(0, total_rows, size=batch)
+        t0 = time.perf_counter()
+        O.attention_rows(q, k, v, rows, w["mask"], w["window"], w["n_sink"], scale)
+        secs += time.perf_counter() - t0
+        i = rows % N
+        for r in i:
+            work += 4 * d * acc.visible_pairs(1, int(r) + 1, w["mask"], w["window"], w["n_sink"]) \
+                if w["mask"] != FULL else 4 * d * N
+        done_rows += batch
+        batch = min(batch * 2, 4096)
+    return work, secs, cores, "%d random output rows of %d (%.2f%%)" % (
+        done_rows, total_rows, 100.0 * done_rows / total_rows)
+
+
+def _draw_slice(w, tid, b, count):
+    """Elements [b * count, (b + 1) * count) of a tensor (one sequence's cache), as fp64."""
+    import numpy as np
+
+    import synth
+
+    x = synth._box_muller(synth.splitmix64_np(synth._keys(w["seed"], tid, b * count, count)))
+    bits = synth.f32_to_bf16_bits(x.astype(np.float32))
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def cpu_baseline(name, budget_s=12.0):
+    work, secs, cores, desc = oracle_sample(name, budget_s)
+    _, unit, scale = work_of(WORKLOADS[name])
+    return {"value": round(work / secs / scale, 6), "unit": unit, "cores": cores,
+            "kind": "oracle", "sample": desc + ", %.1f s" % secs}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    name = HEADLINE if args.workload in (None, "all") else args.workload
+    w = WORKLOADS[name]
+    _, unit, scale = work_of(w)
+    per_step = []
+    for i in range(args.warmup + args.steps):
+        work, secs, cores, desc = oracle_sample(name, 1.0, seed=i)
+        if i >= args.warmup:
+            per_step.append((work, secs))
+    work = sum(x for x, _ in per_step)
+    secs = sum(s for _, s in per_step)
+    value = work / secs / scale
+    line = {"metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * secs / len(per_step), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(name, w, 1), "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": cores,
+                             "kind": "oracle",
+                             "sample": "each step: random output rows or sequences of the "
+                                       "workload for about 1 s of oracle time"},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None, help="one of %s, or 'all'" % ", ".join(WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 runs under torch.distributed.run with N processes")
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (there is no CPU fallback)")
+    torch.cuda.set_device(local)
+    dist_on = world > 1
+    if dist_on:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    from exact_io_aware_82_b200 import build
+
+    if rank == 0:
+        build.build()
+    if dist_on:
+        torch.distributed.barrier()
+    peaks, peak_kind = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    names = list(WORKLOADS) if args.workload == "all" else [args.workload or HEADLINE]
+    for name in names:
+        r = measure_ours(name, args.steps, args.warmup, rank, world, dist_on, flush, peaks,
+                         peak_kind)
+        w = WORKLOADS[name]
+        line = {"metric": METRIC, "value": round(r["value"], 3), "unit": r["unit"],
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(r["ms_per_step"], 5), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32" if w["kind"] == "fwd_f32" else "bf16",
+                "data": "synthetic (iid N(0,1), seeded counter-based generator)",
+                "config": config_of(name, w, world), "roofline": r["roofline"], "e2e": r["e2e"],
+                "gpu_launches": r["launches"], "clocks": r["clocks"]}
+        del r["wl"]
+        if args.workload is None and name == HEADLINE:
+            d = measure_ours(DECODE, max(5, args.steps // 5), args.warmup, rank, world, dist_on,
+                             flush, peaks, peak_kind)
+            del d["wl"]
+            line["decode"] = {"workload": DECODE, "value": round(d["value"], 2), "unit": d["unit"],
+                              "ms_per_step": round(d["ms_per_step"], 4),
+                              "roofline": d["roofline"], "e2e": d["e2e"], "clocks": d["clocks"],
+                              "gpu_launches": d["launches"]}
+            line["gpu_launches"] += d["launches"]
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(name)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    if dist_on:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,10 +1,11 @@
 """Exact IO-aware attention for NVIDIA B200 (sm_100a).
 
-The compute lives in the CUDA library ``libattn.so`` built from ``csrc/``; ``attn`` is its thin
-ctypes binding.  Importing the package does not load the library; the first call does, and it
-raises if the library is missing or no CUDA device is present.
+The compute lives in the CUDA library ``libattn.so`` built from ``csrc/`` (``build.py``);
+``attn`` is its thin ctypes binding.  Importing the package does not load the library; the
+first call does, and raises if the library is missing or no sm_100 device is present.
 """
 
 from . import accounting  # noqa: F401
-
-__all__ = ["accounting"]
+from .attn import (MASK_CAUSAL, MASK_FULL, MASK_SLIDING, AttnError, attn_decode,  # noqa: F401
+                   attn_decode_num_splits, attn_decode_workspace_bytes, attn_fwd, attn_fwd_f32,
+                   attn_get_device_error)

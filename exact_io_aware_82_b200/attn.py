@@ -1,0 +1,194 @@
+"""Thin ctypes binding of libattn.so (the C ABI in include/attn.h).
+
+Argument marshalling only: torch tensors are checked for device, dtype and contiguity and
+passed as raw device pointers together with the current CUDA stream; every step of the
+computation runs in the library's kernels.  Output and workspace tensors the caller does not
+supply are allocated with torch (device memory is PyTorch's job here).  A non-zero status from
+the library raises ``AttnError`` with the library's own message.  There is no fallback: if the
+library is missing or no sm_100 device is present, calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+MASK_FULL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_CUDA = -3
+ATTN_ERR_WORKSPACE = -4
+ATTN_ERR_DEVICE_TIMEOUT = -5
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
+
+# every symbol include/attn.h declares
+EXPORTS = ("attn_abi_version", "attn_status_string", "attn_fwd", "attn_fwd_f32",
+           "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
+           "attn_get_device_error", "attn_debug_timeout_probe")
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+
+
+def lib():
+    """Load libattn.so once; raise if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libattn.so is missing (%s): build it with "
+                               "`python -m exact_io_aware_82_b200.build`" % LIB_PATH)
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.attn_abi_version.argtypes, L.attn_abi_version.restype = [], i
+        L.attn_status_string.argtypes, L.attn_status_string.restype = [i], ctypes.c_char_p
+        L.attn_fwd.argtypes = [vp] * 5 + [i] * 9 + [f, vp]
+        L.attn_fwd.restype = i
+        L.attn_fwd_f32.argtypes = [vp] * 5 + [i] * 9 + [f, vp]
+        L.attn_fwd_f32.restype = i
+        L.attn_decode_workspace_bytes.argtypes = [i] * 6
+        L.attn_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.attn_decode.argtypes = [vp] * 5 + [i] * 5 + [f, i, vp, ctypes.c_size_t, vp]
+        L.attn_decode.restype = i
+        L.attn_decode_num_splits.argtypes, L.attn_decode_num_splits.restype = [i] * 5, i
+        L.attn_get_device_error.argtypes, L.attn_get_device_error.restype = [vp], i
+        L.attn_debug_timeout_probe.argtypes = [ctypes.c_longlong, vp]
+        L.attn_debug_timeout_probe.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def abi_version() -> int:
+    return int(lib().attn_abi_version())
+
+
+def _stream_ptr(stream=None):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check(t, name, dtype, ndim):
+    import torch
+
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device.type != "cuda":
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if t.dim() != ndim or not t.is_contiguous():
+        raise ValueError("%s must be a contiguous %d-d tensor" % (name, ndim))
+
+
+def _raise(rc, where):
+    if rc != ATTN_OK:
+        raise AttnError(rc, where)
+
+
+def attn_fwd(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None,
+             return_lse=True, stream=None):
+    """Exact attention forward on bf16 tensors q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d].
+
+    Returns (o, lse) with o bf16 [B,Hq,Nq,d] and lse fp32 [B,Hq,Nq] (None if not requested).
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                        int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
+    _raise(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_f32(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None,
+                 return_lse=True, stream=None):
+    """Exact attention forward on fp32 tensors (same shapes and rules as attn_fwd)."""
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.float32, 4)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk,
+                            d, int(mask_kind), int(window), int(n_sink), scale,
+                            _stream_ptr(stream))
+    _raise(rc, "attn_fwd_f32")
+    return o, lse
+
+
+def attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits=0) -> int:
+    return int(lib().attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits))
+
+
+def attn_decode_num_splits(B, Hq, Hkv, Nk, d) -> int:
+    return int(lib().attn_decode_num_splits(B, Hq, Hkv, Nk, d))
+
+
+def attn_decode(q, k, v, o=None, lse=None, scale=None, num_splits=0, workspace=None,
+                return_lse=True, stream=None):
+    """Split-K decode: q [B,Hq,1,d] bf16 against the cache k/v [B,Hkv,Nk,d] bf16.
+
+    Returns (o [B,Hq,1,d] bf16, lse [B,Hq] fp32).  ``workspace`` (a uint8 CUDA tensor of at
+    least attn_decode_workspace_bytes(...) bytes) is allocated with torch when not given.
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk, d,
+                           scale, int(num_splits), _ptr(workspace), workspace.numel(),
+                           _stream_ptr(stream))
+    _raise(rc, "attn_decode")
+    return o, lse
+
+
+def attn_get_device_error(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device error flag (0 = none)."""
+    return int(lib().attn_get_device_error(_stream_ptr(stream)))
+
+
+def attn_debug_timeout_probe(limit_cycles: int, stream=None) -> None:
+    _raise(lib().attn_debug_timeout_probe(int(limit_cycles), _stream_ptr(stream)),
+           "attn_debug_timeout_probe")

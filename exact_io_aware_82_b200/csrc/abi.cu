@@ -1,0 +1,362 @@
+// C ABI of the exact attention library (declared in include/attn.h): argument validation,
+// device checks, TMA descriptor encoding and kernel launches.  No allocation happens here and
+// no pointer is kept after a call returns.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "fwd_f32.cuh"
+#include "fwd_sm100.cuh"
+
+namespace attn {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DeviceInfo {
+  bool probed = false;
+  bool sm100 = false;
+  int num_sms = 0;
+  bool fwd_configured = false;
+};
+
+std::mutex g_mutex;
+DeviceInfo g_devices[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// Looks up the current device once: compute capability 10.x and the SM count; raises the
+// dynamic shared memory limit of the tensor-core kernel on first use.
+int current_device(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceInfo& info = g_devices[dev];
+  if (!info.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    info.sm100 = (major == 10 && minor == 0);
+    info.num_sms = sms;
+    info.probed = true;
+  }
+  if (!info.sm100) return ATTN_ERR_UNSUPPORTED;
+  *out = &info;
+  return ATTN_OK;
+}
+
+int configure_fwd(DeviceInfo* info) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!info->fwd_configured) {
+    if (cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(fwd::kSmemBytes)) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    info->fwd_configured = true;
+  }
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return ATTN_ERR_CUDA;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Common argument rules of the forward entry points.
+int check_fwd_args(const void* q, const void* k, const void* v, const void* o, int B, int Hq,
+                   int Hkv, int Nq, int Nk, int mask_kind, int window, int n_sink, float scale) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_SLIDING) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_SLIDING && window < 1) return ATTN_ERR_INVALID_ARG;
+  if (n_sink < 0) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+MaskSpec make_mask(int mask_kind, int window, int n_sink, int Nk) {
+  MaskSpec m;
+  m.kind = mask_kind;
+  m.window = mask_kind == ATTN_MASK_SLIDING ? window : 0;
+  m.n_sink = mask_kind == ATTN_MASK_SLIDING ? n_sink : 0;
+  m.Nk = Nk;
+  return m;
+}
+
+// O = 0 and LSE = -inf for rows that can see no key at all (Nk = 0).
+template <typename T>
+__global__ void fill_empty_kernel(T* o, float* lse, size_t rows, int d) {
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (i < rows * d) o[i] = T(0.f);
+  if (lse != nullptr && i < rows) lse[i] = -INFINITY;
+}
+
+template <typename T>
+int launch_fill_empty(T* o, float* lse, size_t rows, int d, cudaStream_t stream) {
+  const size_t n = rows * static_cast<size_t>(d);
+  if (n == 0) return ATTN_OK;
+  const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
+  fill_empty_kernel<T><<<blocks, 256, 0, stream>>>(o, lse, rows, d);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x 128 rows,
+// 128-byte swizzle (the layout tcgen05.mma descriptors read).  Rows past `rows` read as zero.
+int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
+                                 static_cast<cuuint64_t>(rows) * fwd::kD * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+constexpr int kMaxSplits = 256;
+
+int decode_splits(int B, int Hkv, int Nk, int G, int requested, int num_sms) {
+  int max_chunk;
+  switch (G) {
+    case 1: max_chunk = dec::max_chunk<1>(); break;
+    case 2: max_chunk = dec::max_chunk<2>(); break;
+    case 4: max_chunk = dec::max_chunk<4>(); break;
+    default: max_chunk = dec::max_chunk<8>(); break;
+  }
+  const int min_splits = Nk > 0 ? (Nk + max_chunk - 1) / max_chunk : 1;
+  int s = requested;
+  if (s <= 0) {
+    // enough CTAs for several waves of 2 resident CTAs per SM, chunks of at most max_chunk
+    const int groups = B * Hkv > 0 ? B * Hkv : 1;
+    const int want = (4 * 2 * num_sms + groups - 1) / groups;
+    const int by_len = Nk > 0 ? (Nk + 255) / 256 : 1;  // at least 256 keys per split
+    s = want < by_len ? want : by_len;
+  }
+  if (s < min_splits) s = min_splits;
+  if (s < 1) s = 1;
+  if (s > kMaxSplits) s = kMaxSplits;
+  return s;
+}
+
+size_t decode_ws_bytes(int B, int Hq, int splits) {
+  const size_t rows = static_cast<size_t>(B) * Hq * splits;
+  return rows * dec::kD * sizeof(float) + ((rows * sizeof(float) + 15) & ~size_t(15));
+}
+
+template <int G>
+void launch_decode_split(dim3 grid, int chunk, cudaStream_t stream, const __nv_bfloat16* q,
+                         const __nv_bfloat16* k, const __nv_bfloat16* v, float* ws_o,
+                         float* ws_lse, int Hq, int Hkv, int Nk, int splits, float c) {
+  const size_t smem = static_cast<size_t>(dec::smem_floats(G, chunk)) * sizeof(float);
+  dec::decode_split_kernel<G><<<grid, dec::kThreads, smem, stream>>>(q, k, v, ws_o, ws_lse, Hq,
+                                                                      Hkv, Nk, chunk, splits, c);
+}
+
+__global__ void timeout_probe_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    dev::mbar_init(dev::smem_u32(&bar), 1);
+    abort_flag = 0;
+    dev::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) wait_bounded(dev::smem_u32(&bar), 0, &abort_flag, limit);
+  __syncthreads();
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (head dim, group size, alignment or device)";
+    case ATTN_ERR_CUDA: return "CUDA runtime error";
+    case ATTN_ERR_WORKSPACE: return "decode workspace missing or too small";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait expired";
+    default: return "unknown status";
+  }
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink, float scale,
+             attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  if (d != fwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Nk == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
+                             static_cast<size_t>(B) * Hq * Nq, d, st);
+  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
+
+  CUtensorMap tq, tk, tv;
+  if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  fwd::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.c = scale * kLog2e;
+  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  fwd::fwd_bf16_sm100_kernel<<<static_cast<unsigned>(units), fwd::kThreads, fwd::kSmemBytes, st>>>(
+      tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                 float scale, attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Nk == 0) return launch_fill_empty(o, lse, static_cast<size_t>(B) * Hq * Nq, d, st);
+  if (Hq > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  f32::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.c = scale * kLog2e;
+  if (d == 64) {
+    dim3 grid((Nq + f32::rows_per_cta<64>() - 1) / f32::rows_per_cta<64>(), Hq, B);
+    f32::fwd_f32_kernel<64><<<grid, f32::kWarps * 32, 0, st>>>(q, k, v, o, lse, p);
+  } else {
+    dim3 grid((Nq + f32::rows_per_cta<128>() - 1) / f32::rows_per_cta<128>(), Hq, B);
+    f32::fwd_f32_kernel<128><<<grid, f32::kWarps * 32, 0, st>>>(q, k, v, o, lse, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_decode_num_splits(int B, int Hq, int Hkv, int Nk, int d) {
+  (void)d;
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  const int num_sms = current_device(&info) == ATTN_OK ? info->num_sms : 148;
+  return decode_splits(B, Hkv, Nk, Hq / Hkv, 0, num_sms);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nk, int d, int num_splits) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Nk < 0 || d != dec::kD) return 0;
+  DeviceInfo* info = nullptr;
+  const int num_sms = current_device(&info) == ATTN_OK ? info->num_sms : 148;
+  const int splits = decode_splits(B, Hkv, Nk, Hq / Hkv, num_splits, num_sms);
+  return decode_ws_bytes(B, Hq, splits);
+}
+
+int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nk, int d, float scale, int num_splits, void* workspace,
+                size_t workspace_bytes, attn_stream_t stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (B < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 0 || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (d != dec::kD) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  int rc = current_device(&info);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0) return ATTN_OK;
+  if (Nk == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq, d, st);
+  if (B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  const int splits = decode_splits(B, Hkv, Nk, G, num_splits, info->num_sms);
+  const size_t need = decode_ws_bytes(B, Hq, splits);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    return ATTN_ERR_WORKSPACE;
+  const int chunk = (Nk + splits - 1) / splits;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_lse = ws_o + static_cast<size_t>(B) * Hq * splits * dec::kD;
+  const float c = scale * kLog2e;
+  const dim3 grid(splits, Hkv, B);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  switch (G) {
+    case 1: launch_decode_split<1>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
+    case 2: launch_decode_split<2>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
+    case 4: launch_decode_split<4>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
+    default: launch_decode_split<8>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(ws_o, ws_lse,
+                                                         static_cast<__nv_bfloat16*>(o), lse, splits);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+int attn_get_device_error(attn_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (flag != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    return flag;
+  }
+  return ATTN_OK;
+}
+
+int attn_debug_timeout_probe(long long limit_cycles, attn_stream_t stream) {
+  if (limit_cycles < 1 || limit_cycles > (1ll << 34)) return ATTN_ERR_INVALID_ARG;
+  DeviceInfo* info = nullptr;
+  int rc = current_device(&info);
+  if (rc != ATTN_OK) return rc;
+  timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // extern "C"

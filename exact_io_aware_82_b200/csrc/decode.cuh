@@ -1,0 +1,268 @@
+// Split-K decode: one new query token per sequence against a long, contiguous KV cache.
+//
+// "Attention Research" (learning-materials), section 1: decode reads the whole O(S) KV cache
+// every step, so it is bound by HBM bandwidth; section 2: FlashDecoding splits the keys of a
+// decode step across thread blocks ("split-K over keys").  Each split produces a partial
+// output normalised by its own softmax sum together with its log-sum-exp; the combine merges
+// the splits exactly, O = sum_s exp(lse_s - LSE) O_s with LSE = ln sum_s exp(lse_s), which is
+// the online-softmax rescaling of "FlashAttention and sparse attention" (grasp.study),
+// section 1, applied once per split.
+//
+// Split kernel: grid (splits, Hkv, B), 256 threads.  The G query heads of a kv group share
+// every K/V byte read.  A half-warp covers one 256-byte key (or value) row with 16-byte loads,
+// so every load instruction of a warp reads two whole rows (fully coalesced); thread lane%16
+// owns head-dimension slice [8*(lane%16), 8*(lane%16)+8) for the whole kernel and keeps the
+// matching slice of the G query vectors in registers.  Scores are finished with a
+// reduce-scatter across the 16 lanes of a row, written to shared memory, turned into
+// probabilities, and the value pass accumulates P V per slice; partial sums of the 16
+// half-warps are reduced through shared memory at the end.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace attn {
+namespace dec {
+
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxScoreFloats = 8192;  // per-CTA score buffer: chunk * G floats (32 KB)
+
+// keys each half-warp loads per pass iteration: U * G = 32 partial dot products per thread
+template <int G>
+__host__ __device__ constexpr int unroll() { return G == 1 ? 16 : 32 / G; }
+template <int G>
+__host__ __device__ constexpr int keys_per_iter() { return 2 * unroll<G>() * kWarps; }
+template <int G>
+__host__ __device__ constexpr int max_chunk() { return kMaxScoreFloats / G; }
+
+__host__ __device__ constexpr int smem_floats(int G, int chunk) {
+  return (chunk * G > kWarps * G * kD) ? chunk * G : kWarps * G * kD;
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads)
+    decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                        const __nv_bfloat16* __restrict__ v, float* __restrict__ ws_o,
+                        float* __restrict__ ws_lse, int Hq, int Hkv, int Nk, int chunk,
+                        int splits, float c) {
+  constexpr int U = unroll<G>();
+  constexpr int NV = U * G;        // partial dot products per thread per iteration
+  constexpr int PER_LANE = NV / 16;  // fully reduced scores each lane ends with
+  extern __shared__ float smem[];   // scores/probabilities [chunk][G], later the P V partials
+  __shared__ float red_m[kWarps][G];
+  __shared__ float stat[2][G];     // max (log2 units) and sum per head
+
+  const int s = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = lane >> 4, sl = lane & 15;
+  const int j0 = s * chunk;
+  const int n = max(0, min(Nk - j0, chunk));
+  const size_t kv_base = (static_cast<size_t>(b) * Hkv + hk) * Nk;
+  const __nv_bfloat16* kb = k + (kv_base + j0) * kD + 8 * sl;
+  const __nv_bfloat16* vb = v + (kv_base + j0) * kD + 8 * sl;
+
+  // this thread's slice of the G query vectors, pre-multiplied by scale * log2(e)
+  float qf[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const uint4 u = *reinterpret_cast<const uint4*>(
+        q + (static_cast<size_t>(b) * Hq + hk * G + g) * kD + 8 * sl);
+    bf16x8_to_f32(u, qf[g]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qf[g][e] *= c;
+  }
+
+  // ---------------- pass 1: scores (log2 units) into shared memory ----------------
+  for (int base = 0; base < n; base += keys_per_iter<G>()) {
+    const int kw = base + warp * 2 * U;  // first key of this warp's group
+    uint4 kr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int key = kw + 2 * u + half;
+      kr[u] = key < n ? ldg_stream(kb + static_cast<size_t>(key) * kD) : make_uint4(0, 0, 0, 0);
+    }
+    float part[NV];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float kf[8];
+      bf16x8_to_f32(kr[u], kf);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc = fmaf(qf[g][e], kf[e], acc);
+        part[u * G + g] = acc;
+      }
+    }
+    // reduce-scatter over the 16 lanes of each row: after the step with lane bit m, a lane
+    // keeps the half of the vector selected by that bit; a lane ends with entries
+    // 2*sl*PER_LANE/2 ... i.e. indices [sl * PER_LANE, sl * PER_LANE + PER_LANE)
+#pragma unroll
+    for (int m = 8, width = NV; m >= 1; m >>= 1, width >>= 1) {
+      const bool upper = (sl & m) != 0;
+#pragma unroll
+      for (int i = 0; i < width / 2; ++i) {
+        const float lo = part[i], hi = part[i + width / 2];
+        const float send = upper ? lo : hi;
+        const float keep = upper ? hi : lo;
+        part[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < PER_LANE; ++i) {
+      const int idx = sl * PER_LANE + i;  // = u * G + g
+      const int u = idx / G, g = idx % G;
+      const int key = kw + 2 * u + half;
+      if (key < n) smem[key * G + g] = part[i];
+    }
+  }
+  __syncthreads();
+
+  // ---------------- softmax statistics per head ----------------
+  float mx[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
+  for (int key = tid; key < n; key += kThreads)
+#pragma unroll
+    for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], smem[key * G + g]);
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) mx[g] = fmaxf(mx[g], __shfl_xor_sync(0xffffffffu, mx[g], sh));
+    if (lane == 0) red_m[warp][g] = mx[g];
+  }
+  __syncthreads();
+  if (tid < G) {
+    float m = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) m = fmaxf(m, red_m[w][tid]);
+    stat[0][tid] = m;
+  }
+  __syncthreads();
+  float sum[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    mx[g] = stat[0][g];
+    sum[g] = 0.f;
+  }
+  for (int key = tid; key < n; key += kThreads)
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float pr = exp2f(smem[key * G + g] - mx[g]);
+      smem[key * G + g] = pr;
+      sum[g] += pr;
+    }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int sh = 16; sh > 0; sh >>= 1) sum[g] += __shfl_xor_sync(0xffffffffu, sum[g], sh);
+  }
+  __syncthreads();  // every thread has read red_m; reuse it for the sums
+  if (lane == 0)
+#pragma unroll
+    for (int g = 0; g < G; ++g) red_m[warp][g] = sum[g];
+  __syncthreads();
+  if (tid < G) {
+    float t = 0.f;
+    for (int w = 0; w < kWarps; ++w) t += red_m[w][tid];
+    stat[1][tid] = t;
+  }
+
+  // ---------------- pass 2: O_s = sum_j p_j V_j per head-dimension slice ----------------
+  float acc[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] = 0.f;
+  for (int base = 0; base < n; base += keys_per_iter<G>()) {
+    const int kw = base + warp * 2 * U;
+    uint4 vr[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int key = kw + 2 * u + half;
+      vr[u] = key < n ? ldg_stream(vb + static_cast<size_t>(key) * kD) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int key = kw + 2 * u + half;
+      if (key < n) {
+        float vf[8];
+        bf16x8_to_f32(vr[u], vf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = smem[key * G + g];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[g][e] = fmaf(pr, vf[e], acc[g][e]);
+        }
+      }
+    }
+  }
+  // combine the two half-warps, then the 8 warps through shared memory
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[g][e] += __shfl_xor_sync(0xffffffffu, acc[g][e], 16);
+  __syncthreads();  // all probabilities consumed; the score buffer becomes the partial buffer
+  if (half == 0)
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) smem[(warp * G + g) * kD + 8 * sl + e] = acc[g][e];
+  __syncthreads();
+  for (int idx = tid; idx < G * kD; idx += kThreads) {
+    const int g = idx / kD, dcol = idx % kD;
+    float t = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) t += smem[(w * G + g) * kD + dcol];
+    const float l = stat[1][g];
+    const size_t row = (static_cast<size_t>(b) * Hq + hk * G + g) * splits + s;
+    ws_o[row * kD + dcol] = l > 0.f ? t / l : 0.f;
+    if (dcol == 0)
+      ws_lse[row] = l > 0.f ? (stat[0][g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+// Combine: grid B * Hq, one thread per head-dimension column.
+__global__ void __launch_bounds__(kD)
+    decode_combine_kernel(const float* __restrict__ ws_o, const float* __restrict__ ws_lse,
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, int splits) {
+  const int bh = blockIdx.x, dcol = threadIdx.x;
+  const float* L = ws_lse + static_cast<size_t>(bh) * splits;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, L[s]);
+  float out = 0.f, tot = -INFINITY;
+  if (M != -INFINITY) {
+    float z = 0.f;
+    for (int s = 0; s < splits; ++s) z += expf(L[s] - M);
+    tot = M + logf(z);
+    const float* Os = ws_o + static_cast<size_t>(bh) * splits * kD + dcol;
+    for (int s = 0; s < splits; ++s) {
+      const float w = expf(L[s] - tot);
+      out = fmaf(w, Os[static_cast<size_t>(s) * kD], out);
+    }
+  }
+  o[static_cast<size_t>(bh) * kD + dcol] = __float2bfloat16_rn(out);
+  if (dcol == 0 && lse != nullptr) lse[bh] = tot;
+}
+
+}  // namespace dec
+}  // namespace attn

@@ -1,0 +1,388 @@
+// bf16 exact attention forward for sm_100a: TMA -> shared memory -> tcgen05.mma (TMEM
+// accumulators) -> online softmax in registers -> P back to TMEM -> tcgen05.mma for P V.
+//
+// The method: "FlashAttention and sparse attention" (grasp.study), section 1 (tiling, kernel
+// fusion, online softmax: running max and running sum, earlier partial results rescaled when
+// the max grows); "Chapter 3.1 - The Cost of Attention" (llmis.ru), sections 5 and 6 (the score
+// matrix never reaches HBM; work partitioned across thread blocks and warps); "Attention
+// Research" (learning-materials), section 2 (TMA and warp specialisation as in
+// FlashAttention-3, here re-expressed with tcgen05 and tensor memory).
+//
+// One CTA computes 256 query rows of one (batch, query head) as two 128-row tiles Q0, Q1 that
+// share every K/V tile.  Warp roles (14 warps, 448 threads):
+//   warps 0-3   softmax + epilogue for Q0 (thread t owns row t, TMEM lanes 0-127)
+//   warps 4-7   softmax + epilogue for Q1
+//   warps 8-11  idle after set-up (kept so the MMA and load warps are not in a softmax warpgroup)
+//   warp 12     TMEM allocation and the single-thread tcgen05.mma issuer
+//   warp 13     TMA producer (Q once, then K_j and V_j through two 2-stage rings)
+// Tensor memory (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 [256,384)
+// O1 [384,512).  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
+// MMA issue order per key tile j (ping-pong between the two query tiles):
+//   PV0(j), S0(j+1), PV1(j), S1(j+1)
+// so the tensor core computes one tile while the other tile's softmax runs.  tcgen05.mma
+// executes in issue order, so S_t(j+1) never overwrites P_t(j) before PV_t(j) has read it, and
+// the commit that signals S_t(j+1) also covers PV_t(j): the softmax may then rescale O_t.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace attn {
+namespace fwd {
+
+constexpr int kBM = 128;             // query rows per tile
+constexpr int kBN = 128;             // keys per tile
+constexpr int kD = 128;              // head dimension
+constexpr int kRowsPerCta = 2 * kBM;
+constexpr int kThreads = 448;
+constexpr uint32_t kTileBytes = kBM * kD * 2;  // 32 KB, bf16
+constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column half
+constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
+
+struct Params {
+  int B, Hq, Hkv, Nq, Nk, G;
+  MaskSpec mask;
+  float c;  // scale * log2(e): scores are handled in log2 units
+  int num_qblocks;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+struct __align__(1024) Smem {
+  uint8_t q[2][kTileBytes];
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
+  uint64_t bar_q;
+  uint64_t bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
+  uint64_t bar_s[2], bar_p[2], bar_o[2], bar_drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base to 1024 B
+
+// Is every (row, key) of the 128x128 block of query tile rows [P0, P0+127] x keys of tile kt
+// visible?  Conservative (uses all 128 rows even past Nq).
+__device__ __forceinline__ bool tile_is_full(const MaskSpec& m, int P0, int kt) {
+  const int c0 = kt * kBN, c1 = c0 + kBN - 1, P1 = P0 + kBM - 1;
+  if (c1 >= m.Nk) return false;
+  if (m.kind == ATTN_MASK_FULL) return true;
+  if (c1 > P0) return false;
+  if (m.kind == ATTN_MASK_CAUSAL) return true;
+  return (c0 > P1 - m.window) || (c1 < m.n_sink);
+}
+
+__device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                      ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+
+  // ---- work unit: heaviest query blocks first (causal), the G heads of a kv head adjacent ----
+  const int nbh = p.B * p.Hq;
+  const int unit = blockIdx.x;
+  const int qb = p.num_qblocks - 1 - unit / nbh;
+  const int bh = unit % nbh;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int bkv = b * p.Hkv + h / p.G;
+  const int r0 = qb * kRowsPerCta;
+  const int off = p.Nk - p.Nq;
+  const int last_row = min(r0 + kRowsPerCta, p.Nq) - 1;
+  const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kBN);
+  const int nk = tr.count();
+
+  // ---- set-up ----
+  if (tid == 0) {
+    dev::mbar_init(dev::smem_u32(&sm.bar_q), 1);
+    for (int s = 0; s < 2; ++s) {
+      dev::mbar_init(dev::smem_u32(&sm.bar_kfull[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_kempty[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_vfull[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_vempty[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kBM);
+      dev::mbar_init(dev::smem_u32(&sm.bar_o[s]), 1);
+    }
+    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
+    sm.abort = 0;
+    dev::fence_barrier_init();
+  }
+  if (warp == 13 && lane == 0) {
+    dev::tma_prefetch_desc(&tm_q);
+    dev::tma_prefetch_desc(&tm_k);
+    dev::tma_prefetch_desc(&tm_v);
+  }
+  if (warp == 12) {
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == 13) {
+    // =============================== TMA producer ===============================
+    if (lane == 0) {
+      int k_issued = 0, v_issued = 0;
+      bool q_issued = false;
+      if (nk > 0) {
+        const uint32_t bq = dev::smem_u32(&sm.bar_q);
+        dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int half = 0; half < 2; ++half)
+            dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
+                             r0 + t * kBM, bh);
+        q_issued = true;
+        for (int j = 0; j < nk; ++j) {
+          const int kt = tr.tile(j);
+          const int s = j & 1;
+          const uint32_t ph = ((j >> 1) & 1) ^ 1;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_kempty[s]), ph, abort)) break;
+          const uint32_t bk = dev::smem_u32(&sm.bar_kfull[s]);
+          dev::mbar_arrive_expect_tx(bk, kTileBytes);
+          for (int half = 0; half < 2; ++half)
+            dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
+                             kt * kBN, bkv);
+          ++k_issued;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_vempty[s]), ph, abort)) break;
+          const uint32_t bv = dev::smem_u32(&sm.bar_vfull[s]);
+          dev::mbar_arrive_expect_tx(bv, kTileBytes);
+          for (int half = 0; half < 2; ++half)
+            dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
+                             kt * kBN, bkv);
+          ++v_issued;
+        }
+      }
+      // ---- drain: wait until every copy this thread started has landed ----
+      if (q_issued) wait_drain(dev::smem_u32(&sm.bar_q), 0);
+      for (int s = 0; s < 2; ++s) {
+        // the last load into stage s among loads 0..n-1 is u = largest u < n with u % 2 == s;
+        // it completed phase (u / 2) of that stage's full barrier
+        const int uk = (k_issued - 1 - s) >= 0 ? ((k_issued - 1 - s) & ~1) + s : -1;
+        if (uk >= 0) wait_drain(dev::smem_u32(&sm.bar_kfull[s]), (uk >> 1) & 1);
+        const int uv = (v_issued - 1 - s) >= 0 ? ((v_issued - 1 - s) & ~1) + s : -1;
+        if (uv >= 0) wait_drain(dev::smem_u32(&sm.bar_vfull[s]), (uv >> 1) & 1);
+      }
+    }
+  } else if (warp == 12) {
+    // ============================ tcgen05.mma issuer =============================
+    if (lane == 0 && nk > 0) {
+      constexpr uint32_t idesc_s = dev::idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
+      constexpr uint32_t idesc_o = dev::idesc_bf16_f32(kBM, kD, 0, 1);   // P (TMEM), V MN-major
+      const uint32_t q_base[2] = {dev::smem_u32(sm.q[0]), dev::smem_u32(sm.q[1])};
+      const uint32_t tm_s[2] = {tmem + 0, tmem + 128};
+      const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
+
+      auto issue_s = [&](int t, int s) {
+        const uint32_t kb = dev::smem_u32(sm.k[s]);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t koff = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
+          const uint64_t a = dev::smem_desc(q_base[t] + koff, 16, 1024, dev::kSwizzle128B);
+          const uint64_t bdesc = dev::smem_desc(kb + koff, 16, 1024, dev::kSwizzle128B);
+          dev::umma_ss(tm_s[t], a, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t vb = dev::smem_u32(sm.v[s]);
+#pragma unroll
+        for (int ks = 0; ks < kBN / 16; ++ks) {
+          const uint64_t bdesc =
+              dev::smem_desc(vb + ks * 16 * 128, kHalfBytes, 1024, dev::kSwizzle128B);
+          dev::umma_ts(tm_o[t], tm_s[t] + ks * 8, bdesc, idesc_o, (acc || ks > 0) ? 1u : 0u);
+        }
+      };
+
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
+      if (ok) ok = wait_bounded(dev::smem_u32(&sm.bar_kfull[0]), 0, abort);
+      if (ok) {
+        dev::tc_fence_after();
+        issue_s(0, 0);
+        dev::umma_commit(dev::smem_u32(&sm.bar_s[0]));
+        issue_s(1, 0);
+        dev::umma_commit(dev::smem_u32(&sm.bar_s[1]));
+        dev::umma_commit(dev::smem_u32(&sm.bar_kempty[0]));
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const bool more = j + 1 < nk;
+        const int s1 = (j + 1) & 1;
+        const uint32_t ph1 = ((j + 1) >> 1) & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_vfull[s]), ph, abort))) break;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[0]), j & 1, abort))) break;
+        dev::tc_fence_after();
+        issue_pv(0, s, j > 0);
+        if (more) {
+          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_kfull[s1]), ph1, abort))) break;
+          dev::tc_fence_after();
+          issue_s(0, s1);
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[0]));
+        } else {
+          dev::umma_commit(dev::smem_u32(&sm.bar_o[0]));
+        }
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[1]), j & 1, abort))) break;
+        dev::tc_fence_after();
+        issue_pv(1, s, j > 0);
+        dev::umma_commit(dev::smem_u32(&sm.bar_vempty[s]));
+        if (more) {
+          issue_s(1, s1);
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[1]));
+          dev::umma_commit(dev::smem_u32(&sm.bar_kempty[s1]));
+        } else {
+          dev::umma_commit(dev::smem_u32(&sm.bar_o[1]));
+        }
+      }
+      // drain: every MMA issued above has completed once this commit arrives
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
+      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+    }
+  } else if (warp < 8) {
+    // ====================== softmax + epilogue (one row per thread) ======================
+    const int t = warp >> 2;            // query tile of this warpgroup
+    const int row = tid & 127;          // row inside the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem + lane_off + t * 128;
+    const uint32_t t_o = tmem + lane_off + 256 + t * 128;
+    const int P0 = r0 + t * kBM + off;  // key position of the tile's first row
+    const int prow = P0 + row;          // key position of this thread's row
+    const float c = p.c;
+    float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
+    float l = 0.f;            // running sum of exp2(s*c - m_ref)
+    bool ok = true;
+
+    for (int j = 0; j < nk; ++j) {
+      ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), j & 1, abort);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      dev::tc_fence_after();
+      const int kt = tr.tile(j);
+      const int key0 = kt * kBN;
+      const bool full = tile_is_full(p.mask, P0, kt);
+
+      // pass 1: row max of the (masked) scores of this tile
+      float mx = neg_inf();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        dev::tmem_ld32(t_s + cc * 32, r);
+        dev::tmem_wait_ld();
+        if (full) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[e]) * c);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float x = key_visible(p.mask, prow, key0 + cc * 32 + e)
+                                ? __uint_as_float(r[e]) * c
+                                : neg_inf();
+            mx = fmaxf(mx, x);
+          }
+        }
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      float alpha = 1.f;
+      if (m_new > m_ref + kRescaleThreshold) {
+        alpha = dev::ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
+        m_ref = m_new;
+      }
+      l *= alpha;
+      const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
+
+      // rescale the running output O_t (complete: the commit for S_t(j) covered PV_t(j-1))
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t r[32];
+          dev::tmem_ld32(t_o + cc * 32, r);
+          dev::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          dev::tmem_st32(t_o + cc * 32, r);
+        }
+      }
+
+      // pass 2: P = exp2(s*c - m_use) -> bf16, written over the consumed S columns
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        dev::tmem_ld32(t_s + cc * 32, r);
+        dev::tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[e]), c, -m_use));
+          float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[e + 1]), c, -m_use));
+          if (!full) {
+            if (!key_visible(p.mask, prow, key0 + cc * 32 + e)) p0 = 0.f;
+            if (!key_visible(p.mask, prow, key0 + cc * 32 + e + 1)) p1 = 0.f;
+          }
+          l += p0 + p1;
+          pk[e >> 1] = dev::pack_bf16x2(p0, p1);
+        }
+        dev::tmem_st16(t_s + cc * 16, pk);
+      }
+      dev::tmem_wait_st();
+      dev::tc_fence_before();
+      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));
+    }
+
+    // ---- epilogue: O = O / l in bf16, LSE = ln(sum exp(scale * s)) ----
+    if (ok && nk > 0) ok = wait_bounded(dev::smem_u32(&sm.bar_o[t]), 0, abort);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      dev::tc_fence_after();
+      const int grow = r0 + t * kBM + row;
+      const bool valid = grow < p.Nq;
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.Nq + grow) * kD);
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t r[32];
+        if (nk > 0) {
+          dev::tmem_ld32(t_o + cc * 32, r);
+          dev::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = 0u;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2)
+          pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(r[e]) * inv_l,
+                                        __uint_as_float(r[e + 1]) * inv_l);
+        if (valid) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      if (valid && p.lse != nullptr) {
+        const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
+        p.lse[static_cast<size_t>(bh) * p.Nq + grow] =
+            l > 0.f ? (m_use + log2f(l)) * 0.69314718055994531f : neg_inf();
+      }
+    }
+  }
+
+  // ---- teardown ----
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == 12) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace fwd
+}  // namespace attn

@@ -1,0 +1,136 @@
+/*
+ * attn.h - C ABI of the exact IO-aware attention library for NVIDIA B200 (sm_100a).
+ *
+ * Operation (all entry points): for every batch b, query head h and query row i,
+ *
+ *     O[b,h,i,:]  = sum_j P_ij V[b,hk,j,:],   P_ij = exp(s_ij) / sum_{visible j'} exp(s_ij'),
+ *     s_ij        = scale * Q[b,h,i,:] . K[b,hk,j,:]   over the keys j visible to row i,
+ *     LSE[b,h,i]  = ln sum_{visible j} exp(s_ij)       (natural log),
+ *
+ * i.e. scaled dot-product attention softmax(Q K^T / sqrt(d)) V with Q, K, V of shape (n, d)
+ * ("Chapter 3.1 - The Cost of Attention", section 2), computed exactly, FlashAttention-style:
+ * Q/K/V tiles pass through on-chip memory and an online (running max / running sum) softmax
+ * is used, so the n x n score matrix never reaches HBM ("FlashAttention and sparse
+ * attention", section 1: tiling, kernel fusion and online softmax; same page as above,
+ * section 5).
+ *
+ * Masks (mask_kind), with p_i = i + Nk - Nq the key position of query row i (bottom-right
+ * alignment when Nq != Nk):
+ *   ATTN_MASK_FULL     every key visible;
+ *   ATTN_MASK_CAUSAL   key j visible iff j <= p_i;
+ *   ATTN_MASK_SLIDING  causal, and (p_i - window < j  or  j < n_sink): a left window of `window`
+ *                      keys including the diagonal ("Quadratic Complexity Bottleneck",
+ *                      sliding-window attention) plus n_sink always-visible sink tokens at key
+ *                      positions 0..n_sink-1 ("Attention Research", section 4).
+ * Rows with no visible key get O = 0 and LSE = -inf.
+ * GQA ("Quadratic Complexity Bottleneck", grouped-query attention): Hq = G * Hkv and query head
+ * h reads kv head hk = h / G (contiguous groups); Hkv = 1 is multi-query attention.
+ *
+ * Layouts: contiguous, row-major, head dimension innermost.
+ *   Q, O  [B][Hq][Nq][d]      K, V  [B][Hkv][Nk][d]      LSE  [B][Hq][Nq] fp32
+ *
+ * Ownership and execution: every pointer is a DEVICE pointer owned by the caller; the library
+ * never allocates, frees or keeps a pointer after the call returns.  Calls only enqueue work
+ * on `stream` (asynchronous, reentrant); results are valid once the stream reaches them.
+ * No CPU fallback exists: without an sm_100 device a call returns ATTN_ERR_UNSUPPORTED.
+ *
+ * Errors: a call that returns non-zero has launched nothing (except ATTN_ERR_CUDA, returned
+ * when a launch itself failed).  Device-side waits are bounded; if one expires the kernel
+ * stops early, records the event in a device flag and `attn_get_device_error` reports
+ * ATTN_ERR_DEVICE_TIMEOUT after the stream has been synchronised.
+ */
+#ifndef EXACT_ATTN_B200_ATTN_H
+#define EXACT_ATTN_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t (NULL = the legacy default stream). */
+typedef struct CUstream_st *attn_stream_t;
+
+enum attn_mask_kind { ATTN_MASK_FULL = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_SLIDING = 2 };
+
+enum attn_status {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,    /* null pointer, negative size, Hq % Hkv != 0, bad mask, ... */
+  ATTN_ERR_UNSUPPORTED = -2,    /* head dim, group size, alignment or device not supported */
+  ATTN_ERR_CUDA = -3,           /* a CUDA runtime call or launch failed */
+  ATTN_ERR_WORKSPACE = -4,      /* decode workspace missing or too small */
+  ATTN_ERR_DEVICE_TIMEOUT = -5  /* a bounded device-side wait expired (see attn_get_device_error) */
+};
+
+/* Version of this ABI (bumped on any incompatible change). */
+ATTN_API int attn_abi_version(void);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+ATTN_API const char *attn_status_string(int status);
+
+/*
+ * attn_fwd - bf16 prefill / full forward.
+ *   q, o   bf16 [B][Hq][Nq][d];  k, v  bf16 [B][Hkv][Nk][d];  lse fp32 [B][Hq][Nq] or NULL.
+ *   B >= 0, Nq >= 0, Nk >= 0 (B = 0 or Nq = 0: nothing to do; Nk = 0: O = 0, LSE = -inf),
+ *   Hq >= 1, Hkv >= 1, Hq % Hkv == 0, d == 128.
+ *   mask_kind in attn_mask_kind; window >= 1 for ATTN_MASK_SLIDING (ignored otherwise);
+ *   n_sink >= 0 (used by ATTN_MASK_SLIDING only); scale finite (1/sqrt(d) in the usual case).
+ *   All pointers 16-byte aligned.  Accumulation is fp32; O is rounded to bf16 once.
+ */
+ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink, float scale,
+             attn_stream_t stream);
+
+/*
+ * attn_fwd_f32 - the same operation on fp32 Q, K, V, O (fp32 arithmetic throughout).
+ *   d in {64, 128}; all other arguments and rules as attn_fwd.
+ */
+ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float *o, float *lse, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                 float scale, attn_stream_t stream);
+
+/*
+ * Decode: one new query token per sequence against a contiguous KV cache, split-K over the
+ * keys with a log-sum-exp combine ("Attention Research", section 2: split-K over keys for
+ * decode; "Quadratic Complexity Bottleneck", KV cache).  Every cached key is visible.
+ *   q, o   bf16 [B][Hq][1][d];  k, v  bf16 [B][Hkv][Nk][d];  lse fp32 [B][Hq] or NULL.
+ *   d == 128; G = Hq / Hkv in {1, 2, 4, 8}; num_splits = 0 picks a split count for the device.
+ *   workspace: caller-owned device scratch of at least attn_decode_workspace_bytes(...) bytes
+ *   (same B, Hq, Hkv, Nk, d, num_splits), 16-byte aligned; every call overwrites the part it
+ *   uses before reading it, so it needs no clearing.  attn_decode_workspace_bytes returns 0 for
+ *   arguments attn_decode would reject.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nk, int d, int num_splits);
+
+ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,
+                int Hkv, int Nk, int d, float scale, int num_splits, void *workspace,
+                size_t workspace_bytes, attn_stream_t stream);
+
+/* The split count attn_decode uses for num_splits = 0 on the current device. */
+ATTN_API int attn_decode_num_splits(int B, int Hq, int Hkv, int Nk, int d);
+
+/*
+ * Reads and clears the device error flag of the current device after synchronising `stream`.
+ * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT, or ATTN_ERR_CUDA if the synchronisation failed.
+ */
+ATTN_API int attn_get_device_error(attn_stream_t stream);
+
+/*
+ * Test hook: wait on an mbarrier that nothing will complete, with a wait limit of
+ * `limit_cycles` SM clocks, to exercise the bounded-wait path.  The kernel returns normally
+ * and records ATTN_ERR_DEVICE_TIMEOUT in the device flag.
+ */
+ATTN_API int attn_debug_timeout_probe(long long limit_cycles, attn_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTN_B200_ATTN_H */

@@ -1,0 +1,91 @@
+"""Host-side checks of the C ABI: the library builds and loads, exports every declared symbol,
+and rejects invalid arguments with the documented status before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_82_b200 import attn as A
+from exact_io_aware_82_b200 import build as B
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return A.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
+
+
+def test_header_declarations_match_binding():
+    assert declared_functions() == sorted(A.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    # nothing else of ours leaks out of the library (hidden visibility)
+    out = os.popen("nm -D --defined-only %s" % A.LIB_PATH).read()
+    ours = sorted(set(re.findall(r"\b(attn_\w+)\b", out)))
+    assert ours == declared_functions()
+
+
+def test_status_strings(lib):
+    assert A.abi_version() == 1
+    for rc in (0, -1, -2, -3, -4, -5):
+        assert A.status_string(rc) and A.status_string(rc) != "unknown status"
+    assert A.status_string(42) == "unknown status"
+
+
+P = ctypes.c_void_p(16)  # a non-null, 16-byte aligned dummy: invalid-argument paths never use it
+N = ctypes.c_void_p(0)
+
+
+def fwd(lib, q=P, k=P, v=P, o=P, B=1, Hq=2, Hkv=1, Nq=4, Nk=4, d=128, mask=0, w=0, s=0, scale=0.1,
+        f32=False):
+    fn = lib.attn_fwd_f32 if f32 else lib.attn_fwd
+    return fn(q, k, v, o, N, B, Hq, Hkv, Nq, Nk, d, mask, w, s, scale, N)
+
+
+@pytest.mark.parametrize("f32", [False, True])
+def test_invalid_arguments_are_rejected(lib, f32):
+    E = A.ATTN_ERR_INVALID_ARG
+    assert fwd(lib, q=N, f32=f32) == E
+    assert fwd(lib, k=N, f32=f32) == E
+    assert fwd(lib, v=N, f32=f32) == E
+    assert fwd(lib, o=N, f32=f32) == E
+    assert fwd(lib, B=-1, f32=f32) == E
+    assert fwd(lib, Nq=-1, f32=f32) == E
+    assert fwd(lib, Nk=-1, f32=f32) == E
+    assert fwd(lib, Hq=0, f32=f32) == E
+    assert fwd(lib, Hkv=0, f32=f32) == E
+    assert fwd(lib, Hq=3, Hkv=2, f32=f32) == E
+    assert fwd(lib, mask=3, f32=f32) == E
+    assert fwd(lib, mask=-1, f32=f32) == E
+    assert fwd(lib, mask=2, w=0, f32=f32) == E
+    assert fwd(lib, mask=2, w=4, s=-1, f32=f32) == E
+    assert fwd(lib, scale=float("nan"), f32=f32) == E
+    assert fwd(lib, scale=float("inf"), f32=f32) == E
+
+
+def test_unsupported_shapes_are_rejected(lib):
+    U = A.ATTN_ERR_UNSUPPORTED
+    assert fwd(lib, d=64) == U
+    assert fwd(lib, d=96, f32=True) == U
+    assert fwd(lib, q=ctypes.c_void_p(24)) == U  # misaligned
+    dec = lib.attn_decode
+    assert dec(P, P, P, P, N, 1, 16, 1, 8, 128, 0.1, 0, P, 1 << 20, N) == U  # G = 16
+    assert dec(P, P, P, P, N, 1, 4, 1, 8, 64, 0.1, 0, P, 1 << 20, N) == U  # d = 64
+    E = A.ATTN_ERR_INVALID_ARG
+    assert dec(N, P, P, P, N, 1, 4, 1, 8, 128, 0.1, 0, P, 1 << 20, N) == E
+    assert dec(P, P, P, P, N, 1, 4, 3, 8, 128, 0.1, 0, P, 1 << 20, N) == E
+    assert dec(P, P, P, P, N, 1, 4, 1, 8, 128, 0.1, -1, P, 1 << 20, N) == E
+    assert lib.attn_decode_workspace_bytes(1, 4, 3, 8, 128, 0) == 0
+    assert lib.attn_decode_workspace_bytes(64, 32, 8, 32768, 128, 16) == 64 * 32 * 16 * 129 * 4
