@@ -25,7 +25,7 @@ ATTN_ERR_DEVICE_TIMEOUT = -5
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so")
 
 # every symbol include/attn.h declares
-EXPORTS = ("attn_abi_version", "attn_status_string", "attn_fwd", "attn_fwd_f32",
+EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
            "attn_get_device_error", "attn_debug_timeout_probe")
 
@@ -35,7 +35,10 @@ _lib = None
 class AttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__("%s: %s (status %d)" % (where, status_string(status), status))
+        msg = "%s: %s (status %d)" % (where, status_string(status), status)
+        if status == ATTN_ERR_CUDA:
+            msg += ": " + lib().attn_last_error_detail().decode()
+        super().__init__(msg)
 
 
 def lib():
@@ -49,6 +52,7 @@ def lib():
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.attn_abi_version.argtypes, L.attn_abi_version.restype = [], i
         L.attn_status_string.argtypes, L.attn_status_string.restype = [i], ctypes.c_char_p
+        L.attn_last_error_detail.argtypes, L.attn_last_error_detail.restype = [], ctypes.c_char_p
         L.attn_fwd.argtypes = [vp] * 5 + [i] * 9 + [f, vp]
         L.attn_fwd.restype = i
         L.attn_fwd_f32.argtypes = [vp] * 5 + [i] * 9 + [f, vp]

@@ -31,13 +31,22 @@ struct DeviceInfo {
 
 std::mutex g_mutex;
 DeviceInfo g_devices[kMaxDevices];
+thread_local const char* g_last_detail = "no error";
+
+// Maps a CUDA runtime result to a status, remembering the runtime's text for
+// attn_last_error_detail().
+int cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return ATTN_OK;
+  g_last_detail = cudaGetErrorString(e);
+  return ATTN_ERR_CUDA;
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // Looks up the current device once: compute capability 10.x and the SM count; raises the
 // dynamic shared memory limit of the tensor-core kernel on first use.
 int current_device(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaGetLastError());
   if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceInfo& info = g_devices[dev];
@@ -59,10 +68,14 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    if (cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(fwd::kSmemBytes)) != cudaSuccess)
-      return ATTN_ERR_CUDA;
+    int rc = cuda_status(cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel<false>,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(fwd::kSmemBytes)));
+    if (rc == ATTN_OK)
+      rc = cuda_status(cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel<true>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(fwd::kSmemBytes)));
+    if (rc != ATTN_OK) return rc;
     info->fwd_configured = true;
   }
   if (g_encode == nullptr) {
@@ -82,8 +95,11 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Common argument rules of the forward entry points.
 int check_fwd_args(const void* q, const void* k, const void* v, const void* o, int B, int Hq,
                    int Hkv, int Nq, int Nk, int mask_kind, int window, int n_sink, float scale) {
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (B < 0 || Nq < 0 || Nk < 0 || Hq < 1 || Hkv < 1) return ATTN_ERR_INVALID_ARG;
+  // a pointer may be NULL only when its tensor holds no element
+  const bool q_empty = B == 0 || Nq == 0, kv_empty = B == 0 || Nk == 0;
+  if ((!q_empty && (q == nullptr || o == nullptr)) || (!kv_empty && (k == nullptr || v == nullptr)))
+    return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
   if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_SLIDING) return ATTN_ERR_INVALID_ARG;
   if (mask_kind == ATTN_MASK_SLIDING && window < 1) return ATTN_ERR_INVALID_ARG;
@@ -115,7 +131,7 @@ int launch_fill_empty(T* o, float* lse, size_t rows, int d, cudaStream_t stream)
   if (n == 0) return ATTN_OK;
   const unsigned blocks = static_cast<unsigned>((n + 255) / 256);
   fill_empty_kernel<T><<<blocks, 256, 0, stream>>>(o, lse, rows, d);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 // 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x 128 rows,
@@ -195,6 +211,8 @@ extern "C" {
 
 int attn_abi_version(void) { return 1; }
 
+const char* attn_last_error_detail(void) { return g_last_detail; }
+
 const char* attn_status_string(int status) {
   switch (status) {
     case ATTN_OK: return "ok";
@@ -238,13 +256,19 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.Nk = Nk;
   p.G = Hq / Hkv;
   p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  // scale = 0 makes every visible weight equal; a tiny positive c gives exactly that (every
+  // exp2 argument rounds to 0) while masked scores (-inf) still map to weight 0
   p.c = scale * kLog2e;
+  if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
-  fwd::fwd_bf16_sm100_kernel<<<static_cast<unsigned>(units), fwd::kThreads, fwd::kSmemBytes, st>>>(
-      tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(units));
+  if (scale < 0.f)
+    fwd::fwd_bf16_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  else
+    fwd::fwd_bf16_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
 }
 
 int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float* lse, int B,
@@ -276,7 +300,7 @@ int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float
     dim3 grid((Nq + f32::rows_per_cta<128>() - 1) / f32::rows_per_cta<128>(), Hq, B);
     f32::fwd_f32_kernel<128><<<grid, f32::kWarps * 32, 0, st>>>(q, k, v, o, lse, p);
   }
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int attn_decode_num_splits(int B, int Hq, int Hkv, int Nk, int d) {
@@ -298,8 +322,9 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int Nk, int d, int nu
 int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                 int Hkv, int Nk, int d, float scale, int num_splits, void* workspace,
                 size_t workspace_bytes, attn_stream_t stream) {
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (B < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (B > 0 && (q == nullptr || o == nullptr || (Nk > 0 && (k == nullptr || v == nullptr))))
+    return ATTN_ERR_INVALID_ARG;
   if (num_splits < 0 || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   if (d != dec::kD) return ATTN_ERR_UNSUPPORTED;
   const int G = Hq / Hkv;
@@ -331,20 +356,22 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
     case 4: launch_decode_split<4>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
     default: launch_decode_split<8>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
   }
-  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(ws_o, ws_lse,
                                                          static_cast<__nv_bfloat16*>(o), lse, splits);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 int attn_get_device_error(attn_stream_t stream) {
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  int rc = cuda_status(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  if (rc != ATTN_OK) return rc;
   int flag = 0;
-  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if ((rc = cuda_status(cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(int)))) != ATTN_OK)
+    return rc;
   if (flag != 0) {
     const int zero = 0;
-    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    if ((rc = cuda_status(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)))) != ATTN_OK)
+      return rc;
     return flag;
   }
   return ATTN_OK;
@@ -356,7 +383,7 @@ int attn_debug_timeout_probe(long long limit_cycles, attn_stream_t stream) {
   int rc = current_device(&info);
   if (rc != ATTN_OK) return rc;
   timeout_probe_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(limit_cycles);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  return cuda_status(cudaGetLastError());
 }
 
 }  // extern "C"

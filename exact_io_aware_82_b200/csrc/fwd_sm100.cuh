@@ -9,12 +9,16 @@
 // FlashAttention-3, here re-expressed with tcgen05 and tensor memory).
 //
 // One CTA computes 256 query rows of one (batch, query head) as two 128-row tiles Q0, Q1 that
-// share every K/V tile.  Warp roles (14 warps, 448 threads):
+// share every K/V tile.  Warp roles (12 warps = 3 warpgroups, 384 threads):
 //   warps 0-3   softmax + epilogue for Q0 (thread t owns row t, TMEM lanes 0-127)
 //   warps 4-7   softmax + epilogue for Q1
-//   warps 8-11  idle after set-up (kept so the MMA and load warps are not in a softmax warpgroup)
-//   warp 12     TMEM allocation and the single-thread tcgen05.mma issuer
-//   warp 13     TMA producer (Q once, then K_j and V_j through two 2-stage rings)
+//   warp 8      TMEM allocation and the single-thread tcgen05.mma issuer
+//   warp 9      TMA producer (Q once, then K_j and V_j through two 2-stage rings)
+//   warps 10-11 idle (they complete the third warpgroup)
+// Registers: launched at kRegsLaunch per thread; the two softmax warpgroups then raise their
+// limit to kRegsSoftmax (a whole 128-column score row lives in registers) and the third
+// warpgroup lowers its own to kRegsOther.  Per SM sub-partition (3 warps each) the split sums
+// to the launch budget: 2 * kRegsSoftmax + kRegsOther == 3 * kRegsLaunch.
 // Tensor memory (512 columns x 128 lanes, fp32): S0 [0,128) S1 [128,256) O0 [256,384)
 // O1 [384,512).  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
 // MMA issue order per key tile j (ping-pong between the two query tiles):
@@ -24,19 +28,26 @@
 // the commit that signals S_t(j+1) also covers PV_t(j): the softmax may then rescale O_t.
 #pragma once
 
-#include <cuda_bf16.h>
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "common.cuh"
 
 namespace attn {
 namespace fwd {
 
-constexpr int kBM = 128;             // query rows per tile
-constexpr int kBN = 128;             // keys per tile
-constexpr int kD = 128;              // head dimension
+constexpr int kBM = 128;  // query rows per tile
+constexpr int kBN = 128;  // keys per tile
+constexpr int kD = 128;   // head dimension
 constexpr int kRowsPerCta = 2 * kBM;
-constexpr int kThreads = 448;
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr uint32_t kRegsLaunch = 168;
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsOther = 88;
+static_assert(2 * kRegsSoftmax + kRegsOther == 3 * kRegsLaunch, "register split must balance");
+static_assert(kThreads * kRegsLaunch <= 65536, "launch register budget");
 constexpr uint32_t kTileBytes = kBM * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column half
 constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
@@ -44,7 +55,7 @@ constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if 
 struct Params {
   int B, Hq, Hkv, Nq, Nk, G;
   MaskSpec mask;
-  float c;  // scale * log2(e): scores are handled in log2 units
+  float c;  // scale * log2(e): scores are handled in log2 units (never 0, see the host code)
   int num_qblocks;
   __nv_bfloat16* o;
   float* lse;
@@ -75,7 +86,10 @@ __device__ __forceinline__ bool tile_is_full(const MaskSpec& m, int P0, int kt) 
 }
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
+__device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
+// kNeg: the scale is negative, so the largest scaled score comes from the smallest raw score.
+template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -116,12 +130,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     sm.abort = 0;
     dev::fence_barrier_init();
   }
-  if (warp == 13 && lane == 0) {
+  if (warp == kLoadWarp && lane == 0) {
     dev::tma_prefetch_desc(&tm_q);
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
   }
-  if (warp == 12) {
+  if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
     dev::tmem_relinquish();
   }
@@ -130,8 +144,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
-
-  if (warp == 13) {
+  if (warp >= 8) {
+    // ========== third warpgroup: TMA producer, MMA issuer, two idle warps ==========
+    dev::regs_decrease<kRegsOther>();
+  if (warp == kLoadWarp) {
     // =============================== TMA producer ===============================
     if (lane == 0) {
       int k_issued = 0, v_issued = 0;
@@ -175,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (uv >= 0) wait_drain(dev::smem_u32(&sm.bar_vfull[s]), (uv >> 1) & 1);
       }
     }
-  } else if (warp == 12) {
+  } else if (warp == kMmaWarp) {
     // ============================ tcgen05.mma issuer =============================
     if (lane == 0 && nk > 0) {
       constexpr uint32_t idesc_s = dev::idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
@@ -248,16 +264,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
       wait_drain(dev::smem_u32(&sm.bar_drain), 0);
     }
-  } else if (warp < 8) {
+  }
+  } else {
     // ====================== softmax + epilogue (one row per thread) ======================
-    const int t = warp >> 2;            // query tile of this warpgroup
-    const int row = tid & 127;          // row inside the tile == TMEM lane
+    dev::regs_increase<kRegsSoftmax>();
+    const int t = warp >> 2;    // query tile of this warpgroup
+    const int row = tid & 127;  // row inside the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_off + t * 128;
     const uint32_t t_o = tmem + lane_off + 256 + t * 128;
     const int P0 = r0 + t * kBM + off;  // key position of the tile's first row
     const int prow = P0 + row;          // key position of this thread's row
     const float c = p.c;
+    const float masked = kNeg ? pos_inf() : neg_inf();
     float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
     bool ok = true;
@@ -268,29 +287,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_fence_after();
       const int kt = tr.tile(j);
       const int key0 = kt * kBN;
-      const bool full = tile_is_full(p.mask, P0, kt);
 
-      // pass 1: row max of the (masked) scores of this tile
-      float mx = neg_inf();
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        dev::tmem_ld32(t_s + cc * 32, r);
-        dev::tmem_wait_ld();
-        if (full) {
+      // the whole 128-column score row of this thread, one wait
+      uint32_t r[128];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(r[e]) * c);
-        } else {
+      for (int cc = 0; cc < 4; ++cc) dev::tmem_ld32(t_s + cc * 32, r + cc * 32);
+      dev::tmem_wait_ld_regs(r);
+
+      if (!tile_is_full(p.mask, P0, kt)) {
+        // visible columns of this row inside the tile: col <= hi and (col >= lo or col < sk)
+        const int hi = min(p.mask.kind == ATTN_MASK_FULL ? p.mask.Nk - 1 : prow, p.mask.Nk - 1) - key0;
+        const bool sl = p.mask.kind == ATTN_MASK_SLIDING;
+        const int lo = sl ? prow - p.mask.window + 1 - key0 : -(1 << 30);
+        const int sk = sl ? p.mask.n_sink - key0 : -(1 << 30);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x = key_visible(p.mask, prow, key0 + cc * 32 + e)
-                                ? __uint_as_float(r[e]) * c
-                                : neg_inf();
-            mx = fmaxf(mx, x);
-          }
-        }
+        for (int e = 0; e < 128; ++e)
+          if (!(e <= hi && (e >= lo || e < sk))) r[e] = __float_as_uint(masked);
       }
-      const float m_new = fmaxf(m_ref, mx);
+
+      // row max of the raw scores (min when the scale is negative): 3-input max tree
+      float mx;
+      {
+        float a[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r[i]);
+#pragma unroll
+        for (int e = 8; e < 120; e += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            a[i] = kNeg ? dev::min3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]))
+                        : dev::max3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]));
+        }
+        // the loop folded columns 8..119 into a[]; fold 120..127, then reduce a[] to one value
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          a[i] = kNeg ? fminf(a[i], __uint_as_float(r[120 + i])) : fmaxf(a[i], __uint_as_float(r[120 + i]));
+        mx = kNeg ? dev::min3(dev::min3(a[0], a[1], a[2]), dev::min3(a[3], a[4], a[5]), fminf(a[6], a[7]))
+                  : dev::max3(dev::max3(a[0], a[1], a[2]), dev::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+      }
+      const float tmax = (mx == masked) ? neg_inf() : mx * c;
+      const float m_new = fmaxf(m_ref, tmax);
       float alpha = 1.f;
       if (m_new > m_ref + kRescaleThreshold) {
         alpha = dev::ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
@@ -303,35 +339,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
-          uint32_t r[32];
-          dev::tmem_ld32(t_o + cc * 32, r);
-          dev::tmem_wait_ld();
+          uint32_t o[32];
+          dev::tmem_ld32(t_o + cc * 32, o);
+          dev::tmem_wait_ld_regs(o);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          dev::tmem_st32(t_o + cc * 32, r);
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          dev::tmem_st32(t_o + cc * 32, o);
         }
       }
 
-      // pass 2: P = exp2(s*c - m_use) -> bf16, written over the consumed S columns
-#pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
-        dev::tmem_ld32(t_s + cc * 32, r);
-        dev::tmem_wait_ld();
-        uint32_t pk[16];
+      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t; the row sum
+      // accumulates in 8 independent packed pairs
+      float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[e]), c, -m_use));
-          float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[e + 1]), c, -m_use));
-          if (!full) {
-            if (!key_visible(p.mask, prow, key0 + cc * 32 + e)) p0 = 0.f;
-            if (!key_visible(p.mask, prow, key0 + cc * 32 + e + 1)) p1 = 0.f;
-          }
-          l += p0 + p1;
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 64; e += 2) {
+          const int col = half * 64 + e;
+          const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
+          const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
+          acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
           pk[e >> 1] = dev::pack_bf16x2(p0, p1);
         }
-        dev::tmem_st16(t_s + cc * 16, pk);
+        dev::tmem_st32(t_s + half * 32, pk);
       }
+      acc[0] = dev::add2(acc[0], acc[1]);
+      acc[2] = dev::add2(acc[2], acc[3]);
+      acc[0] = dev::add2(acc[0], acc[2]);
+      l += acc[0].x + acc[0].y;
       dev::tmem_wait_st();
       dev::tc_fence_before();
       dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));
@@ -348,19 +384,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.Nq + grow) * kD);
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t r[32];
+        uint32_t o[32];
         if (nk > 0) {
-          dev::tmem_ld32(t_o + cc * 32, r);
-          dev::tmem_wait_ld();
+          dev::tmem_ld32(t_o + cc * 32, o);
+          dev::tmem_wait_ld_regs(o);
         } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = 0u;
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2)
-          pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(r[e]) * inv_l,
-                                        __uint_as_float(r[e + 1]) * inv_l);
+          pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
+                                        __uint_as_float(o[e + 1]) * inv_l);
         if (valid) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
@@ -378,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- teardown ----
   dev::tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == kMmaWarp) {
     dev::tc_fence_after();
     dev::tmem_dealloc(tmem, 512);
   }

@@ -29,7 +29,8 @@
  * Layouts: contiguous, row-major, head dimension innermost.
  *   Q, O  [B][Hq][Nq][d]      K, V  [B][Hkv][Nk][d]      LSE  [B][Hq][Nq] fp32
  *
- * Ownership and execution: every pointer is a DEVICE pointer owned by the caller; the library
+ * Ownership and execution: every pointer is a DEVICE pointer owned by the caller (a tensor with
+ * no element may be passed as NULL; LSE may always be NULL when not wanted); the library
  * never allocates, frees or keeps a pointer after the call returns.  Calls only enqueue work
  * on `stream` (asynchronous, reentrant); results are valid once the stream reaches them.
  * No CPU fallback exists: without an sm_100 device a call returns ATTN_ERR_UNSUPPORTED.
@@ -74,6 +75,10 @@ ATTN_API int attn_abi_version(void);
 
 /* Human-readable text for a status code (static storage, never NULL). */
 ATTN_API const char *attn_status_string(int status);
+
+/* The CUDA runtime's text for the last ATTN_ERR_CUDA returned on the calling thread
+ * (static storage, never NULL; "no error" if there was none). */
+ATTN_API const char *attn_last_error_detail(void);
 
 /*
  * attn_fwd - bf16 prefill / full forward.
