@@ -27,7 +27,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 # every symbol include/attn.h declares
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
-           "attn_get_device_error", "attn_debug_timeout_probe")
+           "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc")
+
+# size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
+DECODE_NOALLOC_MAX_BYTES = 32 << 20
 
 _lib = None
 
@@ -65,6 +68,8 @@ def lib():
         L.attn_get_device_error.argtypes, L.attn_get_device_error.restype = [vp], i
         L.attn_debug_timeout_probe.argtypes = [ctypes.c_longlong, vp]
         L.attn_debug_timeout_probe.restype = i
+        L.attn_decode_noalloc.argtypes = [vp] * 5 + [i] * 5 + [f, i, vp]
+        L.attn_decode_noalloc.restype = i
         _lib = L
     return _lib
 
@@ -185,6 +190,31 @@ def attn_decode(q, k, v, o=None, lse=None, scale=None, num_splits=0, workspace=N
                            scale, int(num_splits), _ptr(workspace), workspace.numel(),
                            _stream_ptr(stream))
     _raise(rc, "attn_decode")
+    return o, lse
+
+
+def attn_decode_noalloc(q, k, v, o=None, lse=None, scale=None, num_splits=0, return_lse=True,
+                        stream=None):
+    """attn_decode without a workspace, for callers that cannot allocate device memory: the
+    split partials live in a fixed library-owned device array of DECODE_NOALLOC_MAX_BYTES
+    (shared by every call on the device, so calls that overlap on the GPU race).  Raises
+    AttnError(ATTN_ERR_WORKSPACE) when the call would need more than that array."""
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 4)
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk,
+                                   d, scale, int(num_splits), _stream_ptr(stream))
+    _raise(rc, "attn_decode_noalloc")
     return o, lse
 
 

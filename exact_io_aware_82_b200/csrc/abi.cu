@@ -387,3 +387,58 @@ int attn_debug_timeout_probe(long long limit_cycles, attn_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------
+// Decode without allocation: the same split-K decode, with its partial results kept in a
+// fixed array that the library owns instead of a caller-provided workspace.
+// ------------------------------------------------------------------------------------------
+namespace attn {
+namespace {
+
+// Every GPU that loads this library holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_DECODE_NOALLOC_MAX_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once per device (in
+// host code the array's name is only a host-side stand-in, never a device address).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  int rc = cuda_status(cudaGetDevice(&dev));
+  if (rc != ATTN_OK) return rc;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    rc = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (rc != ATTN_OK) return rc;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_decode_noalloc(const void* q, const void* k, const void* v, void* o,
+                                   float* lse, int B, int Hq, int Hkv, int Nk, int d,
+                                   float scale, int num_splits, attn_stream_t stream) {
+  // same argument rules as attn_decode; the scratch size is checked before anything runs
+  if (B < 0 || Nk < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != dec::kD) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  int rc = current_device(&info);
+  if (rc != ATTN_OK) return rc;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
+  if (B > 0 && Nk > 0) {
+    const int splits = decode_splits(B, Hkv, Nk, G, num_splits, info->num_sms);
+    if (decode_ws_bytes(B, Hq, splits) > ATTN_DECODE_NOALLOC_MAX_BYTES) return ATTN_ERR_WORKSPACE;
+  }
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch)) != ATTN_OK) return rc;
+  return attn_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, scale, num_splits, scratch,
+                     ATTN_DECODE_NOALLOC_MAX_BYTES, stream);
+}

@@ -118,6 +118,34 @@ ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, f
                 int Hkv, int Nk, int d, float scale, int num_splits, void *workspace,
                 size_t workspace_bytes, attn_stream_t stream);
 
+/*
+ * attn_decode_noalloc - attn_decode for callers that cannot allocate device memory.
+ *
+ * Some callers must not call cudaMalloc themselves: code that runs where an allocation (which
+ * can synchronise the whole device) would stall other work, code whose device memory is all
+ * owned and budgeted up front by a host framework or pool allocator, or a plugin that is handed
+ * tensors but no allocator.  This variant takes the same arguments as attn_decode minus the
+ * workspace: the split partials go to a fixed array of ATTN_DECODE_NOALLOC_MAX_BYTES bytes
+ * that the library defines in device memory (every GPU that loads the library holds it until
+ * the process exits).  The library calls no allocation routine here.
+ *
+ * Limits and rules:
+ *  - a call whose partials would need more than ATTN_DECODE_NOALLOC_MAX_BYTES (see
+ *    attn_decode_workspace_bytes) returns ATTN_ERR_WORKSPACE and launches nothing; a smaller
+ *    num_splits lowers the need;
+ *  - the first call on each device looks up the array's device address (and may make CUDA load
+ *    the library's device code on that device); make that first call before any stream capture;
+ *  - all calls on a device share the one array, which keeps the last call's contents; every call
+ *    writes the part it reads, so nothing needs clearing, but two calls that overlap on the GPU
+ *    (different streams, or different host threads, without ordering between them) race on it.
+ * The pages describe no counterpart of this entry point; it exists for callers only.
+ */
+#define ATTN_DECODE_NOALLOC_MAX_BYTES (32u << 20)
+
+ATTN_API int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
+                                 int B, int Hq, int Hkv, int Nk, int d, float scale,
+                                 int num_splits, attn_stream_t stream);
+
 /* The split count attn_decode uses for num_splits = 0 on the current device. */
 ATTN_API int attn_decode_num_splits(int B, int Hq, int Hkv, int Nk, int d);
 
