@@ -23,9 +23,12 @@
 // O1 [384,512).  P_t (bf16, two per column) overwrites the first 64 columns of S_t.
 // MMA issue order per key tile j (ping-pong between the two query tiles):
 //   PV0(j), S0(j+1), PV1(j), S1(j+1)
-// so the tensor core computes one tile while the other tile's softmax runs.  tcgen05.mma
-// executes in issue order, so S_t(j+1) never overwrites P_t(j) before PV_t(j) has read it, and
-// the commit that signals S_t(j+1) also covers PV_t(j): the softmax may then rescale O_t.
+// so the tensor core computes one tile while the other tile's softmax runs; one thread issues
+// both tiles' MMAs, so each tile's P V and next S run back to back at full rate (measured:
+// two issuing threads interleave the tiles on the tensor core and lengthen both chains).
+// tcgen05.mma executes in issue order, so S_t(j+1) never overwrites P_t(j) before PV_t(j)
+// has read it, and the commit that signals S_t(j+1) also covers PV_t(j): the softmax may then
+// rescale O_t.  A query tile skips the key tiles none of its rows can see.
 #pragma once
 
 #include <cuda.h>
@@ -111,8 +114,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r0 = qb * kRowsPerCta;
   const int off = p.Nk - p.Nq;
   const int last_row = min(r0 + kRowsPerCta, p.Nq) - 1;
+  // key tiles of the whole CTA (what the producer loads, in this order) ...
   const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kBN);
   const int nk = tr.count();
+  // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
+  TileRange trt[2];
+  for (int t = 0; t < 2; ++t) {
+    const int lo_row = r0 + t * kBM, hi_row = min(lo_row + kBM, p.Nq) - 1;
+    trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
+                             : key_tiles(p.mask, lo_row + off, hi_row + off, kBN);
+  }
+  // does a query tile with key-tile range r take part in step j (key tile tr.tile(j))?
+  auto in_range = [&](const TileRange& r, int j) {
+    const int u = tr.tile(j);
+    return u < r.ns || (u >= r.lo && u <= r.hi);
+  };
 
   // ---- set-up ----
   if (tid == 0) {
@@ -200,64 +216,95 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tm_s[2] = {tmem + 0, tmem + 128};
       const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
 
+      // Descriptors are built once per buffer; a K-step only moves the start address, which is
+      // the low field of the descriptor (addresses stay far below its 256 KB range, so adding
+      // the offset >> 4 never carries out of the field).
+      const uint64_t dq[2] = {dev::smem_desc(q_base[0], 16, 1024, dev::kSwizzle128B),
+                              dev::smem_desc(q_base[1], 16, 1024, dev::kSwizzle128B)};
+      const uint64_t dk[2] = {dev::smem_desc(dev::smem_u32(sm.k[0]), 16, 1024, dev::kSwizzle128B),
+                              dev::smem_desc(dev::smem_u32(sm.k[1]), 16, 1024, dev::kSwizzle128B)};
+      const uint64_t dv[2] = {
+          dev::smem_desc(dev::smem_u32(sm.v[0]), kHalfBytes, 1024, dev::kSwizzle128B),
+          dev::smem_desc(dev::smem_u32(sm.v[1]), kHalfBytes, 1024, dev::kSwizzle128B)};
       auto issue_s = [&](int t, int s) {
-        const uint32_t kb = dev::smem_u32(sm.k[s]);
+        const uint64_t a0 = t ? dq[1] : dq[0];
+        const uint64_t b0 = s ? dk[1] : dk[0];
+        const uint32_t d = t ? tm_s[1] : tm_s[0];
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = (ks >> 2) * kHalfBytes + (ks & 3) * 32;
-          const uint64_t a = dev::smem_desc(q_base[t] + koff, 16, 1024, dev::kSwizzle128B);
-          const uint64_t bdesc = dev::smem_desc(kb + koff, 16, 1024, dev::kSwizzle128B);
-          dev::umma_ss(tm_s[t], a, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+          dev::umma_ss(d, a0 + koff, b0 + koff, idesc_s, ks > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int s, bool acc) {
-        const uint32_t vb = dev::smem_u32(sm.v[s]);
+        const uint64_t b0 = s ? dv[1] : dv[0];
+        const uint32_t d = t ? tm_o[1] : tm_o[0];
+        const uint32_t a = t ? tm_s[1] : tm_s[0];
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks) {
-          const uint64_t bdesc =
-              dev::smem_desc(vb + ks * 16 * 128, kHalfBytes, 1024, dev::kSwizzle128B);
-          dev::umma_ts(tm_o[t], tm_s[t] + ks * 8, bdesc, idesc_o, (acc || ks > 0) ? 1u : 0u);
-        }
+        for (int ks = 0; ks < kBN / 16; ++ks)
+          dev::umma_ts(d, a + ks * 8, b0 + ((ks * 16 * 128) >> 4), idesc_o, (acc || ks > 0) ? 1u : 0u);
       };
 
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
-      if (ok) ok = wait_bounded(dev::smem_u32(&sm.bar_kfull[0]), 0, abort);
-      if (ok) {
+      // K_j lives in k[j & 1] (phase (j >> 1) & 1 of its barriers), V_j likewise in v[j & 1]
+      auto wait_k = [&](int j) {
+        return wait_bounded(dev::smem_u32(&sm.bar_kfull[j & 1]), (j >> 1) & 1, abort);
+      };
+      auto wait_v = [&](int j) {
+        return wait_bounded(dev::smem_u32(&sm.bar_vfull[j & 1]), (j >> 1) & 1, abort);
+      };
+      auto next_step = [&](const TileRange& r, int j) {
+        int q = j + 1;
+        while (q < nk && !in_range(r, q)) ++q;
+        return q;
+      };
+      // per tile: cur = the step whose S has been issued and whose P V is next; cnt = steps
+      // whose P V has been issued (the tile's barrier phases count only its own steps)
+      int cur0 = next_step(trt[0], -1), cur1 = next_step(trt[1], -1);
+      int cnt0 = 0, cnt1 = 0;
+      auto first_s = [&](int t, int cur) {
+        if (cur >= nk) return true;
+        if (!wait_k(cur)) return false;
         dev::tc_fence_after();
-        issue_s(0, 0);
-        dev::umma_commit(dev::smem_u32(&sm.bar_s[0]));
-        issue_s(1, 0);
-        dev::umma_commit(dev::smem_u32(&sm.bar_s[1]));
-        dev::umma_commit(dev::smem_u32(&sm.bar_kempty[0]));
+        issue_s(t, cur & 1);
+        dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
+        return true;
+      };
+      // one step of tile t at step j: P V, then the S of its next step (or the final commit)
+      auto step = [&](int t, int j, int& cur, int& cnt) {
+        if (cur != j) return true;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_p[t]), cnt & 1, abort)) return false;
+        dev::tc_fence_after();
+        issue_pv(t, j & 1, cnt > 0);
+        ++cnt;
+        const int nxt = next_step(trt[t], j);
+        if (nxt < nk) {
+          if (!wait_k(nxt)) return false;
+          dev::tc_fence_after();
+          issue_s(t, nxt & 1);
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
+        } else {
+          dev::umma_commit(dev::smem_u32(&sm.bar_o[t]));
+        }
+        cur = nxt;
+        return true;
+      };
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
+      // first S of each tile, earlier key tile first (the producer loads in step order)
+      if (ok) ok = cur0 <= cur1 ? (first_s(0, cur0) && first_s(1, cur1))
+                                : (first_s(1, cur1) && first_s(0, cur0));
+      // K_0 is released once every S that reads it is issued; a slot is always waited for
+      // before it is handed back, so a copy still landing is never overwritten
+      if (ok && nk > 0) {
+        if ((ok = wait_k(0))) dev::umma_commit(dev::smem_u32(&sm.bar_kempty[0]));
       }
       for (int j = 0; ok && j < nk; ++j) {
-        const int s = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        const bool more = j + 1 < nk;
-        const int s1 = (j + 1) & 1;
-        const uint32_t ph1 = ((j + 1) >> 1) & 1;
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_vfull[s]), ph, abort))) break;
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[0]), j & 1, abort))) break;
-        dev::tc_fence_after();
-        issue_pv(0, s, j > 0);
-        if (more) {
-          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_kfull[s1]), ph1, abort))) break;
-          dev::tc_fence_after();
-          issue_s(0, s1);
-          dev::umma_commit(dev::smem_u32(&sm.bar_s[0]));
-        } else {
-          dev::umma_commit(dev::smem_u32(&sm.bar_o[0]));
-        }
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[1]), j & 1, abort))) break;
-        dev::tc_fence_after();
-        issue_pv(1, s, j > 0);
-        dev::umma_commit(dev::smem_u32(&sm.bar_vempty[s]));
-        if (more) {
-          issue_s(1, s1);
-          dev::umma_commit(dev::smem_u32(&sm.bar_s[1]));
-          dev::umma_commit(dev::smem_u32(&sm.bar_kempty[s1]));
-        } else {
-          dev::umma_commit(dev::smem_u32(&sm.bar_o[1]));
+        if (!(ok = wait_v(j))) break;
+        if (!(ok = step(0, j, cur0, cnt0) && step(1, j, cur1, cnt1))) break;
+        // every P V reading V_j and every S reading K_(j+1) is issued by now
+        dev::umma_commit(dev::smem_u32(&sm.bar_vempty[j & 1]));
+        if (j + 1 < nk) {
+          if (!(ok = wait_k(j + 1))) break;
+          dev::umma_commit(dev::smem_u32(&sm.bar_kempty[(j + 1) & 1]));
         }
       }
       // drain: every MMA issued above has completed once this commit arrives
@@ -281,8 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
     bool ok = true;
 
+    const TileRange mine = t ? trt[1] : trt[0];
+    int cnt = 0;  // steps this tile has processed
     for (int j = 0; j < nk; ++j) {
-      ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), j & 1, abort);
+      if (!in_range(mine, j)) continue;
+      ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), cnt & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       dev::tc_fence_after();
       const int kt = tr.tile(j);
@@ -336,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
 
       // rescale the running output O_t (complete: the commit for S_t(j) covered PV_t(j-1))
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      if (cnt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -371,10 +421,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_wait_st();
       dev::tc_fence_before();
       dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));
+      ++cnt;
     }
 
     // ---- epilogue: O = O / l in bf16, LSE = ln(sum exp(scale * s)) ----
-    if (ok && nk > 0) ok = wait_bounded(dev::smem_u32(&sm.bar_o[t]), 0, abort);
+    if (ok && cnt > 0) ok = wait_bounded(dev::smem_u32(&sm.bar_o[t]), 0, abort);
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       dev::tc_fence_after();
@@ -385,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
-        if (nk > 0) {
+        if (cnt > 0) {
           dev::tmem_ld32(t_o + cc * 32, o);
           dev::tmem_wait_ld_regs(o);
         } else {
