@@ -51,6 +51,11 @@ WORKLOADS = {
                                                     seed=4),
     "decode_b64_h32_kv8_n32768_d128": dict(kind="decode", B=64, Hq=32, Hkv=8, N=32768, d=128,
                                            mask=FULL, window=0, n_sink=0, seed=5),
+    # 16 packed sequences of mixed lengths (32,768 tokens), causal, cu_seqlens form
+    "varlen_causal_16seq_32k_h16_d128": dict(kind="fwd_varlen", B=16, Hq=16, Hkv=16, N=32768,
+                                             d=128, mask=CAUSAL, window=0, n_sink=0, seed=6,
+                                             lens=[4096, 3584, 3072, 2816, 2560, 2304, 2048, 1792,
+                                                   1664, 1536, 1536, 1280, 1280, 1024, 1024, 1152]),
     # an eighth of the decode workload (1 GiB of cache), for ncu captures that must stay small
     "decode_b8_h32_kv8_n32768_d128": dict(kind="decode", B=8, Hq=32, Hkv=8, N=32768, d=128,
                                           mask=FULL, window=0, n_sink=0, seed=5),
@@ -104,6 +109,10 @@ def work_of(w):
 
     if w["kind"] == "decode":
         return acc.decode_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"]), "GB/s", 1e9
+    if w["kind"] == "fwd_varlen":
+        fl = sum(acc.attn_flops(1, w["Hq"], n, n, w["d"], w["mask"], w["window"], w["n_sink"])
+                 for n in w["lens"])
+        return fl, "TFLOP/s", 1e12
     fl = acc.attn_flops(w["B"], w["Hq"], w["N"], w["N"], w["d"], w["mask"], w["window"],
                         w["n_sink"])
     return fl, "TFLOP/s", 1e12
@@ -114,6 +123,8 @@ def config_of(name, w, n_gpus):
          "mask": MASK_NAMES[w["mask"]]}
     if w["kind"] == "decode":
         c.update({"q_tokens": 1, "kv_len": w["N"]})
+    elif w["kind"] == "fwd_varlen":
+        c.update({"num_seqs": len(w["lens"]), "total_tokens": sum(w["lens"]), "seq_lens": w["lens"]})
     else:
         c.update({"n": w["N"]})
     if w["mask"] == SLIDING:
@@ -211,6 +222,23 @@ class Workload:
         seed = rank_seed(w["seed"], rank)
         dt = torch.float32 if w["kind"] == "fwd_f32" else torch.bfloat16
         nq = 1 if w["kind"] == "decode" else w["N"]
+        if w["kind"] == "fwd_varlen":
+            # packed token-major tensors and the per-sequence offsets
+            total = sum(w["lens"])
+            assert total == w["N"]
+            self.q = synth.normal_torch(seed, synth.Q_ID, (total, w["Hq"], w["d"]), dt, "cuda")
+            self.k = synth.normal_torch(seed, synth.K_ID, (total, w["Hkv"], w["d"]), dt, "cuda")
+            self.v = synth.normal_torch(seed, synth.V_ID, (total, w["Hkv"], w["d"]), dt, "cuda")
+            self.o = torch.empty_like(self.q)
+            self.lse = torch.empty((total, w["Hq"]), dtype=torch.float32, device="cuda")
+            cu = [0]
+            for n in w["lens"]:
+                cu.append(cu[-1] + n)
+            self.cu = torch.tensor(cu, dtype=torch.int32, device="cuda")
+            self.max_len = max(w["lens"])
+            self.ws = None
+            self.launches_per_step = 1
+            return
         self.q = synth.normal_torch(seed, synth.Q_ID, (w["B"], w["Hq"], nq, w["d"]), dt, "cuda")
         self.k = synth.normal_torch(seed, synth.K_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
         self.v = synth.normal_torch(seed, synth.V_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
@@ -232,6 +260,9 @@ class Workload:
         lse = self.lse if lse is None else lse
         if w["kind"] == "decode":
             A.attn_decode(q, k, v, o=o, lse=lse, workspace=self.ws)
+        elif w["kind"] == "fwd_varlen":
+            A.attn_fwd_varlen(q, k, v, self.cu, self.cu, self.max_len, o=o, lse=lse,
+                              mask_kind=w["mask"], window=w["window"], n_sink=w["n_sink"])
         elif w["kind"] == "fwd_f32":
             A.attn_fwd_f32(q, k, v, o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
                            n_sink=w["n_sink"])
@@ -388,6 +419,25 @@ def oracle_sample(name, budget_s, seed=0, host=None):
             return synth.normal_f32(w["seed"], tid, shape).astype(np.float64)
         return synth.bf16_bits_to_f32(synth.normal_bf16_bits(w["seed"], tid, shape)).astype(np.float64)
 
+    if w["kind"] == "fwd_varlen":
+        # one sequence at a time, random rows of it
+        done, secs, rows_done = 0, 0.0, 0
+        lens = w["lens"]
+        while secs < budget_s and rows_done < sum(lens):
+            si = int(rng.integers(0, len(lens)))
+            n = lens[si]
+            base = sum(lens[:si])
+            q = _draw_rows(w, synth.Q_ID, base, n, Hq, d)
+            k = _draw_rows(w, synth.K_ID, base, n, Hkv, d)
+            v = _draw_rows(w, synth.V_ID, base, n, Hkv, d)
+            rows = rng.integers(0, Hq * n, size=min(64, Hq * n))
+            t0 = time.perf_counter()
+            O.attention_rows(q, k, v, rows, w["mask"], w["window"], w["n_sink"], scale)
+            secs += time.perf_counter() - t0
+            done += sum(4 * d * acc.visible_pairs(1, int(r % n) + 1, w["mask"], w["window"], w["n_sink"])
+                        for r in rows)
+            rows_done += len(rows)
+        return done, secs, cores, "%d output rows drawn at random from random sequences of the batch" % rows_done
     if w["kind"] == "decode":
         # one sequence at a time: its query (Hq x d) against its own Hkv heads of the cache
         done, secs, seqs = 0, 0.0, 0
@@ -424,6 +474,18 @@ def oracle_sample(name, budget_s, seed=0, host=None):
         batch = min(batch * 2, 4096)
     return work, secs, cores, "%d output rows drawn at random (with replacement) from the %d rows" % (
         done_rows, total_rows)
+
+
+def _draw_rows(w, tid, base, n, H, d):
+    """Rows [base, base + n) of a packed [total][H][d] tensor as a [1][H][n][d] fp64 array."""
+    import numpy as np
+
+    import synth
+
+    count = n * H * d
+    x = synth._box_muller(synth.splitmix64_np(synth._keys(w["seed"], tid, base * H * d, count)))
+    bits = synth.f32_to_bf16_bits(x.astype(np.float32))
+    return synth.bf16_bits_to_f32(bits).astype(np.float64).reshape(n, H, d).transpose(1, 0, 2)[None]
 
 
 def _draw_slice(w, tid, b, count):

@@ -27,7 +27,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 # every symbol include/attn.h declares
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
-           "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc")
+           "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc",
+           "attn_fwd_varlen")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
 DECODE_NOALLOC_MAX_BYTES = 32 << 20
@@ -70,6 +71,8 @@ def lib():
         L.attn_debug_timeout_probe.restype = i
         L.attn_decode_noalloc.argtypes = [vp] * 5 + [i] * 5 + [f, i, vp]
         L.attn_decode_noalloc.restype = i
+        L.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 10 + [f, vp]
+        L.attn_fwd_varlen.restype = i
         _lib = L
     return _lib
 
@@ -131,6 +134,39 @@ def attn_fwd(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sink=0,
     rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
                         int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
     _raise(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, lse=None,
+                    mask_kind=MASK_FULL, window=0, n_sink=0, scale=None, return_lse=True,
+                    stream=None):
+    """Packed variable-length forward: q [total_q, Hq, d], k/v [total_k, Hkv, d] bf16;
+    cu_seqlens_q / cu_seqlens_k int32 CUDA tensors of num_seqs + 1 offsets.
+
+    Returns (o [total_q, Hq, d] bf16, lse [total_q, Hq] fp32).  Rows outside every sequence are
+    left as they were in ``o`` / ``lse`` (allocated uninitialised when not given).
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n, torch.bfloat16, 3)
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
+        _check(t, n, torch.int32, 1)
+    total_q, Hq, d = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    num_seqs = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != num_seqs + 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
+                               _ptr(cu_seqlens_k), num_seqs, Hq, Hkv, total_q, total_k,
+                               int(max_seqlen_q), d, int(mask_kind), int(window), int(n_sink),
+                               scale, _stream_ptr(stream))
+    _raise(rc, "attn_fwd_varlen")
     return o, lse
 
 

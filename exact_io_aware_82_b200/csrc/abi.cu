@@ -68,14 +68,14 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    int rc = cuda_status(cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel<false>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(fwd::kSmemBytes)));
-    if (rc == ATTN_OK)
-      rc = cuda_status(cudaFuncSetAttribute(fwd::fwd_bf16_sm100_kernel<true>,
-                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                            static_cast<int>(fwd::kSmemBytes)));
-    if (rc != ATTN_OK) return rc;
+    void (*kernels[4])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+        fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
+        fwd::fwd_bf16_sm100_kernel<false, true>, fwd::fwd_bf16_sm100_kernel<true, true>};
+    for (auto* kern : kernels) {
+      const int rc = cuda_status(cudaFuncSetAttribute(
+          kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
+      if (rc != ATTN_OK) return rc;
+    }
     info->fwd_configured = true;
   }
   if (g_encode == nullptr) {
@@ -142,6 +142,22 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
                                  static_cast<cuuint64_t>(rows) * fwd::kD * 2};
   const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D tiled TMA map over a token-major packed [rows][heads][128] bf16 tensor, read as boxes of
+// 64 columns x 1 head x 128 rows (same shared-memory layout as encode_map).
+int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(heads),
+                              static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
+                                 static_cast<cuuint64_t>(heads) * fwd::kD * 2};
+  const cuuint32_t box[3] = {64, 1, 128};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -263,11 +279,65 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs, int Hq,
+                    int Hkv, int total_q, int total_k, int max_seqlen_q, int d, int mask_kind,
+                    int window, int n_sink, float scale, attn_stream_t stream) {
+  if (num_seqs < 0 || total_q < 0 || total_k < 0 || max_seqlen_q < 0) return ATTN_ERR_INVALID_ARG;
+  if (num_seqs > 0 && (cu_seqlens_q == nullptr || cu_seqlens_k == nullptr)) return ATTN_ERR_INVALID_ARG;
+  // the packed tensors play the role of one batch row each for the common checks
+  int rc = check_fwd_args(q, k, v, o, num_seqs > 0 ? 1 : 0, Hq, Hkv, total_q, total_k, mask_kind,
+                          window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  if (d != fwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (num_seqs == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
+  if (total_k == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(total_q) * Hq, d, st);
+  const long long units = static_cast<long long>((max_seqlen_q + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) *
+                          num_seqs * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
+      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  fwd::Params p;
+  p.B = num_seqs;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = total_q;
+  p.Nk = total_k;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, total_k);
+  p.c = scale * kLog2e;
+  if (p.c == 0.f) p.c = 1e-30f;
+  p.num_qblocks = (max_seqlen_q + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.cu_q = cu_seqlens_q;
+  p.cu_k = cu_seqlens_k;
+  const dim3 grid(static_cast<unsigned>(units));
+  if (scale < 0.f)
+    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  else
+    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 

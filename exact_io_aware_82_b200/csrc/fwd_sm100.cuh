@@ -56,8 +56,11 @@ constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column h
 constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
 
 struct Params {
-  int B, Hq, Hkv, Nq, Nk, G;
-  MaskSpec mask;
+  int B, Hq, Hkv, Nq, Nk, G;  // packed variable-length mode: B = number of sequences,
+                              // Nq / Nk = total query / key rows of the packed tensors
+  MaskSpec mask;              // mask.Nk is replaced per sequence in variable-length mode
+  const int* cu_q;            // variable-length mode: sequence s owns query rows
+  const int* cu_k;            // [cu_q[s], cu_q[s+1]) and key rows [cu_k[s], cu_k[s+1])
   float c;  // scale * log2(e): scores are handled in log2 units (never 0, see the host code)
   int num_qblocks;
   __nv_bfloat16* o;
@@ -92,7 +95,11 @@ __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); 
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
 // kNeg: the scale is negative, so the largest scaled score comes from the smallest raw score.
-template <bool kNeg>
+// kVarlen: packed variable-length sequences ("What Lost, and Why", the sequence-packing note:
+// attention is block diagonal, reset at every sequence boundary given by cu_seqlens); tensors
+// are token-major, Q/O [total_q][Hq][d], K/V [total_k][Hkv][d], LSE [total_q][Hq], and each
+// sequence is masked on its own (p_i = i + Nk_s - Nq_s).  Otherwise the dense [B][H][N][d] form.
+template <bool kNeg, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -112,17 +119,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bkv = b * p.Hkv + h / p.G;
   const int r0 = qb * kRowsPerCta;
-  const int off = p.Nk - p.Nq;
-  const int last_row = min(r0 + kRowsPerCta, p.Nq) - 1;
+  // rows of this (sequence, head): q_base / k_base = first packed row, nq / nkeys = lengths
+  int q_base = 0, k_base = 0, nq = p.Nq, nkeys = p.Nk;
+  MaskSpec mask = p.mask;
+  if (kVarlen) {
+    q_base = __ldg(p.cu_q + b);
+    k_base = __ldg(p.cu_k + b);
+    // rows are clamped to the packed tensors, so inconsistent offsets cannot reach past them
+    nq = q_base < 0 ? 0 : max(0, min(__ldg(p.cu_q + b + 1), p.Nq) - q_base);
+    nkeys = k_base < 0 ? 0 : max(0, min(__ldg(p.cu_k + b + 1), p.Nk) - k_base);
+    mask.Nk = nkeys;
+    if (r0 >= nq) return;  // the whole CTA leaves together: this sequence is shorter
+  }
+  const int off = nkeys - nq;
+  const int last_row = min(r0 + kRowsPerCta, nq) - 1;
   // key tiles of the whole CTA (what the producer loads, in this order) ...
-  const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kBN);
+  const TileRange tr = key_tiles(mask, r0 + off, last_row + off, kBN);
   const int nk = tr.count();
   // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
   TileRange trt[2];
   for (int t = 0; t < 2; ++t) {
-    const int lo_row = r0 + t * kBM, hi_row = min(lo_row + kBM, p.Nq) - 1;
+    const int lo_row = r0 + t * kBM, hi_row = min(lo_row + kBM, nq) - 1;
     trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
-                             : key_tiles(p.mask, lo_row + off, hi_row + off, kBN);
+                             : key_tiles(mask, lo_row + off, hi_row + off, kBN);
   }
   // does a query tile with key-tile range r take part in step j (key tile tr.tile(j))?
   auto in_range = [&](const TileRange& r, int j) {
@@ -173,8 +192,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int half = 0; half < 2; ++half)
-            dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                             r0 + t * kBM, bh);
+            if (kVarlen)
+              dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
+                               h, q_base + r0 + t * kBM);
+            else
+              dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
+                               r0 + t * kBM, bh);
         q_issued = true;
         for (int j = 0; j < nk; ++j) {
           const int kt = tr.tile(j);
@@ -184,15 +207,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t bk = dev::smem_u32(&sm.bar_kfull[s]);
           dev::mbar_arrive_expect_tx(bk, kTileBytes);
           for (int half = 0; half < 2; ++half)
-            dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
-                             kt * kBN, bkv);
+            if (kVarlen)
+              dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
+                               h / p.G, k_base + kt * kBN);
+            else
+              dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
+                               kt * kBN, bkv);
           ++k_issued;
           if (!wait_bounded(dev::smem_u32(&sm.bar_vempty[s]), ph, abort)) break;
           const uint32_t bv = dev::smem_u32(&sm.bar_vfull[s]);
           dev::mbar_arrive_expect_tx(bv, kTileBytes);
           for (int half = 0; half < 2; ++half)
-            dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
-                             kt * kBN, bkv);
+            if (kVarlen)
+              dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
+                               h / p.G, k_base + kt * kBN);
+            else
+              dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
+                               kt * kBN, bkv);
           ++v_issued;
         }
       }
@@ -344,12 +375,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 0; cc < 4; ++cc) dev::tmem_ld32(t_s + cc * 32, r + cc * 32);
       dev::tmem_wait_ld_regs(r);
 
-      if (!tile_is_full(p.mask, P0, kt)) {
+      if (!tile_is_full(mask, P0, kt)) {
         // visible columns of this row inside the tile: col <= hi and (col >= lo or col < sk)
-        const int hi = min(p.mask.kind == ATTN_MASK_FULL ? p.mask.Nk - 1 : prow, p.mask.Nk - 1) - key0;
-        const bool sl = p.mask.kind == ATTN_MASK_SLIDING;
-        const int lo = sl ? prow - p.mask.window + 1 - key0 : -(1 << 30);
-        const int sk = sl ? p.mask.n_sink - key0 : -(1 << 30);
+        const int hi = min(mask.kind == ATTN_MASK_FULL ? mask.Nk - 1 : prow, mask.Nk - 1) - key0;
+        const bool sl = mask.kind == ATTN_MASK_SLIDING;
+        const int lo = sl ? prow - mask.window + 1 - key0 : -(1 << 30);
+        const int sk = sl ? mask.n_sink - key0 : -(1 << 30);
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           if (!(e <= hi && (e >= lo || e < sk))) r[e] = __float_as_uint(masked);
@@ -430,9 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       dev::tc_fence_after();
       const int grow = r0 + t * kBM + row;
-      const bool valid = grow < p.Nq;
+      const bool valid = grow < nq;
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + (static_cast<size_t>(bh) * p.Nq + grow) * kD);
+      const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + h
+                                  : static_cast<size_t>(bh) * p.Nq + grow;
+      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
@@ -456,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (valid && p.lse != nullptr) {
         const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
-        p.lse[static_cast<size_t>(bh) * p.Nq + grow] =
+        p.lse[orow] =
             l > 0.f ? (m_use + log2f(l)) * 0.69314718055994531f : neg_inf();
       }
     }

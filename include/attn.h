@@ -94,6 +94,24 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
              attn_stream_t stream);
 
 /*
+ * attn_fwd_varlen - attn_fwd on packed variable-length sequences ("What Lost, and Why", the note
+ * on sequence packing: several sequences concatenated in one batch row, attention masked block
+ * diagonally so that it resets at every boundary given by cu_seqlens).
+ *   q, o  bf16 [total_q][Hq][d];  k, v  bf16 [total_k][Hkv][d];  lse fp32 [total_q][Hq] or NULL
+ *   (token-major packing).  cu_seqlens_q / cu_seqlens_k: DEVICE int32 arrays of num_seqs + 1
+ *   non-decreasing offsets; sequence s owns query rows [cu_seqlens_q[s], cu_seqlens_q[s+1]) and
+ *   key rows [cu_seqlens_k[s], cu_seqlens_k[s+1]), and is masked on its own exactly as attn_fwd
+ *   masks one (b, h) slice (p_i = i + Nk_s - Nq_s).  max_seqlen_q >= every Nq_s (host value; rows
+ *   past it are not computed).  Rows outside every sequence are not written.
+ *   Other arguments and rules as attn_fwd (d == 128, GQA by Hq / Hkv, the same masks).
+ */
+ATTN_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *o, float *lse,
+                             const int *cu_seqlens_q, const int *cu_seqlens_k, int num_seqs,
+                             int Hq, int Hkv, int total_q, int total_k, int max_seqlen_q, int d,
+                             int mask_kind, int window, int n_sink, float scale,
+                             attn_stream_t stream);
+
+/*
  * attn_fwd_f32 - the same operation on fp32 Q, K, V, O (fp32 arithmetic throughout).
  *   d in {64, 128}; all other arguments and rules as attn_fwd.
  */
