@@ -56,6 +56,10 @@ WORKLOADS = {
                                              d=128, mask=CAUSAL, window=0, n_sink=0, seed=6,
                                              lens=[4096, 3584, 3072, 2816, 2560, 2304, 2048, 1792,
                                                    1664, 1536, 1536, 1280, 1280, 1024, 1024, 1152]),
+    # the decode workload over a paged cache: 16-token pages in a seeded random order
+    "paged_decode_b64_h32_kv8_n32768_p16_d128": dict(kind="decode_paged", B=64, Hq=32, Hkv=8,
+                                                     N=32768, d=128, mask=FULL, window=0,
+                                                     n_sink=0, seed=7, page_size=16),
     # an eighth of the decode workload (1 GiB of cache), for ncu captures that must stay small
     "decode_b8_h32_kv8_n32768_d128": dict(kind="decode", B=8, Hq=32, Hkv=8, N=32768, d=128,
                                           mask=FULL, window=0, n_sink=0, seed=5),
@@ -109,6 +113,9 @@ def work_of(w):
 
     if w["kind"] == "decode":
         return acc.decode_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"]), "GB/s", 1e9
+    if w["kind"] == "decode_paged":
+        return acc.decode_paged_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], w["page_size"]), \
+            "GB/s", 1e9
     if w["kind"] == "fwd_varlen":
         fl = sum(acc.attn_flops(1, w["Hq"], n, n, w["d"], w["mask"], w["window"], w["n_sink"])
                  for n in w["lens"])
@@ -121,8 +128,10 @@ def work_of(w):
 def config_of(name, w, n_gpus):
     c = {"workload": name, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "d": w["d"],
          "mask": MASK_NAMES[w["mask"]]}
-    if w["kind"] == "decode":
+    if w["kind"] in ("decode", "decode_paged"):
         c.update({"q_tokens": 1, "kv_len": w["N"]})
+    if w["kind"] == "decode_paged":
+        c.update({"page_size": w["page_size"], "page_order": "seeded random permutation"})
     elif w["kind"] == "fwd_varlen":
         c.update({"num_seqs": len(w["lens"]), "total_tokens": sum(w["lens"]), "seq_lens": w["lens"]})
     else:
@@ -208,7 +217,8 @@ class ClockSampler:
 # our implementation
 # ----------------------------------------------------------------------------------------------
 class Workload:
-    """Device buffers and the step function of one workload on the current GPU."""
+    """Device buffers and the step function of one workload on the current GPU.  ``inputs`` lists
+    every tensor a step reads (the end-to-end timing copies each of them from the host)."""
 
     def __init__(self, name, rank):
         import torch
@@ -221,54 +231,80 @@ class Workload:
         self.A = A
         seed = rank_seed(w["seed"], rank)
         dt = torch.float32 if w["kind"] == "fwd_f32" else torch.bfloat16
-        nq = 1 if w["kind"] == "decode" else w["N"]
+        B, Hq, Hkv, N, d = w["B"], w["Hq"], w["Hkv"], w["N"], w["d"]
+        self.ws = None
+        self.launches_per_step = 1
         if w["kind"] == "fwd_varlen":
             # packed token-major tensors and the per-sequence offsets
             total = sum(w["lens"])
-            assert total == w["N"]
-            self.q = synth.normal_torch(seed, synth.Q_ID, (total, w["Hq"], w["d"]), dt, "cuda")
-            self.k = synth.normal_torch(seed, synth.K_ID, (total, w["Hkv"], w["d"]), dt, "cuda")
-            self.v = synth.normal_torch(seed, synth.V_ID, (total, w["Hkv"], w["d"]), dt, "cuda")
-            self.o = torch.empty_like(self.q)
-            self.lse = torch.empty((total, w["Hq"]), dtype=torch.float32, device="cuda")
-            cu = [0]
-            for n in w["lens"]:
-                cu.append(cu[-1] + n)
-            self.cu = torch.tensor(cu, dtype=torch.int32, device="cuda")
+            assert total == N
+            q = synth.normal_torch(seed, synth.Q_ID, (total, Hq, d), dt, "cuda")
+            k = synth.normal_torch(seed, synth.K_ID, (total, Hkv, d), dt, "cuda")
+            v = synth.normal_torch(seed, synth.V_ID, (total, Hkv, d), dt, "cuda")
+            cu = torch.tensor(np_cumsum0(w["lens"]), dtype=torch.int32, device="cuda")
+            self.inputs = [q, k, v, cu]
+            self.lse = torch.empty((total, Hq), dtype=torch.float32, device="cuda")
             self.max_len = max(w["lens"])
-            self.ws = None
-            self.launches_per_step = 1
-            return
-        self.q = synth.normal_torch(seed, synth.Q_ID, (w["B"], w["Hq"], nq, w["d"]), dt, "cuda")
-        self.k = synth.normal_torch(seed, synth.K_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
-        self.v = synth.normal_torch(seed, synth.V_ID, (w["B"], w["Hkv"], w["N"], w["d"]), dt, "cuda")
-        self.o = torch.empty_like(self.q)
-        lse_shape = (w["B"], w["Hq"]) if w["kind"] == "decode" else (w["B"], w["Hq"], nq)
-        self.lse = torch.empty(lse_shape, dtype=torch.float32, device="cuda")
-        self.ws = None
-        if w["kind"] == "decode":
-            nb = A.attn_decode_workspace_bytes(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], 0)
+        elif w["kind"] == "decode_paged":
+            ps = w["page_size"]
+            table = paged_table(w)
+            num_pages = table.size
+            q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, 1, d), dt, "cuda")
+            k = synth.normal_torch(seed, synth.K_ID, (num_pages, ps, Hkv, d), dt, "cuda")
+            v = synth.normal_torch(seed, synth.V_ID, (num_pages, ps, Hkv, d), dt, "cuda")
+            bt = torch.from_numpy(table).cuda()
+            sl = torch.full((B,), N, dtype=torch.int32, device="cuda")
+            self.inputs = [q, k, v, bt, sl]
+            self.lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        else:
+            nq = 1 if w["kind"] == "decode" else N
+            q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, nq, d), dt, "cuda")
+            k = synth.normal_torch(seed, synth.K_ID, (B, Hkv, N, d), dt, "cuda")
+            v = synth.normal_torch(seed, synth.V_ID, (B, Hkv, N, d), dt, "cuda")
+            self.inputs = [q, k, v]
+            lse_shape = (B, Hq) if w["kind"] == "decode" else (B, Hq, nq)
+            self.lse = torch.empty(lse_shape, dtype=torch.float32, device="cuda")
+        self.o = torch.empty_like(self.inputs[0])
+        if w["kind"] in ("decode", "decode_paged"):
+            nb = A.attn_decode_workspace_bytes(B, Hq, Hkv, N, d, 0)
             self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-        self.launches_per_step = 2 if w["kind"] == "decode" else 1
+            self.launches_per_step = 2
 
-    def run(self, q=None, k=None, v=None, o=None, lse=None):
+    def run(self, inputs=None):
         w, A = self.w, self.A
-        q = self.q if q is None else q
-        k = self.k if k is None else k
-        v = self.v if v is None else v
-        o = self.o if o is None else o
-        lse = self.lse if lse is None else lse
+        x = self.inputs if inputs is None else inputs
+        o, lse = self.o, self.lse
         if w["kind"] == "decode":
-            A.attn_decode(q, k, v, o=o, lse=lse, workspace=self.ws)
+            A.attn_decode(x[0], x[1], x[2], o=o, lse=lse, workspace=self.ws)
+        elif w["kind"] == "decode_paged":
+            A.attn_decode_paged(x[0], x[1], x[2], x[3], x[4], w["N"], o=o, lse=lse,
+                                workspace=self.ws)
         elif w["kind"] == "fwd_varlen":
-            A.attn_fwd_varlen(q, k, v, self.cu, self.cu, self.max_len, o=o, lse=lse,
+            A.attn_fwd_varlen(x[0], x[1], x[2], x[3], x[3], self.max_len, o=o, lse=lse,
                               mask_kind=w["mask"], window=w["window"], n_sink=w["n_sink"])
         elif w["kind"] == "fwd_f32":
-            A.attn_fwd_f32(q, k, v, o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
-                           n_sink=w["n_sink"])
+            A.attn_fwd_f32(x[0], x[1], x[2], o=o, lse=lse, mask_kind=w["mask"],
+                           window=w["window"], n_sink=w["n_sink"])
         else:
-            A.attn_fwd(q, k, v, o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
+            A.attn_fwd(x[0], x[1], x[2], o=o, lse=lse, mask_kind=w["mask"], window=w["window"],
                        n_sink=w["n_sink"])
+
+
+def np_cumsum0(lens):
+    out = [0]
+    for n in lens:
+        out.append(out[-1] + n)
+    return out
+
+
+def paged_table(w):
+    """Block table [B][N / page_size] of a paged workload: every page of the pool used once, in
+    a seeded random order (the same on every rank and for the oracle sample)."""
+    import numpy as np
+
+    per_seq = w["N"] // w["page_size"]
+    perm = np.random.default_rng(w["seed"]).permutation(w["B"] * per_seq).astype(np.int32)
+    return perm.reshape(w["B"], per_seq)
 
 
 def timed_loop(fn, steps, warmup, flush, dist_on, sampler=None):
@@ -352,7 +388,7 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
     # roofline of the dominant kernel: algorithmic work per launch / mean launch duration
     mean_ms = sum(times) / len(times)
     achieved = work / (mean_ms * 1e-3) / scale
-    if w["kind"] == "decode":
+    if w["kind"] in ("decode", "decode_paged"):
         bound, peak, punit = "hbm", peaks["hbm_gbs"], "GB/s"
     else:
         bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
@@ -365,29 +401,26 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
             "peak_source": peak_kind + (" burst" if bound == "tensor" else "")}
 
     # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
-    qh = wl.q.cpu().pin_memory()
-    kh = wl.k.cpu().pin_memory()
-    vh = wl.v.cpu().pin_memory()
+    host_in = [t.cpu().pin_memory() for t in wl.inputs]
+    dev_in = [torch.empty_like(t) for t in wl.inputs]
     oh = torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory()
     lh = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
-    qd, kd, vd = torch.empty_like(wl.q), torch.empty_like(wl.k), torch.empty_like(wl.v)
 
     def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        wl.run(qd, kd, vd)
+        for dst, src in zip(dev_in, host_in):
+            dst.copy_(src, non_blocking=True)
+        wl.run(dev_in)
         oh.copy_(wl.o, non_blocking=True)
         lh.copy_(wl.lse, non_blocking=True)
 
     e2e_times = timed_loop(e2e_step, max(3, min(steps, 20)), 2, flush, dist_on)
     e2e_ms = max_over_ranks(sum(e2e_times), dist_on) / len(e2e_times)
-    h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = oh.numel() * oh.element_size() + lh.numel() * 4
     e2e = {"value": round(world * work / (e2e_ms * 1e-3) / scale, 3), "unit": unit,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_ms, 4)}
-    del qh, kh, vh, qd, kd, vd
+    del host_in, dev_in
     return dict(wl=wl, work=work, unit=unit, value=value, ms_per_step=ms_per_step,
                 roofline=roof, e2e=e2e, clocks=sampler.report(),
                 launches=wl.launches_per_step * steps)
@@ -454,6 +487,29 @@ def oracle_sample(name, budget_s, seed=0, host=None):
             seqs += 1
         return done, secs, cores, "%d of %d sequences (all %d heads, %d cached keys each)" % (
             seqs, B, Hq, N)
+
+    if w["kind"] == "decode_paged":
+        # one sequence at a time, its keys gathered from its pages in block-table order
+        ps = w["page_size"]
+        table = paged_table(w)
+        page_elems = ps * Hkv * d
+        done, secs, seqs = 0, 0.0, 0
+        qall = draw(synth.Q_ID, (B, Hq, 1, d))
+        while secs < budget_s and seqs < B:
+            b = int(rng.integers(0, B))
+            kk = np.concatenate([_draw_slice(w, synth.K_ID, int(p), page_elems).reshape(ps, Hkv, d)
+                                 for p in table[b]])
+            vv = np.concatenate([_draw_slice(w, synth.V_ID, int(p), page_elems).reshape(ps, Hkv, d)
+                                 for p in table[b]])
+            kk = kk[:N].transpose(1, 0, 2)[None]
+            vv = vv[:N].transpose(1, 0, 2)[None]
+            t0 = time.perf_counter()
+            O.attention(qall[b:b + 1], kk, vv, FULL, scale=scale)
+            secs += time.perf_counter() - t0
+            done += acc.decode_paged_bytes(1, Hq, Hkv, N, d, ps)
+            seqs += 1
+        return done, secs, cores, "%d of %d sequences (all %d heads, %d cached keys in %d-key pages)" % (
+            seqs, B, Hq, N, ps)
 
     q = draw(synth.Q_ID, (B, Hq, N, d)) if host is None else host[0]
     k = draw(synth.K_ID, (B, Hkv, N, d)) if host is None else host[1]

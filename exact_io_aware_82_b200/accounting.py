@@ -80,3 +80,12 @@ def decode_bytes(B: int, Hq: int, Hkv: int, Nk: int, d: int, elem: int = 2) -> i
     """Algorithmic bytes of one decode call: the K and V cache once (shared by the G query heads
     of a group), Q read, O written, fp32 LSE written."""
     return elem * d * 2 * B * Hkv * Nk + elem * d * 2 * B * Hq + 4 * B * Hq
+
+
+def decode_paged_bytes(B: int, Hq: int, Hkv: int, Nk: int, d: int, page_size: int,
+                       elem: int = 2) -> int:
+    """Algorithmic bytes of one paged decode call with every sequence Nk keys long: the decode
+    bytes plus the block-table entries it follows (int32, one per page of each sequence) and
+    the int32 sequence lengths."""
+    pages = (Nk + page_size - 1) // page_size
+    return decode_bytes(B, Hq, Hkv, Nk, d, elem) + 4 * B * pages + 4 * B

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
            "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc",
-           "attn_fwd_varlen")
+           "attn_fwd_varlen", "attn_decode_paged")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
 DECODE_NOALLOC_MAX_BYTES = 32 << 20
@@ -73,6 +73,8 @@ def lib():
         L.attn_decode_noalloc.restype = i
         L.attn_fwd_varlen.argtypes = [vp] * 7 + [i] * 10 + [f, vp]
         L.attn_fwd_varlen.restype = i
+        L.attn_decode_paged.argtypes = [vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp]
+        L.attn_decode_paged.restype = i
         _lib = L
     return _lib
 
@@ -226,6 +228,47 @@ def attn_decode(q, k, v, o=None, lse=None, scale=None, num_splits=0, workspace=N
                            scale, int(num_splits), _ptr(workspace), workspace.numel(),
                            _stream_ptr(stream))
     _raise(rc, "attn_decode")
+    return o, lse
+
+
+def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len, o=None, lse=None,
+                      scale=None, num_splits=0, workspace=None, return_lse=True, stream=None):
+    """Decode against a paged cache.
+
+    q [B,Hq,1,d] bf16; k_cache/v_cache [num_pages,page_size,Hkv,d] bf16; block_table
+    [B,max_pages_per_seq] int32; seq_lens [B] int32 (device); max_seq_len an int >= every length.
+    Returns (o [B,Hq,1,d] bf16, lse [B,Hq] fp32).
+    """
+    import torch
+
+    _check(q, "q", torch.bfloat16, 4)
+    _check(k_cache, "k_cache", torch.bfloat16, 4)
+    _check(v_cache, "v_cache", torch.bfloat16, 4)
+    _check(block_table, "block_table", torch.int32, 2)
+    _check(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    num_pages, page_size, Hkv, dk = k_cache.shape
+    if v_cache.shape != k_cache.shape or dk != d:
+        raise ValueError("k_cache and v_cache must both be [num_pages, page_size, Hkv, d]")
+    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    max_seq_len = int(max_seq_len)
+    if workspace is None:
+        nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, max_seq_len, d, num_splits)
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                 _ptr(block_table), _ptr(seq_lens), B, Hq, Hkv, num_pages,
+                                 page_size, block_table.shape[1], max_seq_len, d, scale,
+                                 int(num_splits), _ptr(workspace), workspace.numel(),
+                                 _stream_ptr(stream))
+    _raise(rc, "attn_decode_paged")
     return o, lse
 
 

@@ -199,10 +199,54 @@ size_t decode_ws_bytes(int B, int Hq, int splits) {
 template <int G>
 void launch_decode_split(dim3 grid, int chunk, cudaStream_t stream, const __nv_bfloat16* q,
                          const __nv_bfloat16* k, const __nv_bfloat16* v, float* ws_o,
-                         float* ws_lse, int Hq, int Hkv, int Nk, int splits, float c) {
+                         float* ws_lse, int Hq, int Hkv, int Nk, int splits, float c,
+                         const dec::Paged* pg) {
   const size_t smem = static_cast<size_t>(dec::smem_floats(G, chunk)) * sizeof(float);
-  dec::decode_split_kernel<G><<<grid, dec::kThreads, smem, stream>>>(q, k, v, ws_o, ws_lse, Hq,
-                                                                      Hkv, Nk, chunk, splits, c);
+  if (pg == nullptr)
+    dec::decode_split_kernel<G><<<grid, dec::kThreads, smem, stream>>>(
+        q, k, v, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c);
+  else if ((1 << pg->page_shift) >= 2 * dec::unroll<G>())
+    dec::decode_split_paged_kernel<G, 2><<<grid, dec::kThreads, smem, stream>>>(
+        q, k, v, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, *pg);
+  else
+    dec::decode_split_paged_kernel<G, 1><<<grid, dec::kThreads, smem, stream>>>(
+        q, k, v, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, *pg);
+}
+
+// Split kernel + combine over a contiguous cache (pg == nullptr; Nk keys per sequence) or a
+// paged one (Nk = the longest sequence).  Arguments are already checked.
+int decode_run(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Nk, float scale, int num_splits, void* workspace,
+               size_t workspace_bytes, cudaStream_t st, const DeviceInfo* info,
+               const dec::Paged* pg) {
+  const int G = Hq / Hkv;
+  const int splits = decode_splits(B, Hkv, Nk, G, num_splits, info->num_sms);
+  const size_t need = decode_ws_bytes(B, Hq, splits);
+  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
+    return ATTN_ERR_WORKSPACE;
+  int chunk = (Nk + splits - 1) / splits;
+  // paged: chunks of whole 32-key groups (the kernel's one-lookup-per-iteration path needs the
+  // chunk starts aligned); a multiple of 32 keeps chunk <= the kernel's largest chunk, and
+  // splits past the last key see no keys
+  if (pg != nullptr) chunk = (chunk + 31) & ~31;
+  float* ws_o = static_cast<float*>(workspace);
+  float* ws_lse = ws_o + static_cast<size_t>(B) * Hq * splits * dec::kD;
+  const float c = scale * kLog2e;
+  const dim3 grid(splits, Hkv, B);
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  const auto* kb = static_cast<const __nv_bfloat16*>(k);
+  const auto* vb = static_cast<const __nv_bfloat16*>(v);
+  switch (G) {
+    case 1: launch_decode_split<1>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c, pg); break;
+    case 2: launch_decode_split<2>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c, pg); break;
+    case 4: launch_decode_split<4>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c, pg); break;
+    default: launch_decode_split<8>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c, pg); break;
+  }
+  int rc = cuda_status(cudaGetLastError());
+  if (rc != ATTN_OK) return rc;
+  dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(ws_o, ws_lse,
+                                                         static_cast<__nv_bfloat16*>(o), lse, splits);
+  return cuda_status(cudaGetLastError());
 }
 
 __global__ void timeout_probe_kernel(long long limit) {
@@ -408,28 +452,45 @@ int attn_decode(const void* q, const void* k, const void* v, void* o, float* lse
   if (Nk == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq, d, st);
   if (B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
-  const int splits = decode_splits(B, Hkv, Nk, G, num_splits, info->num_sms);
-  const size_t need = decode_ws_bytes(B, Hq, splits);
-  if (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))
-    return ATTN_ERR_WORKSPACE;
-  const int chunk = (Nk + splits - 1) / splits;
-  float* ws_o = static_cast<float*>(workspace);
-  float* ws_lse = ws_o + static_cast<size_t>(B) * Hq * splits * dec::kD;
-  const float c = scale * kLog2e;
-  const dim3 grid(splits, Hkv, B);
-  const auto* qb = static_cast<const __nv_bfloat16*>(q);
-  const auto* kb = static_cast<const __nv_bfloat16*>(k);
-  const auto* vb = static_cast<const __nv_bfloat16*>(v);
-  switch (G) {
-    case 1: launch_decode_split<1>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
-    case 2: launch_decode_split<2>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
-    case 4: launch_decode_split<4>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
-    default: launch_decode_split<8>(grid, chunk, st, qb, kb, vb, ws_o, ws_lse, Hq, Hkv, Nk, splits, c); break;
-  }
-  if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
-  dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(ws_o, ws_lse,
-                                                         static_cast<__nv_bfloat16*>(o), lse, splits);
-  return cuda_status(cudaGetLastError());
+  return decode_run(q, k, v, o, lse, B, Hq, Hkv, Nk, scale, num_splits, workspace,
+                    workspace_bytes, st, info, nullptr);
+}
+
+int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, void* o,
+                      float* lse, const int* block_table, const int* seq_lens, int B, int Hq,
+                      int Hkv, int num_pages, int page_size, int max_pages_per_seq,
+                      int max_seq_len, int d, float scale, int num_splits, void* workspace,
+                      size_t workspace_bytes, attn_stream_t stream) {
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || num_pages < 0 || max_pages_per_seq < 0 ||
+      max_seq_len < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (page_size < dec::kMinPageSize || page_size > (1 << 20) || (page_size & (page_size - 1)) != 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(max_seq_len) > static_cast<long long>(max_pages_per_seq) * page_size)
+    return ATTN_ERR_INVALID_ARG;
+  if (num_splits < 0 || !std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  const bool any_keys = max_seq_len > 0 && num_pages > 0;
+  if (B > 0 && (q == nullptr || o == nullptr || seq_lens == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (B > 0 && any_keys && (k_cache == nullptr || v_cache == nullptr || block_table == nullptr))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != dec::kD) return ATTN_ERR_UNSUPPORTED;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  int rc = current_device(&info);
+  if (rc != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0) return ATTN_OK;
+  if (!any_keys)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq, d, st);
+  if (B > 65535 || Hkv > 65535) return ATTN_ERR_UNSUPPORTED;
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  const dec::Paged pg{block_table, seq_lens, max_pages_per_seq, num_pages, shift};
+  return decode_run(q, k_cache, v_cache, o, lse, B, Hq, Hkv, max_seq_len, scale, num_splits,
+                    workspace, workspace_bytes, st, info, &pg);
 }
 
 int attn_get_device_error(attn_stream_t stream) {

@@ -8,8 +8,9 @@
 
 namespace attn {
 
-// Set (never cleared on the device) when a bounded wait expires; read and cleared by the host
-// through attn_get_device_error().
+// Set (never cleared on the device) when a bounded wait expires (ATTN_ERR_DEVICE_TIMEOUT) or a
+// kernel met an index it refused to follow (ATTN_ERR_INVALID_ARG: a paged-cache page number
+// outside the cache); read and cleared by the host through attn_get_device_error().
 __device__ int g_device_error = 0;
 
 // Longest a role may wait on one barrier before it gives up: 2^32 SM clocks (about 2 s at the

@@ -1,4 +1,4 @@
-// Split-K decode: one new query token per sequence against a long, contiguous KV cache.
+// Split-K decode: one new query token per sequence against a long KV cache, contiguous or paged.
 //
 // "Attention Research" (learning-materials), section 1: decode reads the whole O(S) KV cache
 // every step, so it is bound by HBM bandwidth; section 2: FlashDecoding splits the keys of a
@@ -42,6 +42,23 @@ __host__ __device__ constexpr int smem_floats(int G, int chunk) {
   return (chunk * G > kWarps * G * kD) ? chunk * G : kWarps * G * kD;
 }
 
+// Paged KV cache ("Attention Research", section 2: FlashInfer's paged KV): key j of sequence b
+// is row (j mod page_size) of page block_table[b][j / page_size]; a page holds page_size rows
+// of [Hkv][d] (token-major).  A referenced page outside [0, num_pages) is never dereferenced:
+// it reads as zero rows and records ATTN_ERR_INVALID_ARG in g_device_error.
+struct Paged {
+  const int* block_table;  // [B][max_pages]
+  const int* seq_lens;     // [B]
+  int max_pages;
+  int num_pages;
+  int page_shift;          // log2(page_size)
+};
+
+// The chunk of one split spans at most this many pages (chunk <= max_chunk<1>() keys and
+// page_size >= kMinPageSize), plus one for a chunk that starts mid-page.
+constexpr int kMinPageSize = 8;
+constexpr int kMaxChunkPages = kMaxScoreFloats / kMinPageSize + 1;
+
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -59,12 +76,15 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kThreads)
-    decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                        const __nv_bfloat16* __restrict__ v, float* __restrict__ ws_o,
-                        float* __restrict__ ws_lse, int Hq, int Hkv, int Nk, int chunk,
-                        int splits, float c) {
+// kPage: 0 = contiguous cache; 1 = paged, any page size; 2 = paged, pages of at least 2U keys
+// (one page lookup per warp iteration).
+template <int G, int kPage>
+__device__ __forceinline__ void decode_split(const __nv_bfloat16* __restrict__ q,
+                                             const __nv_bfloat16* __restrict__ k,
+                                             const __nv_bfloat16* __restrict__ v,
+                                             float* __restrict__ ws_o, float* __restrict__ ws_lse,
+                                             int Hq, int Hkv, int Nk, int chunk, int splits,
+                                             float c, Paged pg) {
   constexpr int U = unroll<G>();
   constexpr int NV = U * G;        // partial dot products per thread per iteration
   constexpr int PER_LANE = NV / 16;  // fully reduced scores each lane ends with
@@ -76,10 +96,63 @@ __global__ void __launch_bounds__(kThreads)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int half = lane >> 4, sl = lane & 15;
   const int j0 = s * chunk;
-  const int n = max(0, min(Nk - j0, chunk));
-  const size_t kv_base = (static_cast<size_t>(b) * Hkv + hk) * Nk;
-  const __nv_bfloat16* kb = k + (kv_base + j0) * kD + 8 * sl;
-  const __nv_bfloat16* vb = v + (kv_base + j0) * kD + 8 * sl;
+  // keys of this sequence: Nk (contiguous cache) or its own length (paged cache)
+  constexpr bool kPaged = kPage != 0;
+  const int len = kPaged ? max(0, min(__ldg(pg.seq_lens + b), Nk)) : Nk;
+  const int n = max(0, min(len - j0, chunk));
+  // contiguous cache: this thread's column slice of key row j0 of (b, hk)
+  const size_t kv_row0 = kPaged ? 0 : (static_cast<size_t>(b) * Hkv + hk) * Nk + j0;
+  const __nv_bfloat16* kb = k + kv_row0 * kD + 8 * sl;
+  const __nv_bfloat16* vb = v + kv_row0 * kD + 8 * sl;
+  // paged: the physical pages of this chunk, looked up once into shared memory
+  __shared__ int pages[kPaged ? kMaxChunkPages : 1];
+  const int page0 = j0 >> pg.page_shift;
+  if (kPaged) {
+    const int npg = n > 0 ? ((j0 + n - 1) >> pg.page_shift) - page0 + 1 : 0;
+    for (int i = tid; i < npg; i += kThreads) {
+      const int lp = page0 + i;
+      const int phys = lp < pg.max_pages ? __ldg(pg.block_table + static_cast<size_t>(b) * pg.max_pages + lp) : -1;
+      const bool ok = phys >= 0 && phys < pg.num_pages;
+      if (!ok) atomicExch(&g_device_error, ATTN_ERR_INVALID_ARG);  // read as zero rows instead
+      pages[i] = ok ? phys : -1;
+    }
+    __syncthreads();
+  }
+  // row `key` of this chunk in a cache tensor (contiguous: base + key rows; paged: via pages[])
+  auto row = [&](const __nv_bfloat16* cache, const __nv_bfloat16* base, int key) -> const __nv_bfloat16* {
+    if (!kPaged) return base + static_cast<size_t>(key) * kD;
+    const int L = j0 + key;
+    const int phys = pages[(L >> pg.page_shift) - page0];
+    if (phys < 0) return nullptr;
+    const size_t r = (static_cast<size_t>(phys) << pg.page_shift) + (L & ((1 << pg.page_shift) - 1));
+    return cache + (r * Hkv + hk) * kD + 8 * sl;
+  };
+  auto load = [&](const __nv_bfloat16* p) { return p ? ldg_stream(p) : make_uint4(0, 0, 0, 0); };
+  // paged, pages of at least 2U keys: the 2U keys a warp loads per iteration start at a multiple
+  // of 2U (chunks are multiples of 32 keys), so they share one page; one lookup per iteration,
+  // then a fixed stride of Hkv rows between consecutive keys
+  constexpr bool one_page = kPage == 2;
+  const size_t key_stride = static_cast<size_t>(Hkv) * kD;
+  auto load_keys = [&](const __nv_bfloat16* cache, const __nv_bfloat16* base, int kw, uint4 (&r)[U]) {
+    if constexpr (one_page) {
+      const int L = j0 + kw;
+      const int phys = kw < n ? pages[(L >> pg.page_shift) - page0] : -1;
+      const size_t r0 = (static_cast<size_t>(phys < 0 ? 0 : phys) << pg.page_shift) +
+                        (L & ((1 << pg.page_shift) - 1));
+      const __nv_bfloat16* p = cache + ((r0 + half) * Hkv + hk) * kD + 8 * sl;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int key = kw + 2 * u + half;
+        r[u] = (phys >= 0 && key < n) ? ldg_stream(p + 2 * u * key_stride) : make_uint4(0, 0, 0, 0);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int key = kw + 2 * u + half;
+        r[u] = key < n ? load(row(cache, base, key)) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
 
   // this thread's slice of the G query vectors, pre-multiplied by scale * log2(e)
   float qf[G][8];
@@ -96,11 +169,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int base = 0; base < n; base += keys_per_iter<G>()) {
     const int kw = base + warp * 2 * U;  // first key of this warp's group
     uint4 kr[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int key = kw + 2 * u + half;
-      kr[u] = key < n ? ldg_stream(kb + static_cast<size_t>(key) * kD) : make_uint4(0, 0, 0, 0);
-    }
+    load_keys(k, kb, kw, kr);
     float part[NV];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -196,11 +265,7 @@ __global__ void __launch_bounds__(kThreads)
   for (int base = 0; base < n; base += keys_per_iter<G>()) {
     const int kw = base + warp * 2 * U;
     uint4 vr[U];
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int key = kw + 2 * u + half;
-      vr[u] = key < n ? ldg_stream(vb + static_cast<size_t>(key) * kD) : make_uint4(0, 0, 0, 0);
-    }
+    load_keys(v, vb, kw, vr);
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int key = kw + 2 * u + half;
@@ -239,6 +304,28 @@ __global__ void __launch_bounds__(kThreads)
     if (dcol == 0)
       ws_lse[row] = l > 0.f ? (stat[0][g] + log2f(l)) * 0.69314718055994531f : -INFINITY;
   }
+}
+
+// Contiguous cache: [B][Hkv][Nk][d].
+template <int G>
+__global__ void __launch_bounds__(kThreads)
+    decode_split_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                        const __nv_bfloat16* __restrict__ v, float* __restrict__ ws_o,
+                        float* __restrict__ ws_lse, int Hq, int Hkv, int Nk, int chunk,
+                        int splits, float c) {
+  decode_split<G, 0>(q, k, v, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, Paged{});
+}
+
+// Paged cache (kPage 1 or 2); registers capped so that as many CTAs stay resident per SM as the
+// contiguous kernel of the same G gets (three at G = 4 with one lookup per iteration, two otherwise).
+template <int G, int kPage>
+__global__ void __launch_bounds__(kThreads, (G == 4 && kPage == 2) ? 3 : 2)
+    decode_split_paged_kernel(const __nv_bfloat16* __restrict__ q,
+                              const __nv_bfloat16* __restrict__ k,
+                              const __nv_bfloat16* __restrict__ v, float* __restrict__ ws_o,
+                              float* __restrict__ ws_lse, int Hq, int Hkv, int Nk, int chunk,
+                              int splits, float c, Paged pg) {
+  decode_split<G, kPage>(q, k, v, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, pg);
 }
 
 // Combine: grid B * Hq, one thread per head-dimension column.

@@ -38,7 +38,8 @@
  * Errors: a call that returns non-zero has launched nothing (except ATTN_ERR_CUDA, returned
  * when a launch itself failed).  Device-side waits are bounded; if one expires the kernel
  * stops early, records the event in a device flag and `attn_get_device_error` reports
- * ATTN_ERR_DEVICE_TIMEOUT after the stream has been synchronised.
+ * ATTN_ERR_DEVICE_TIMEOUT after the stream has been synchronised (the same flag reports an
+ * out-of-range page number met by attn_decode_paged).
  */
 #ifndef EXACT_ATTN_B200_ATTN_H
 #define EXACT_ATTN_B200_ATTN_H
@@ -137,6 +138,35 @@ ATTN_API int attn_decode(const void *q, const void *k, const void *v, void *o, f
                 size_t workspace_bytes, attn_stream_t stream);
 
 /*
+ * attn_decode_paged - decode against a paged KV cache ("Attention Research", section 2: FlashInfer
+ * lists paged KV among its kernel variants, after the reading list's PagedAttention entry).  The
+ * cache is a pool of fixed-size pages shared by all sequences; a per-sequence block table says
+ * which page holds each run of page_size consecutive keys.  Same split-K decode and combine as
+ * attn_decode; every key of a sequence is visible.
+ *   q, o        bf16 [B][Hq][1][d] (device);  lse fp32 [B][Hq] or NULL.
+ *   k_cache, v_cache  bf16 [num_pages][page_size][Hkv][d] (device): key j of sequence b lives at
+ *               page block_table[b][j / page_size], row j % page_size.
+ *   block_table int32 [B][max_pages_per_seq] (device); entries past a sequence's last page are
+ *               never read.
+ *   seq_lens    int32 [B] (device): keys of each sequence, clamped on the device to
+ *               [0, max_seq_len]; a sequence of length 0 gets O = 0, LSE = -inf.
+ *   max_seq_len an upper bound of seq_lens (host); it sets the split count and the workspace size
+ *               and must not exceed max_pages_per_seq * page_size.
+ *   page_size   a power of two, 8 <= page_size <= 2^20.
+ *   workspace   as attn_decode, sized by attn_decode_workspace_bytes(B, Hq, Hkv, max_seq_len, d,
+ *               num_splits).
+ * Errors: as attn_decode for shapes, alignment and workspace; ATTN_ERR_INVALID_ARG for a bad
+ * page_size or max_seq_len.  A block-table entry that a sequence uses and that lies outside
+ * [0, num_pages) is not followed: those keys read as zero vectors and the device flag records
+ * ATTN_ERR_INVALID_ARG (see attn_get_device_error).
+ */
+ATTN_API int attn_decode_paged(const void *q, const void *k_cache, const void *v_cache, void *o,
+                               float *lse, const int *block_table, const int *seq_lens, int B,
+                               int Hq, int Hkv, int num_pages, int page_size, int max_pages_per_seq,
+                               int max_seq_len, int d, float scale, int num_splits,
+                               void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * attn_decode_noalloc - attn_decode for callers that cannot allocate device memory.
  *
  * Some callers must not call cudaMalloc themselves: code that runs where an allocation (which
@@ -169,7 +199,9 @@ ATTN_API int attn_decode_num_splits(int B, int Hq, int Hkv, int Nk, int d);
 
 /*
  * Reads and clears the device error flag of the current device after synchronising `stream`.
- * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT, or ATTN_ERR_CUDA if the synchronisation failed.
+ * Returns ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a bounded wait expired), ATTN_ERR_INVALID_ARG (a
+ * paged decode met a page number outside its cache), or ATTN_ERR_CUDA if the synchronisation
+ * failed.
  */
 ATTN_API int attn_get_device_error(attn_stream_t stream);
 

@@ -89,3 +89,27 @@ def test_unsupported_shapes_are_rejected(lib):
     assert dec(P, P, P, P, N, 1, 4, 1, 8, 128, 0.1, -1, P, 1 << 20, N) == E
     assert lib.attn_decode_workspace_bytes(1, 4, 3, 8, 128, 0) == 0
     assert lib.attn_decode_workspace_bytes(64, 32, 8, 32768, 128, 16) == 64 * 32 * 16 * 129 * 4
+
+
+def paged(lib, q=P, k=P, v=P, o=P, bt=P, sl=P, B=2, Hq=8, Hkv=2, num_pages=10, ps=16, max_pages=4,
+          max_len=64, d=128, scale=0.1, splits=0):
+    return lib.attn_decode_paged(q, k, v, o, N, bt, sl, B, Hq, Hkv, num_pages, ps, max_pages,
+                                 max_len, d, scale, splits, P, 1 << 20, N)
+
+
+def test_paged_decode_invalid_arguments_are_rejected(lib):
+    E = A.ATTN_ERR_INVALID_ARG
+    for ps in (0, 4, 12, 24, 1 << 21):
+        assert paged(lib, ps=ps) == E
+    assert paged(lib, max_len=65) == E          # beyond max_pages * page_size
+    assert paged(lib, max_len=-1) == E
+    assert paged(lib, num_pages=-1) == E
+    assert paged(lib, max_pages=-1) == E
+    assert paged(lib, B=-1) == E
+    assert paged(lib, Hq=3) == E
+    assert paged(lib, q=N) == E
+    assert paged(lib, sl=N) == E
+    assert paged(lib, bt=N) == E
+    assert paged(lib, k=N) == E
+    assert paged(lib, splits=-1) == E
+    assert paged(lib, scale=float("nan")) == E
