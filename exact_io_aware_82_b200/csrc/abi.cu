@@ -153,11 +153,14 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
 // 3-D tiled TMA map over a token-major packed [rows][heads][128] bf16 tensor, read as boxes of
 // 64 columns x 1 head x 128 rows (same shared-memory layout as encode_map).
 int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(heads),
-                              static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
-                                 static_cast<cuuint64_t>(heads) * fwd::kD * 2};
-  const cuuint32_t box[3] = {64, 1, 128};
+  // dimensions (d, rows, heads): rows second, so that a box is a 64 x 128 block of one head as
+  // in the dense map (a box that is one element wide in its second dimension copies measurably
+  // slower); the row stride (heads * d) exceeds the head stride (d)
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(heads) * fwd::kD * 2,
+                                 static_cast<cuuint64_t>(fwd::kD) * 2};
+  const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,

@@ -91,6 +91,12 @@ __device__ __forceinline__ bool tile_is_full(const MaskSpec& m, int P0, int kt) 
   return (c0 > P1 - m.window) || (c1 < m.n_sink);
 }
 
+// Columns 32w .. 32w+31 of a tile that are <= x, as bits (bit i = column 32w + i).
+__device__ __forceinline__ uint32_t cols_upto(int x, int w) {
+  const int k = x - 32 * w;
+  return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
+}
+
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
@@ -194,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                               h, q_base + r0 + t * kBM);
+                               q_base + r0 + t * kBM, h);
             else
               dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
                                r0 + t * kBM, bh);
@@ -209,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
-                               h / p.G, k_base + kt * kBN);
+                               k_base + kt * kBN, h / p.G);
             else
               dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
                                kt * kBN, bkv);
@@ -220,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int half = 0; half < 2; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
-                               h / p.G, k_base + kt * kBN);
+                               k_base + kt * kBN, h / p.G);
             else
               dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
                                kt * kBN, bkv);
@@ -376,14 +382,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_wait_ld_regs(r);
 
       if (!tile_is_full(mask, P0, kt)) {
-        // visible columns of this row inside the tile: col <= hi and (col >= lo or col < sk)
+        // visible columns of this row inside the tile: col <= hi and (col >= lo or col < sk),
+        // as a 128-bit set built with shifts, then one bit test and select per column (no
+        // per-column branches, whatever the compiler knows about hi, lo and sk)
         const int hi = min(mask.kind == ATTN_MASK_FULL ? mask.Nk - 1 : prow, mask.Nk - 1) - key0;
         const bool sl = mask.kind == ATTN_MASK_SLIDING;
         const int lo = sl ? prow - mask.window + 1 - key0 : -(1 << 30);
         const int sk = sl ? mask.n_sink - key0 : -(1 << 30);
+        uint32_t vis[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          vis[w] = cols_upto(hi, w) & (~cols_upto(lo - 1, w) | cols_upto(sk - 1, w));
 #pragma unroll
         for (int e = 0; e < 128; ++e)
-          if (!(e <= hi && (e >= lo || e < sk))) r[e] = __float_as_uint(masked);
+          r[e] = ((vis[e >> 5] >> (e & 31)) & 1u) ? r[e] : __float_as_uint(masked);
       }
 
       // row max of the raw scores (min when the scale is negative): 3-input max tree
