@@ -60,38 +60,54 @@ WORKLOADS = {
     "paged_decode_b64_h32_kv8_n32768_p16_d128": dict(kind="decode_paged", B=64, Hq=32, Hkv=8,
                                                      N=32768, d=128, mask=FULL, window=0,
                                                      n_sink=0, seed=7, page_size=16),
-    # an eighth of the decode workload (1 GiB of cache), for ncu captures that must stay small
+    # an eighth of the decode workloads (1 GiB of cache), for ncu captures that must stay small
     "decode_b8_h32_kv8_n32768_d128": dict(kind="decode", B=8, Hq=32, Hkv=8, N=32768, d=128,
                                           mask=FULL, window=0, n_sink=0, seed=5),
+    "paged_decode_b8_h32_kv8_n32768_p16_d128": dict(kind="decode_paged", B=8, Hq=32, Hkv=8,
+                                                    N=32768, d=128, mask=FULL, window=0,
+                                                    n_sink=0, seed=7, page_size=16),
 }
+PROFILING_ONLY = ("decode_b8_h32_kv8_n32768_d128", "paged_decode_b8_h32_kv8_n32768_p16_d128")
 HEADLINE = "causal_b4_h16_n2048_d128"
 DECODE = "decode_b64_h32_kv8_n32768_d128"
 
 # DRAM traffic per launch of each workload's dominant kernel, from one ncu capture
-# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the kernel sources the
-# capture was taken with; reported as null once the sources differ.
-_SRC = "e13832159bf99466"
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the sources of that
+# kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
-    "causal_b4_h16_n2048_d128": {"bytes": 139483392, "src": _SRC},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 463769856, "src": _SRC},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 679208960, "src": _SRC},
-    # captured on the 8-sequence case (1,078,418,456 B); the cache is read once per sequence, so
-    # the 64-sequence launch moves 8x that
-    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1078418456, "src": _SRC},
-    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1078418456, "src": _SRC},
+    "causal_b4_h16_n2048_d128": {"bytes": 141631488, "src": "c1646697c270d7e4"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 471216640, "src": "c1646697c270d7e4"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 690882560, "src": "c1646697c270d7e4"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1290109184, "src": "c1646697c270d7e4"},
+    # captured on the 8-sequence cases; the cache is read once per sequence, so the
+    # 64-sequence launch moves 8x that
+    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1078274048, "src": "5e2d19b554ce67c9"},
+    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1078274048, "src": "5e2d19b554ce67c9"},
+    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1078672128, "src": "5e2d19b554ce67c9"},
+    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1078672128, "src": "5e2d19b554ce67c9"},
 }
+
+# the device sources each kernel family is compiled from (the launch code in abi.cu only sets
+# up grids and tensor maps)
+FAMILY_SOURCES = {
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
+    "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
+}
+
+
+def family_of(w):
+    return "decode" if w["kind"] in ("decode", "decode_paged") else "prefill"
+
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def kernel_sources_hash() -> str:
+def kernel_sources_hash(family: str) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_82_b200", "csrc")
-    for dirpath, _, files in sorted(os.walk(csrc)):
-        for f in sorted(files):
-            if f.endswith((".cu", ".cuh")):
-                with open(os.path.join(dirpath, f), "rb") as fh:
-                    h.update(f.encode() + b"\0" + fh.read())
+    for f in FAMILY_SOURCES[family]:
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 
@@ -395,7 +411,7 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
         if w["kind"] == "fwd_f32":
             bound, peak = "fp32-fma", None
     tr = NCU_TRAFFIC.get(name)
-    traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash() else None
+    traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash(family_of(w)) else None
     roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic,
             "peak_source": peak_kind + (" burst" if bound == "tensor" else "")}
@@ -635,7 +651,7 @@ def main():
     peaks, peak_kind = load_peaks()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
-    names = ([n for n in WORKLOADS if n != "decode_b8_h32_kv8_n32768_d128"]
+    names = ([n for n in WORKLOADS if n not in PROFILING_ONLY]
              if args.workload == "all" else [args.workload or HEADLINE])
     for name in names:
         r = measure_ours(name, args.steps, args.warmup, rank, world, dist_on, flush, peaks,
