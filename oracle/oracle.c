@@ -3,6 +3,8 @@
  *
  *     O = softmax(Q K^T * scale + mask) V,   LSE_i = ln sum_{visible j} exp(scale * q_i . k_j)
  *
+ * and of its backward pass (dQ, dK, dV for a given dO; oracle_attn_bwd at the end).
+ *
  * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the benchmark's CPU
  * baseline leg may load this library.  It shares no code, header or constant with the CUDA
  * library and includes no CUDA header.
@@ -195,4 +197,140 @@ int64_t oracle_visible_pairs(int Nq, int Nk, int mask_kind, int window, int n_si
         for (j = 0; j < Nk; ++j)
             c += oracle_visible(i + (int64_t)Nk - Nq, j, mask_kind, window, n_sink);
     return c;
+}
+
+/*
+ * Backward pass: gradients of a scalar loss L through O = softmax(Q K^T * scale + mask) V,
+ * given dO = dL/dO.  Written from the chain rule of the definition above (the pages name the
+ * backward pass and its recomputation of attention, "Quadratic Complexity Bottleneck",
+ * FlashAttention section, and "Chapter 3.1 - The Cost of Attention", section 5, but print no
+ * formula for it):
+ *
+ *     P_ij  = exp(scale * q_i . k_j - LSE_i) on visible pairs, 0 elsewhere
+ *     dV_j  = sum_i P_ij dO_i
+ *     dP_ij = dO_i . v_j
+ *     D_i   = sum_j P_ij dP_ij
+ *     dS_ij = P_ij (dP_ij - D_i)
+ *     dQ_i  = scale * sum_j dS_ij k_j          dK_j = scale * sum_i dS_ij q_i
+ *
+ * With GQA the kv head's gradients sum over the G query heads that read it.  Rows with no
+ * visible key contribute nothing.  Two plain passes, each parallel over independent rows:
+ * pass 1 (query rows) forms the whole score row, LSE_i, D_i and dQ_i; pass 2 (key rows)
+ * forms column j of P and dS for every query row of every head of the group and sums dK_j,
+ * dV_j.  No tiling, no blocking.
+ *
+ * Layouts as the forward: Q, dO, dQ [B][Hq][Nq][d]; K, V, dK, dV [B][Hkv][Nk][d].
+ */
+int oracle_attn_bwd(const double *q, const double *k, const double *v, const double *dout,
+                    double *dq, double *dk, double *dv, int B, int Hq, int Hkv, int Nq, int Nk,
+                    int d, int mask_kind, int window, int n_sink, double scale) {
+    if (check_args(B, Hq, Hkv, Nq, Nk, d, mask_kind, window, n_sink)) return -1;
+    const int G = Hq / Hkv;
+    const int64_t rows = (int64_t)B * Hq * Nq;
+    const int64_t krows = (int64_t)B * Hkv * Nk;
+    double *lse = (double *)malloc(sizeof(double) * (size_t)(rows > 0 ? rows : 1));
+    double *Dv = (double *)malloc(sizeof(double) * (size_t)(rows > 0 ? rows : 1));
+    int failed = (lse == NULL || Dv == NULL);
+    if (!failed) {
+        /* ---- pass 1: per query row, LSE_i, D_i and dQ_i ---- */
+#pragma omp parallel
+        {
+            double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+            double *dp = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+            unsigned char *vis = (unsigned char *)malloc((size_t)(Nk > 0 ? Nk : 1));
+            if (!s || !dp || !vis) {
+#pragma omp atomic write
+                failed = 1;
+            } else {
+                int64_t r;
+#pragma omp for schedule(dynamic, 16)
+                for (r = 0; r < rows; ++r) {
+                    const int64_t i = r % Nq, bh = r / Nq;
+                    const int64_t h = bh % Hq, b = bh / Hq, hk = h / G;
+                    const int64_t p = i + (int64_t)Nk - Nq;
+                    const double *qi = q + r * d, *doi = dout + r * d;
+                    const double *Kb = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                    const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                    double *dqi = dq + r * d;
+                    int64_t j;
+                    int t, any = 0;
+                    double m = -INFINITY, l = 0.0, D = 0.0;
+                    for (t = 0; t < d; ++t) dqi[t] = 0.0;
+                    for (j = 0; j < Nk; ++j) {
+                        double acc = 0.0;
+                        for (t = 0; t < d; ++t) acc += qi[t] * Kb[j * (int64_t)d + t];
+                        s[j] = scale * acc;
+                        vis[j] = (unsigned char)oracle_visible(p, j, mask_kind, window, n_sink);
+                        if (vis[j]) {
+                            if (!any || s[j] > m) m = s[j];
+                            any = 1;
+                        }
+                    }
+                    if (!any) {
+                        lse[r] = -INFINITY;
+                        Dv[r] = 0.0;
+                        continue;
+                    }
+                    for (j = 0; j < Nk; ++j) l += vis[j] ? exp(s[j] - m) : 0.0;
+                    lse[r] = m + log(l);
+                    /* P_ij, dP_ij and D_i */
+                    for (j = 0; j < Nk; ++j) {
+                        if (!vis[j]) continue;
+                        double acc = 0.0;
+                        for (t = 0; t < d; ++t) acc += doi[t] * Vb[j * (int64_t)d + t];
+                        dp[j] = acc;
+                        s[j] = exp(s[j] - lse[r]); /* s now holds P_ij */
+                        D += s[j] * dp[j];
+                    }
+                    Dv[r] = D;
+                    /* dQ_i = scale * sum_j P_ij (dP_ij - D_i) k_j */
+                    for (j = 0; j < Nk; ++j) {
+                        if (!vis[j]) continue;
+                        const double ds = s[j] * (dp[j] - D);
+                        for (t = 0; t < d; ++t) dqi[t] += scale * ds * Kb[j * (int64_t)d + t];
+                    }
+                }
+            }
+            free(s);
+            free(dp);
+            free(vis);
+        }
+    }
+    if (!failed) {
+        /* ---- pass 2: per key row, dK_j and dV_j over every query row of the group ---- */
+        int64_t kr;
+#pragma omp parallel for schedule(dynamic, 16)
+        for (kr = 0; kr < krows; ++kr) {
+            const int64_t j = kr % Nk, bk = kr / Nk;
+            const int64_t hk = bk % Hkv, b = bk / Hkv;
+            const double *kj = k + kr * d, *vj = v + kr * d;
+            double *dkj = dk + kr * d, *dvj = dv + kr * d;
+            int t, g;
+            for (t = 0; t < d; ++t) dkj[t] = dvj[t] = 0.0;
+            for (g = 0; g < G; ++g) {
+                const int64_t h = hk * G + g;
+                int64_t i;
+                for (i = 0; i < Nq; ++i) {
+                    const int64_t r = (b * Hq + h) * (int64_t)Nq + i;
+                    if (!oracle_visible(i + (int64_t)Nk - Nq, j, mask_kind, window, n_sink))
+                        continue;
+                    const double *qi = q + r * d, *doi = dout + r * d;
+                    double sc = 0.0, dpv = 0.0;
+                    for (t = 0; t < d; ++t) {
+                        sc += qi[t] * kj[t];
+                        dpv += doi[t] * vj[t];
+                    }
+                    const double pij = exp(scale * sc - lse[r]);
+                    const double ds = pij * (dpv - Dv[r]);
+                    for (t = 0; t < d; ++t) {
+                        dvj[t] += pij * doi[t];
+                        dkj[t] += scale * ds * qi[t];
+                    }
+                }
+            }
+        }
+    }
+    free(lse);
+    free(Dv);
+    return failed ? -2 : 0;
 }

@@ -47,6 +47,8 @@ def _load():
         lib.oracle_visible.argtypes = [ctypes.c_int64, ctypes.c_int64, ctypes.c_int,
                                        ctypes.c_int64, ctypes.c_int64]
         lib.oracle_visible.restype = ctypes.c_int
+        lib.oracle_attn_bwd.argtypes = [dp] * 7 + [ctypes.c_int] * 9 + [ctypes.c_double]
+        lib.oracle_attn_bwd.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -100,6 +102,29 @@ def attention_rows(q, k, v, rows, mask_kind=MASK_FULL, window=0, n_sink=0, scale
     if rc != 0:
         raise ValueError("oracle_attn_rows rejected its arguments (rc=%d)" % rc)
     return o, lse
+
+
+def attention_bwd(q, k, v, dout, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None):
+    """Gradients (dq, dk, dv) of a loss whose gradient with respect to O is ``dout``.
+
+    q, dout: [B,Hq,Nq,d]; k, v: [B,Hkv,Nk,d].  Returns fp64 arrays of the same shapes.
+    """
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if dout.shape != q.shape:
+        raise ValueError("dout must have the shape of q")
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    rc = _load().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk),
+                                 _ptr(dv), B, Hq, Hkv, Nq, Nk, d, int(mask_kind), int(window),
+                                 int(n_sink), float(scale))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd rejected its arguments (rc=%d)" % rc)
+    return dq, dk, dv
 
 
 def visible(p: int, j: int, mask_kind: int, window: int = 0, n_sink: int = 0) -> bool:
