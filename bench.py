@@ -56,6 +56,9 @@ WORKLOADS = {
                                              d=128, mask=CAUSAL, window=0, n_sink=0, seed=6,
                                              lens=[4096, 3584, 3072, 2816, 2560, 2304, 2048, 1792,
                                                    1664, 1536, 1536, 1280, 1280, 1024, 1024, 1152]),
+    # backward pass of the headline workload (dQ, dK, dV from the forward's O and LSE)
+    "bwd_causal_b4_h16_n2048_d128": dict(kind="bwd", B=4, Hq=16, Hkv=16, N=2048, d=128,
+                                         mask=CAUSAL, window=0, n_sink=0, seed=8),
     # the decode workload over a paged cache: 16-token pages in a seeded random order
     "paged_decode_b64_h32_kv8_n32768_p16_d128": dict(kind="decode_paged", B=64, Hq=32, Hkv=8,
                                                      N=32768, d=128, mask=FULL, window=0,
@@ -136,6 +139,9 @@ def work_of(w):
         fl = sum(acc.attn_flops(1, w["Hq"], n, n, w["d"], w["mask"], w["window"], w["n_sink"])
                  for n in w["lens"])
         return fl, "TFLOP/s", 1e12
+    if w["kind"] == "bwd":
+        return acc.attn_bwd_flops(w["B"], w["Hq"], w["N"], w["N"], w["d"], w["mask"], w["window"],
+                                  w["n_sink"]), "TFLOP/s", 1e12
     fl = acc.attn_flops(w["B"], w["Hq"], w["N"], w["N"], w["d"], w["mask"], w["window"],
                         w["n_sink"])
     return fl, "TFLOP/s", 1e12
@@ -249,6 +255,7 @@ class Workload:
         dt = torch.float32 if w["kind"] == "fwd_f32" else torch.bfloat16
         B, Hq, Hkv, N, d = w["B"], w["Hq"], w["Hkv"], w["N"], w["d"]
         self.ws = None
+        self.lse = None
         self.launches_per_step = 1
         if w["kind"] == "fwd_varlen":
             # packed token-major tensors and the per-sequence offsets
@@ -272,6 +279,19 @@ class Workload:
             sl = torch.full((B,), N, dtype=torch.int32, device="cuda")
             self.inputs = [q, k, v, bt, sl]
             self.lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        elif w["kind"] == "bwd":
+            # the forward's outputs for these inputs are inputs of the backward step
+            q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, N, d), dt, "cuda")
+            k = synth.normal_torch(seed, synth.K_ID, (B, Hkv, N, d), dt, "cuda")
+            v = synth.normal_torch(seed, synth.V_ID, (B, Hkv, N, d), dt, "cuda")
+            dout = synth.normal_torch(seed, synth.DO_ID, (B, Hq, N, d), dt, "cuda")
+            o, lse = A.attn_fwd(q, k, v, mask_kind=w["mask"], window=w["window"],
+                                n_sink=w["n_sink"])
+            self.inputs = [q, k, v, o, lse, dout]
+            self.grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
+            self.ws = torch.empty(A.attn_bwd_workspace_bytes(B, Hq, N), dtype=torch.uint8,
+                                  device="cuda")
+            self.launches_per_step = 3
         else:
             nq = 1 if w["kind"] == "decode" else N
             q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, nq, d), dt, "cuda")
@@ -281,6 +301,8 @@ class Workload:
             lse_shape = (B, Hq) if w["kind"] == "decode" else (B, Hq, nq)
             self.lse = torch.empty(lse_shape, dtype=torch.float32, device="cuda")
         self.o = torch.empty_like(self.inputs[0])
+        # what a step hands back to its caller (read back in the end-to-end timing)
+        self.outputs = self.grads if w["kind"] == "bwd" else [self.o, self.lse]
         if w["kind"] in ("decode", "decode_paged"):
             nb = A.attn_decode_workspace_bytes(B, Hq, Hkv, N, d, 0)
             self.ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
@@ -292,6 +314,10 @@ class Workload:
         o, lse = self.o, self.lse
         if w["kind"] == "decode":
             A.attn_decode(x[0], x[1], x[2], o=o, lse=lse, workspace=self.ws)
+        elif w["kind"] == "bwd":
+            g = self.grads
+            A.attn_bwd(x[0], x[1], x[2], x[3], x[4], x[5], mask_kind=w["mask"], window=w["window"],
+                       n_sink=w["n_sink"], dq=g[0], dk=g[1], dv=g[2], workspace=self.ws)
         elif w["kind"] == "decode_paged":
             A.attn_decode_paged(x[0], x[1], x[2], x[3], x[4], w["N"], o=o, lse=lse,
                                 workspace=self.ws)
@@ -419,20 +445,19 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
     # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
     host_in = [t.cpu().pin_memory() for t in wl.inputs]
     dev_in = [torch.empty_like(t) for t in wl.inputs]
-    oh = torch.empty(wl.o.shape, dtype=wl.o.dtype).pin_memory()
-    lh = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.outputs]
 
     def e2e_step():
         for dst, src in zip(dev_in, host_in):
             dst.copy_(src, non_blocking=True)
         wl.run(dev_in)
-        oh.copy_(wl.o, non_blocking=True)
-        lh.copy_(wl.lse, non_blocking=True)
+        for dst, src in zip(host_out, wl.outputs):
+            dst.copy_(src, non_blocking=True)
 
     e2e_times = timed_loop(e2e_step, max(3, min(steps, 20)), 2, flush, dist_on)
     e2e_ms = max_over_ranks(sum(e2e_times), dist_on) / len(e2e_times)
     h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = oh.numel() * oh.element_size() + lh.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
     e2e = {"value": round(world * work / (e2e_ms * 1e-3) / scale, 3), "unit": unit,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_ms, 4)}
@@ -504,6 +529,23 @@ def oracle_sample(name, budget_s, seed=0, host=None):
         return done, secs, cores, "%d of %d sequences (all %d heads, %d cached keys each)" % (
             seqs, B, Hq, N)
 
+    if w["kind"] == "bwd":
+        # one (b, kv head) slice at a time: the gradients of a slice depend on that slice only
+        done, secs, slices = 0, 0.0, 0
+        while secs < budget_s and slices < B * Hkv:
+            b, hk = int(rng.integers(0, B)), int(rng.integers(0, Hkv))
+            qs = np.stack([_draw_slice(w, synth.Q_ID, b * Hq + hk * G + g, N * d) for g in range(G)])
+            ds = np.stack([_draw_slice(w, synth.DO_ID, b * Hq + hk * G + g, N * d) for g in range(G)])
+            kk = _draw_slice(w, synth.K_ID, b * Hkv + hk, N * d).reshape(1, 1, N, d)
+            vv = _draw_slice(w, synth.V_ID, b * Hkv + hk, N * d).reshape(1, 1, N, d)
+            t0 = time.perf_counter()
+            O.attention_bwd(qs.reshape(1, G, N, d), kk, vv, ds.reshape(1, G, N, d), w["mask"],
+                            w["window"], w["n_sink"], scale)
+            secs += time.perf_counter() - t0
+            done += acc.attn_bwd_flops(1, G, N, N, d, w["mask"], w["window"], w["n_sink"])
+            slices += 1
+        return done, secs, cores, "%d of %d (b, kv head) slices (%d query heads, %d rows each)" % (
+            slices, B * Hkv, G, N)
     if w["kind"] == "decode_paged":
         # one sequence at a time, its keys gathered from its pages in block-table order
         ps = w["page_size"]

@@ -89,3 +89,11 @@ def decode_paged_bytes(B: int, Hq: int, Hkv: int, Nk: int, d: int, page_size: in
     the int32 sequence lengths."""
     pages = (Nk + page_size - 1) // page_size
     return decode_bytes(B, Hq, Hkv, Nk, d, elem) + 4 * B * pages + 4 * B
+
+
+def attn_bwd_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int, window: int = 0,
+                   n_sink: int = 0) -> int:
+    """Algorithmic FLOPs of the backward pass: five d-long products per visible pair (recomputed
+    score, dP, and the dV, dK, dQ contributions), 2 * d each, i.e. 10 * d = 2.5 x the forward.
+    The extra score and dP recomputation of a split dQ kernel is not credited."""
+    return 10 * d * B * Hq * visible_pairs(Nq, Nk, mask_kind, window, n_sink)

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
            "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc",
-           "attn_fwd_varlen", "attn_decode_paged")
+           "attn_fwd_varlen", "attn_decode_paged", "attn_bwd", "attn_bwd_workspace_bytes")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
 DECODE_NOALLOC_MAX_BYTES = 32 << 20
@@ -75,6 +75,10 @@ def lib():
         L.attn_fwd_varlen.restype = i
         L.attn_decode_paged.argtypes = [vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp]
         L.attn_decode_paged.restype = i
+        L.attn_bwd_workspace_bytes.argtypes = [i] * 3
+        L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.attn_bwd.argtypes = [vp] * 9 + [i] * 9 + [f, vp, ctypes.c_size_t, vp]
+        L.attn_bwd.restype = i
         _lib = L
     return _lib
 
@@ -191,6 +195,39 @@ def attn_fwd_f32(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sin
                             _stream_ptr(stream))
     _raise(rc, "attn_fwd_f32")
     return o, lse
+
+
+def attn_bwd_workspace_bytes(B, Hq, Nq) -> int:
+    return int(lib().attn_bwd_workspace_bytes(B, Hq, Nq))
+
+
+def attn_bwd(q, k, v, o, lse, dout, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward of attn_fwd: returns (dq, dk, dv), bf16 with the shapes of q, k, v.
+
+    o and lse are the forward's outputs for the same q, k, v, mask and scale; dout = dL/dO.
+    """
+    import torch
+
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _check(t, n, torch.bfloat16, 4)
+    _check(lse, "lse", torch.float32, 3)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("o and dout must have the shape of q, lse [B, Hq, Nq]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(max(attn_bwd_workspace_bytes(B, Hq, Nq), 16), dtype=torch.uint8,
+                                device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, int(mask_kind), int(window),
+                        int(n_sink), scale, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _raise(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits=0) -> int:

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/attn.h"
+#include "bwd_sm100.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "fwd_f32.cuh"
@@ -27,6 +28,7 @@ struct DeviceInfo {
   bool sm100 = false;
   int num_sms = 0;
   bool fwd_configured = false;
+  bool bwd_configured = false;
 };
 
 std::mutex g_mutex;
@@ -91,6 +93,29 @@ int configure_fwd(DeviceInfo* info) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raises the dynamic shared memory limit of the backward kernels on first use.
+int configure_bwd(DeviceInfo* info) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!info->bwd_configured) {
+    int rc = cuda_status(cudaFuncSetAttribute(bwd::bwd_dkdv_kernel,
+                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(bwd::kSmemKVBytes)));
+    if (rc != ATTN_OK) return rc;
+    rc = cuda_status(cudaFuncSetAttribute(bwd::bwd_dq_kernel,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                          static_cast<int>(bwd::kSmemQBytes)));
+    if (rc != ATTN_OK) return rc;
+    info->bwd_configured = true;
+  }
+  return ATTN_OK;
+}
+
+// Backward workspace: LSE * log2(e) and D per query row, rows padded to whole 128-row tiles.
+size_t bwd_ws_bytes(int B, int Hq, int Nq) {
+  const size_t npad = static_cast<size_t>((Nq + bwd::kT - 1) / bwd::kT) * bwd::kT;
+  return 2 * static_cast<size_t>(B) * Hq * npad * sizeof(float);
+}
 
 // Common argument rules of the forward entry points.
 int check_fwd_args(const void* q, const void* k, const void* v, const void* o, int B, int Hq,
@@ -494,6 +519,84 @@ int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, v
   const dec::Paged pg{block_table, seq_lens, max_pages_per_seq, num_pages, shift};
   return decode_run(q, k_cache, v_cache, o, lse, B, Hq, Hkv, max_seq_len, scale, num_splits,
                     workspace, workspace_bytes, st, info, &pg);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq) {
+  if (B < 1 || Hq < 1 || Nq < 0) return 0;
+  return bwd_ws_bytes(B, Hq, Nq);
+}
+
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+             int Nk, int d, int mask_kind, int window, int n_sink, float scale, void* workspace,
+             size_t workspace_bytes, attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  const bool q_empty = B == 0 || Nq == 0, kv_empty = B == 0 || Nk == 0;
+  if (!q_empty && (lse == nullptr || dout == nullptr || dq == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (!kv_empty && (dk == nullptr || dv == nullptr)) return ATTN_ERR_INVALID_ARG;
+  if (d != bwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0) return ATTN_OK;
+  const size_t q_bytes = static_cast<size_t>(B) * Hq * Nq * d * 2;
+  const size_t kv_bytes = static_cast<size_t>(B) * Hkv * Nk * d * 2;
+  // no query: every key gets zero gradients; no key: every query does
+  if (Nq == 0 || Nk == 0) {
+    if (Nq == 0 && Nk > 0) {
+      if ((rc = cuda_status(cudaMemsetAsync(dk, 0, kv_bytes, st))) != ATTN_OK) return rc;
+      return cuda_status(cudaMemsetAsync(dv, 0, kv_bytes, st));
+    }
+    if (Nq > 0) return cuda_status(cudaMemsetAsync(dq, 0, q_bytes, st));
+    return ATTN_OK;
+  }
+  const int nqt = (Nq + bwd::kT - 1) / bwd::kT, nkb = (Nk + bwd::kT - 1) / bwd::kT;
+  const long long units_q = static_cast<long long>(nqt) * B * Hq;
+  const long long units_kv = static_cast<long long>(nkb) * B * Hkv;
+  if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (workspace == nullptr || workspace_bytes < bwd_ws_bytes(B, Hq, Nq) || !aligned16(workspace))
+    return ATTN_ERR_WORKSPACE;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;  // the tensor-map encoder
+  if ((rc = configure_bwd(info)) != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv, tdo;
+  if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK || encode_map(&tdo, dout, Nq, B * Hq) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  bwd::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.scale = scale;
+  p.c = scale * kLog2e;
+  p.num_kblocks = nkb;
+  p.num_qtiles = nqt;
+  p.npad = nqt * bwd::kT;
+  float* lse2 = static_cast<float*>(workspace);
+  float* dsum = lse2 + static_cast<size_t>(B) * Hq * p.npad;
+  p.lse2 = lse2;
+  p.dsum = dsum;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  const long long prow = static_cast<long long>(B) * Hq * p.npad;
+  bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
+      dsum, Nq, p.npad, prow);
+  if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
+  bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(units_kv), bwd::kThreads, bwd::kSmemKVBytes, st>>>(
+      tq, tk, tv, tdo, p);
+  if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
+  bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
+      tq, tk, tv, tdo, p);
+  return cuda_status(cudaGetLastError());
 }
 
 int attn_get_device_error(attn_stream_t stream) {

@@ -1,0 +1,654 @@
+// Backward pass of exact attention on sm_100a: dQ, dK, dV from Q, K, V, dO and the forward's
+// row log-sum-exp, recomputing the attention weights instead of storing them.
+//
+// "Quadratic Complexity Bottleneck" (inferensys.com), FlashAttention section: the backward pass
+// recomputes attention instead of keeping the n x n matrix; "Chapter 3.1 - The Cost of
+// Attention" (llmis.ru), section 5: FlashAttention trades "somewhat more FLOPs" for memory.
+// With P_ij = exp(scale * q_i.k_j - LSE_i) on visible pairs (the LSE saved by the forward makes
+// P exact without a second softmax pass):
+//
+//     dV_j = sum_i P_ij dO_i       dP_ij = dO_i . v_j       D_i = dO_i . O_i (= sum_j P_ij dP_ij)
+//     dS_ij = P_ij (dP_ij - D_i)   dK_j = scale sum_i dS_ij q_i   dQ_i = scale sum_j dS_ij k_j
+//
+// Three launches:
+//  1. bwd_prep_kernel: D_i and LSE_i * log2(e) per query row (memory-bound, one warp per row).
+//  2. bwd_dkdv_kernel: one CTA per (b, kv head, 128-key block).  It walks the query tiles that see
+//     the block, for each of the G query heads of the group, and keeps dK and dV of its keys in
+//     tensor memory for the whole walk (no atomics; GQA sums in place).  Per step, four tcgen05
+//     MMAs (128 x 128 x 128, bf16 in, fp32 accumulate): S^T = K Q^T and dP^T = V dO^T into TMEM;
+//     the row warps (one TMEM lane = one key each) turn them into P^T and dS^T (bf16, written
+//     back over S^T and dP^T); then dV += P^T dO and dK += dS^T Q with P^T / dS^T as the A operand
+//     read from TMEM.
+//  3. bwd_dq_kernel: one CTA per (b, query head, 128-row query tile), walking the key tiles the
+//     tile sees: S = Q K^T, dP = dO V^T, dS in TMEM (bf16), dQ += dS K.
+// Splitting dQ from dK/dV recomputes S and dP once more (7 MMA tiles per visible tile pair
+// instead of 5) but needs neither atomics nor a second accumulator set, and the result does not
+// depend on the order in which CTAs finish.
+//
+// Roles of each 192-thread CTA: warps 0-3 are the row workers (thread t owns TMEM lane t), warp
+// 4 issues every tcgen05.mma from one thread, warp 5 issues the TMA copies from one thread.
+// Tensor memory (512 columns): [0,128) S or S^T, [128,256) dP or dP^T, [256,384) dV or dQ,
+// [384,512) dK.  Every wait is bounded (see common.cuh).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+
+namespace attn {
+namespace bwd {
+
+constexpr int kT = 128;  // tile rows and columns (queries and keys)
+constexpr int kD = 128;  // head dimension
+constexpr int kThreads = 192;
+constexpr int kMmaWarp = 4;
+constexpr int kLoadWarp = 5;
+constexpr uint32_t kTileBytes = kT * kD * 2;  // 32 KB, bf16
+constexpr uint32_t kHalfBytes = kT * 64 * 2;  // one 128-byte-swizzled 64-column half
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct Params {
+  int B, Hq, Hkv, Nq, Nk, G;
+  MaskSpec mask;
+  float c;      // scale * log2(e)
+  float scale;
+  const float* lse2;  // [B][Hq][npad] LSE * log2(e); +inf for a row that sees no key or is padding
+  const float* dsum;  // [B][Hq][npad] D_i = dO_i . O_i; 0 for padding rows
+  __nv_bfloat16* dq;  // [B][Hq][Nq][d]
+  __nv_bfloat16* dk;  // [B][Hkv][Nk][d]
+  __nv_bfloat16* dv;  // [B][Hkv][Nk][d]
+  int num_kblocks;    // ceil(Nk / 128)
+  int num_qtiles;     // ceil(Nq / 128)
+  int npad;           // num_qtiles * 128: row stride of lse2 and dsum
+};
+
+// ------------------------------------------------------------------------------------------
+// helpers
+// ------------------------------------------------------------------------------------------
+__device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
+
+// Columns 32w .. 32w+31 of a tile that are <= x, as bits (bit i = column 32w + i).
+__device__ __forceinline__ uint32_t cols_upto(int x, int w) {
+  const int k = x - 32 * w;
+  return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
+}
+
+// clamp a 64-bit column bound into [-1, 128] (every bound outside the tile acts the same)
+__device__ __forceinline__ int clamp_col(long long x) {
+  return x < -1 ? -1 : (x > kT ? kT : static_cast<int>(x));
+}
+
+// Is every pair of the block (query positions P0 .. P0+127) x (keys c0 .. c0+127) visible?
+// Conservative: rows past Nq count as visible here (their weights are zero through LSE = +inf).
+__device__ __forceinline__ bool block_full(const MaskSpec& m, int P0, int c0) {
+  const int c1 = c0 + kT - 1, P1 = P0 + kT - 1;
+  if (c1 >= m.Nk) return false;
+  if (m.kind == ATTN_MASK_FULL) return true;
+  if (c1 > P0) return false;
+  if (m.kind == ATTN_MASK_CAUSAL) return true;
+  return (static_cast<long long>(c0) > static_cast<long long>(P1) - m.window) || (c1 < m.n_sink);
+}
+
+__device__ __forceinline__ int floor_div128(long long a) {
+  return static_cast<int>(a >= 0 ? a / kT : -((-a + kT - 1) / kT));
+}
+
+// Query tiles [lo, hi] whose rows see at least one key of [c0, c1] (off = Nk - Nq; query row i
+// sits at key position i + off).  Empty when lo > hi.
+__device__ __forceinline__ void query_tiles(const MaskSpec& m, int c0, int c1, int off, int Nq,
+                                            int& lo, int& hi) {
+  const int nqt = (Nq + kT - 1) / kT;
+  lo = 0;
+  hi = nqt - 1;
+  if (m.kind == ATTN_MASK_FULL) return;
+  // causal: p = i + off >= key  ->  i >= c0 - off for the block's first key
+  lo = max(0, floor_div128(static_cast<long long>(c0) - off));
+  // window: p < key + w for keys past the sinks (a block holding a sink key is seen by every
+  // later row)
+  if (m.kind == ATTN_MASK_SLIDING && c0 >= m.n_sink)
+    hi = min(hi, floor_div128(static_cast<long long>(c1) + m.window - 1 - off));
+}
+
+// Producer drain: wait until the last copy issued into stage s (of `issued` copies alternating
+// between two stages) has landed.
+__device__ __forceinline__ void drain_stage(uint32_t bar, int issued, int s) {
+  const int u = (issued - 1 - s) >= 0 ? ((issued - 1 - s) & ~1) + s : -1;
+  if (u >= 0) wait_drain(bar, (u >> 1) & 1);
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16),
+// completion counted on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Row r of a 128 x 128 fp32 accumulator in TMEM -> bf16 row of global memory (times mul).
+__device__ __forceinline__ void store_acc_row(uint32_t t_acc, float mul, __nv_bfloat16* dst,
+                                              bool valid) {
+#pragma unroll 1
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t a[32];
+    dev::tmem_ld32(t_acc + cc * 32, a);
+    dev::tmem_wait_ld_regs(a);
+    uint32_t pk[16];
+#pragma unroll
+    for (int e = 0; e < 32; e += 2)
+      pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(a[e]) * mul, __uint_as_float(a[e + 1]) * mul);
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4)
+        d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// ------------------------------------------------------------------------------------------
+// 1. D_i = dO_i . O_i and LSE_i * log2(e): one warp per query row
+// ------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+                    const float* __restrict__ lse, float* __restrict__ lse2,
+                    float* __restrict__ dsum, int Nq, int npad, long long padded_rows) {
+  // padded row index -> (b*Hq + h, i); rows i >= Nq only get the padding values
+  const long long prow = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (prow >= padded_rows) return;
+  const long long bh = prow / npad;
+  const int i = static_cast<int>(prow % npad);
+  if (i >= Nq) {
+    if (lane == 0) {
+      dsum[prow] = 0.f;
+      lse2[prow] = pos_inf();
+    }
+    return;
+  }
+  const long long row = bh * Nq + i;
+  const uint2 a = *reinterpret_cast<const uint2*>(o + row * kD + lane * 4);
+  const uint2 g = *reinterpret_cast<const uint2*>(dout + row * kD + lane * 4);
+  float acc = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16);
+  acc = fmaf(__uint_as_float(a.x & 0xffff0000u), __uint_as_float(g.x & 0xffff0000u), acc);
+  acc = fmaf(__uint_as_float(a.y << 16), __uint_as_float(g.y << 16), acc);
+  acc = fmaf(__uint_as_float(a.y & 0xffff0000u), __uint_as_float(g.y & 0xffff0000u), acc);
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+  if (lane == 0) {
+    dsum[prow] = acc;
+    const float l = lse[row];
+    lse2[prow] = (l == -pos_inf()) ? pos_inf() : l * kLog2e;
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 2. dK, dV: one CTA per (b, kv head, key block)
+// ------------------------------------------------------------------------------------------
+struct __align__(1024) SmemKV {
+  uint8_t k[kTileBytes];
+  uint8_t v[kTileBytes];
+  uint8_t q[2][kTileBytes];
+  uint8_t dout[2][kTileBytes];
+  float lse2[2][kT];  // per stage: the query tile's LSE * log2(e) and D, copied with Q and dO
+  float dsum[2][kT];
+  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s, bar_p, bar_done, bar_drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemKVBytes = sizeof(SmemKV) + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_do, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                          ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // key block kb of (b, hk); lowest blocks first (they have the most query tiles under a
+  // causal mask)
+  const int nbk = p.B * p.Hkv;
+  const int kb = blockIdx.x / nbk;
+  const int bk = blockIdx.x % nbk;
+  const int b = bk / p.Hkv, hk = bk % p.Hkv;
+  const int c0 = kb * kT, c1 = min(c0 + kT, p.Nk) - 1;
+  const int off = p.Nk - p.Nq;
+  int qlo, qhi;
+  query_tiles(p.mask, c0, c1, off, p.Nq, qlo, qhi);
+  const int nqt = qhi >= qlo ? qhi - qlo + 1 : 0;
+  const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qlo + n % nqt
+
+  if (tid == 0) {
+    dev::mbar_init(dev::smem_u32(&sm.bar_kv), 1);
+    for (int s = 0; s < 2; ++s) {
+      dev::mbar_init(dev::smem_u32(&sm.bar_qfull[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_qempty[s]), 1);
+    }
+    dev::mbar_init(dev::smem_u32(&sm.bar_s), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_p), kT);
+    dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
+    sm.abort = 0;
+    dev::fence_barrier_init();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    dev::tma_prefetch_desc(&tm_q);
+    dev::tma_prefetch_desc(&tm_k);
+    dev::tma_prefetch_desc(&tm_v);
+    dev::tma_prefetch_desc(&tm_do);
+  }
+  if (warp == kMmaWarp) {
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == kLoadWarp) {
+    // ================================ TMA producer ================================
+    if (lane == 0 && nsteps > 0) {
+      const uint32_t bkv = dev::smem_u32(&sm.bar_kv);
+      dev::mbar_arrive_expect_tx(bkv, 2 * kTileBytes);
+      for (int half = 0; half < 2; ++half) {
+        dev::tma_load_3d(dev::smem_u32(sm.k) + half * kHalfBytes, &tm_k, bkv, half * 64, c0, bk);
+        dev::tma_load_3d(dev::smem_u32(sm.v) + half * kHalfBytes, &tm_v, bkv, half * 64, c0, bk);
+      }
+      int issued = 0;
+      for (int n = 0; n < nsteps; ++n) {
+        const int s = n & 1;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_qempty[s]), ((n >> 1) & 1) ^ 1, abort)) break;
+        const int hq = hk * p.G + n / nqt;
+        const int r0 = (qlo + n % nqt) * kT;
+        const uint32_t bq = dev::smem_u32(&sm.bar_qfull[s]);
+        const size_t vrow = static_cast<size_t>(b * p.Hq + hq) * p.npad + r0;
+        dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes + 2 * kT * 4);
+        for (int half = 0; half < 2; ++half) {
+          dev::tma_load_3d(dev::smem_u32(sm.q[s]) + half * kHalfBytes, &tm_q, bq, half * 64, r0,
+                           b * p.Hq + hq);
+          dev::tma_load_3d(dev::smem_u32(sm.dout[s]) + half * kHalfBytes, &tm_do, bq, half * 64,
+                           r0, b * p.Hq + hq);
+        }
+        bulk_load(dev::smem_u32(sm.lse2[s]), p.lse2 + vrow, kT * 4, bq);
+        bulk_load(dev::smem_u32(sm.dsum[s]), p.dsum + vrow, kT * 4, bq);
+        ++issued;
+      }
+      wait_drain(bkv, 0);
+      for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_qfull[s]), issued, s);
+    }
+  } else if (warp == kMmaWarp) {
+    // ============================= tcgen05.mma issuer ==============================
+    if (lane == 0 && nsteps > 0) {
+      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kT, 0, 0);  // both K-major
+      constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);  // A in TMEM, B MN-major
+      const uint32_t t_st = tmem, t_dpt = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 384;
+      const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
+      const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
+      uint64_t dqk[2], dok[2], dqm[2], dom[2];
+      for (int s = 0; s < 2; ++s) {
+        dqk[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), 16, 1024, dev::kSwizzle128B);
+        dok[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), 16, 1024, dev::kSwizzle128B);
+        dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+      }
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort);
+      for (int n = 0; ok && n < nsteps; ++n) {
+        const int s = n & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort))) break;
+        dev::tc_fence_after();
+        // S^T = K Q^T and dP^T = V dO^T (the previous step's dV/dK MMAs, which read the P^T
+        // and dS^T these overwrite, were issued earlier and complete first)
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+          dev::umma_ss(t_st, dka + koff, (s ? dqk[1] : dqk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+          dev::umma_ss(t_dpt, dva + koff, (s ? dok[1] : dok[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+        }
+        dev::umma_commit(dev::smem_u32(&sm.bar_s));
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p), n & 1, abort))) break;
+        dev::tc_fence_after();
+        // dV += P^T dO and dK += dS^T Q (K = the 128 queries of the tile, 16 per MMA)
+#pragma unroll
+        for (int ks = 0; ks < kT / 16; ++ks) {
+          const uint32_t acc = (n > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t boff = (ks * 16 * 128) >> 4;
+          dev::umma_ts(t_dv, t_st + ks * 8, (s ? dom[1] : dom[0]) + boff, idesc_tm, acc);
+          dev::umma_ts(t_dk, t_dpt + ks * 8, (s ? dqm[1] : dqm[0]) + boff, idesc_tm, acc);
+        }
+        dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));
+      }
+      if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
+      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+    }
+  } else {
+    // ========================== row workers: one key each ==========================
+    const int r = tid;  // TMEM lane = key c0 + r
+    const int j = c0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_st = tmem + lane_off, t_dpt = t_st + 128;
+    const float c = p.c;
+    bool ok = true;
+    for (int n = 0; n < nsteps; ++n) {
+      const int slot = n & 1;
+      const int r0 = (qlo + n % nqt) * kT;
+      // the stage's LSE / D vectors came with its Q and dO tiles; the stage cannot be refilled
+      // before this step's P^T and dS^T are released, so its phase is still this step's
+      ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[slot]), (n >> 1) & 1, abort) &&
+           wait_bounded(dev::smem_u32(&sm.bar_s), n & 1, abort);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      dev::tc_fence_after();
+
+      // visible query columns of key j in this tile (columns past Nq are zeroed by LSE = +inf)
+      const int P0 = r0 + off;
+      const bool full = block_full(p.mask, P0, c0);
+      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      if (!full) {
+        int lo = -1, hi = kT;
+        if (j >= p.mask.Nk) {
+          hi = -1;
+        } else if (p.mask.kind != ATTN_MASK_FULL) {
+          lo = clamp_col(static_cast<long long>(j) - P0);  // p >= j
+          if (p.mask.kind == ATTN_MASK_SLIDING && j >= p.mask.n_sink)
+            hi = clamp_col(static_cast<long long>(j) + p.mask.window - 1 - P0);  // p < j + w
+        }
+#pragma unroll
+        for (int w = 0; w < 4; ++w) vis[w] = cols_upto(hi, w) & ~cols_upto(lo - 1, w);
+      }
+      const float* l2v = sm.lse2[slot];
+      const float* ddv = sm.dsum[slot];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32], dr[32];
+        dev::tmem_ld32(t_st + cc * 32, sr);
+        dev::tmem_ld32(t_dpt + cc * 32, dr);
+        dev::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
+        uint32_t pk[16], dk16[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int col = cc * 32 + e;
+          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2v[col]));
+          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2v[col + 1]));
+          p0 = ((vis[cc] >> e) & 1u) ? p0 : 0.f;
+          p1 = ((vis[cc] >> (e + 1)) & 1u) ? p1 : 0.f;
+          const float d0 = p0 * (__uint_as_float(dr[e]) - ddv[col]);
+          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - ddv[col + 1]);
+          pk[e >> 1] = dev::pack_bf16x2(p0, p1);
+          dk16[e >> 1] = dev::pack_bf16x2(d0, d1);
+        }
+        // P^T over S^T and dS^T over dP^T, packed two per column: chunk cc fills columns
+        // [16cc, 16cc+16), which chunks 0..cc have already read
+        dev::tmem_st16(t_st + cc * 16, pk);
+        dev::tmem_st16(t_dpt + cc * 16, dk16);
+      }
+      dev::tmem_wait_st();
+      dev::tc_fence_before();
+      dev::mbar_arrive(dev::smem_u32(&sm.bar_p));
+    }
+
+    // ---- epilogue: dV and scale * dK rows of this CTA's keys, bf16 ----
+    const bool valid = j < p.Nk;
+    const size_t krow = static_cast<size_t>(bk) * p.Nk + j;
+    __nv_bfloat16* dst_v = p.dv + krow * kD;
+    __nv_bfloat16* dst_k = p.dk + krow * kD;
+    if (nsteps == 0) {
+      if (valid) {
+        store_zero_row(dst_v);
+        store_zero_row(dst_k);
+      }
+    } else if (ok) {
+      ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
+      if (__all_sync(0xffffffffu, ok)) {
+        dev::tc_fence_after();
+        store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid);
+        store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid);
+      }
+    }
+  }
+
+  // ---- teardown ----
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, 512);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// 3. dQ: one CTA per (b, query head, query tile)
+// ------------------------------------------------------------------------------------------
+struct __align__(1024) SmemQ {
+  uint8_t q[kTileBytes];
+  uint8_t dout[kTileBytes];
+  uint8_t k[2][kTileBytes];
+  uint8_t v[2][kTileBytes];
+  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s, bar_p, bar_done, bar_drain;
+  uint32_t tmem_base;
+  int abort;
+};
+constexpr size_t kSmemQBytes = sizeof(SmemQ) + 1024;
+
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_do, const Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemQ& sm = *reinterpret_cast<SmemQ*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                        ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+  // heaviest query tiles (causal) first
+  const int nbh = p.B * p.Hq;
+  const int qt = p.num_qtiles - 1 - static_cast<int>(blockIdx.x) / nbh;
+  const int bh = blockIdx.x % nbh;
+  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int bkv = b * p.Hkv + h / p.G;
+  const int r0 = qt * kT;
+  const int off = p.Nk - p.Nq;
+  const int last_row = min(r0 + kT, p.Nq) - 1;
+  const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kT);
+  const int nk = tr.count();
+
+  if (tid == 0) {
+    dev::mbar_init(dev::smem_u32(&sm.bar_q), 1);
+    for (int s = 0; s < 2; ++s) {
+      dev::mbar_init(dev::smem_u32(&sm.bar_kvfull[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_kvempty[s]), 1);
+    }
+    dev::mbar_init(dev::smem_u32(&sm.bar_s), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_p), kT);
+    dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
+    sm.abort = 0;
+    dev::fence_barrier_init();
+  }
+  if (warp == kLoadWarp && lane == 0) {
+    dev::tma_prefetch_desc(&tm_q);
+    dev::tma_prefetch_desc(&tm_k);
+    dev::tma_prefetch_desc(&tm_v);
+    dev::tma_prefetch_desc(&tm_do);
+  }
+  if (warp == kMmaWarp) {
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
+    dev::tmem_relinquish();
+  }
+  dev::tc_fence_before();
+  __syncthreads();
+  dev::tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  volatile int* abort = &sm.abort;
+
+  if (warp == kLoadWarp) {
+    // ================================ TMA producer ================================
+    if (lane == 0 && nk > 0) {
+      const uint32_t bq = dev::smem_u32(&sm.bar_q);
+      dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes);
+      for (int half = 0; half < 2; ++half) {
+        dev::tma_load_3d(dev::smem_u32(sm.q) + half * kHalfBytes, &tm_q, bq, half * 64, r0, bh);
+        dev::tma_load_3d(dev::smem_u32(sm.dout) + half * kHalfBytes, &tm_do, bq, half * 64, r0,
+                         bh);
+      }
+      int issued = 0;
+      for (int jj = 0; jj < nk; ++jj) {
+        const int s = jj & 1;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_kvempty[s]), ((jj >> 1) & 1) ^ 1, abort)) break;
+        const int key0 = tr.tile(jj) * kT;
+        const uint32_t bk = dev::smem_u32(&sm.bar_kvfull[s]);
+        dev::mbar_arrive_expect_tx(bk, 2 * kTileBytes);
+        for (int half = 0; half < 2; ++half) {
+          dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64, key0,
+                           bkv);
+          dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bk, half * 64, key0,
+                           bkv);
+        }
+        ++issued;
+      }
+      wait_drain(bq, 0);
+      for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_kvfull[s]), issued, s);
+    }
+  } else if (warp == kMmaWarp) {
+    // ============================= tcgen05.mma issuer ==============================
+    if (lane == 0 && nk > 0) {
+      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kT, 0, 0);
+      constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);
+      const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
+      const uint64_t dqa = dev::smem_desc(dev::smem_u32(sm.q), 16, 1024, dev::kSwizzle128B);
+      const uint64_t doa = dev::smem_desc(dev::smem_u32(sm.dout), 16, 1024, dev::kSwizzle128B);
+      uint64_t dkk[2], dvk[2], dkm[2];
+      for (int s = 0; s < 2; ++s) {
+        dkk[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), 16, 1024, dev::kSwizzle128B);
+        dvk[s] = dev::smem_desc(dev::smem_u32(sm.v[s]), 16, 1024, dev::kSwizzle128B);
+        dkm[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+      }
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
+      for (int jj = 0; ok && jj < nk; ++jj) {
+        const int s = jj & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort))) break;
+        dev::tc_fence_after();
+        // S = Q K^T and dP = dO V^T
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+          dev::umma_ss(t_s, dqa + koff, (s ? dkk[1] : dkk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+          dev::umma_ss(t_dp, doa + koff, (s ? dvk[1] : dvk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+        }
+        dev::umma_commit(dev::smem_u32(&sm.bar_s));
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p), jj & 1, abort))) break;
+        dev::tc_fence_after();
+        // dQ += dS K (K = the 128 keys of the tile, 16 per MMA)
+#pragma unroll
+        for (int ks = 0; ks < kT / 16; ++ks)
+          dev::umma_ts(t_dq, t_s + ks * 8, (s ? dkm[1] : dkm[0]) + ((ks * 16 * 128) >> 4),
+                       idesc_tm, (jj > 0 || ks > 0) ? 1u : 0u);
+        dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));
+      }
+      if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
+      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+    }
+  } else {
+    // ======================== row workers: one query row each ========================
+    const int r = tid;
+    const int i = r0 + r;
+    const int prow = i + off;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128;
+    const float c = p.c;
+    // padding rows (i >= Nq) hold LSE = +inf and D = 0: their weights are zero
+    const float l2 = p.lse2[static_cast<size_t>(bh) * p.npad + i];
+    const float dd = p.dsum[static_cast<size_t>(bh) * p.npad + i];
+    bool ok = true;
+    for (int jj = 0; jj < nk; ++jj) {
+      ok = wait_bounded(dev::smem_u32(&sm.bar_s), jj & 1, abort);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      dev::tc_fence_after();
+      const int key0 = tr.tile(jj) * kT;
+      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
+      if (!block_full(p.mask, r0 + off, key0)) {
+        // visible key columns of this row: col <= hi and (col >= lo or col < sk)
+        const long long last = p.mask.kind == ATTN_MASK_FULL ? p.mask.Nk - 1
+                                                             : min(prow, p.mask.Nk - 1);
+        const int hi = clamp_col(last - key0);
+        const bool sl = p.mask.kind == ATTN_MASK_SLIDING;
+        const int lo = sl ? clamp_col(static_cast<long long>(prow) - p.mask.window + 1 - key0) : -1;
+        const int sk = sl ? clamp_col(static_cast<long long>(p.mask.n_sink) - key0) : -1;
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          vis[w] = cols_upto(hi, w) & (~cols_upto(lo - 1, w) | cols_upto(sk - 1, w));
+      }
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t sr[32], dr[32];
+        dev::tmem_ld32(t_s + cc * 32, sr);
+        dev::tmem_ld32(t_dp + cc * 32, dr);
+        dev::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2));
+          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2));
+          p0 = ((vis[cc] >> e) & 1u) ? p0 : 0.f;
+          p1 = ((vis[cc] >> (e + 1)) & 1u) ? p1 : 0.f;
+          pk[e >> 1] = dev::pack_bf16x2(p0 * (__uint_as_float(dr[e]) - dd),
+                                        p1 * (__uint_as_float(dr[e + 1]) - dd));
+        }
+        dev::tmem_st16(t_s + cc * 16, pk);  // dS over S (see the dK/dV kernel)
+      }
+      dev::tmem_wait_st();
+      dev::tc_fence_before();
+      dev::mbar_arrive(dev::smem_u32(&sm.bar_p));
+    }
+
+    // ---- epilogue: scale * dQ row, bf16 ----
+    const bool valid = i < p.Nq;
+    __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
+    if (nk == 0) {
+      if (valid) store_zero_row(dst);
+    } else if (ok) {
+      ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
+      if (__all_sync(0xffffffffu, ok)) {
+        dev::tc_fence_after();
+        store_acc_row(tmem + lane_off + 256, p.scale, dst, valid);
+      }
+    }
+  }
+
+  // ---- teardown ----
+  dev::tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    dev::tc_fence_after();
+    dev::tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace bwd
+}  // namespace attn

@@ -121,6 +121,29 @@ ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float 
                  float scale, attn_stream_t stream);
 
 /*
+ * attn_bwd - backward pass of attn_fwd: dQ, dK, dV for a given dO, recomputing the attention
+ * weights from the forward's LSE instead of storing them ("Quadratic Complexity Bottleneck",
+ * FlashAttention section: the backward pass recomputes attention; "Chapter 3.1 - The Cost of
+ * Attention", section 5).  With P_ij = exp(scale q_i.k_j - LSE_i) on visible pairs:
+ *   dV_j = sum_i P_ij dO_i,  dS_ij = P_ij (dO_i.v_j - dO_i.O_i),
+ *   dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j  (GQA: dK, dV sum over the group).
+ *   q, o, dout, dq  bf16 [B][Hq][Nq][d];  k, v, dk, dv  bf16 [B][Hkv][Nk][d];
+ *   lse  fp32 [B][Hq][Nq], the forward's LSE for the same inputs, mask and scale (required).
+ *   d == 128; mask, window, n_sink, scale as attn_fwd.  dq, dk, dv are fully written (rows and
+ *   keys that see nothing get zeros).
+ *   workspace: device scratch of at least attn_bwd_workspace_bytes(B, Hq, Nq) bytes, 16-byte
+ *   aligned, overwritten before it is read.
+ * Errors: as attn_fwd; ATTN_ERR_WORKSPACE for a missing or short workspace.  Three kernels are
+ * queued on `stream`; the result does not depend on their scheduling (no atomics).
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
+
+ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
+                      const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,
+                      int Nq, int Nk, int d, int mask_kind, int window, int n_sink, float scale,
+                      void *workspace, size_t workspace_bytes, attn_stream_t stream);
+
+/*
  * Decode: one new query token per sequence against a contiguous KV cache, split-K over the
  * keys with a log-sum-exp combine ("Attention Research", section 2: split-K over keys for
  * decode; "Quadratic Complexity Bottleneck", KV cache).  Every cached key is visible.

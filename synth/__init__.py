@@ -22,6 +22,7 @@ from __future__ import annotations
 import numpy as np
 
 Q_ID, K_ID, V_ID = 0, 1, 2
+DO_ID = 3  # dL/dO of the backward pass
 
 _GOLDEN = 0x9E3779B97F4A7C15
 _M1 = 0xBF58476D1CE4E5B9

@@ -113,3 +113,26 @@ def test_paged_decode_invalid_arguments_are_rejected(lib):
     assert paged(lib, k=N) == E
     assert paged(lib, splits=-1) == E
     assert paged(lib, scale=float("nan")) == E
+
+
+def bwd(lib, q=P, k=P, v=P, o=P, lse=P, do=P, dq=P, dk=P, dv=P, B=1, Hq=2, Hkv=1, Nq=4, Nk=4,
+        d=128, mask=1, w=0, s=0, scale=0.1, ws=P, ws_bytes=1 << 20):
+    return lib.attn_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, mask, w, s, scale,
+                        ws, ws_bytes, N)
+
+
+def test_bwd_invalid_arguments_are_rejected(lib):
+    E = A.ATTN_ERR_INVALID_ARG
+    for name in ("q", "k", "v", "o", "lse", "do", "dq", "dk", "dv"):
+        assert bwd(lib, **{name: N}) == E, name
+    assert bwd(lib, B=-1) == E
+    assert bwd(lib, Hq=3, Hkv=2) == E
+    assert bwd(lib, mask=2, w=0) == E
+    assert bwd(lib, scale=float("nan")) == E
+    assert bwd(lib, d=64) == A.ATTN_ERR_UNSUPPORTED
+
+
+def test_bwd_workspace_size():
+    assert A.attn_bwd_workspace_bytes(4, 16, 2048) == 2 * 4 * 16 * 2048 * 4
+    assert A.attn_bwd_workspace_bytes(1, 2, 300) == 2 * 1 * 2 * 384 * 4  # rows padded to 128
+    assert A.attn_bwd_workspace_bytes(0, 2, 300) == 0
