@@ -25,8 +25,9 @@
 // instead of 5) but needs neither atomics nor a second accumulator set, and the result does not
 // depend on the order in which CTAs finish.
 //
-// Roles of each 192-thread CTA: warps 0-3 are the row workers (thread t owns TMEM lane t), warp
-// 4 issues every tcgen05.mma from one thread, warp 5 issues the TMA copies from one thread.
+// Roles of each 320-thread CTA: warps 0-7 are the row workers (warps w and w+4 share TMEM lanes
+// 32(w%4) .. 32(w%4)+31 and split the columns), warp 8 issues every tcgen05.mma from one thread,
+// warp 9 issues the TMA copies from one thread.
 // Tensor memory (512 columns): [0,128) S or S^T, [128,256) dP or dP^T, [256,384) dV or dQ,
 // [384,512) dK.  Every wait is bounded (see common.cuh).
 #pragma once
@@ -41,9 +42,10 @@ namespace bwd {
 
 constexpr int kT = 128;  // tile rows and columns (queries and keys)
 constexpr int kD = 128;  // head dimension
-constexpr int kThreads = 192;
-constexpr int kMmaWarp = 4;
-constexpr int kLoadWarp = 5;
+constexpr int kRowThreads = 256;  // warps 0-7: two warps per TMEM lane quarter
+constexpr int kThreads = kRowThreads + 64;
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
 constexpr uint32_t kTileBytes = kT * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kT * 64 * 2;  // one 128-byte-swizzled 64-column half
 constexpr float kLog2e = 1.4426950408889634f;
@@ -74,15 +76,16 @@ __device__ __forceinline__ uint32_t cols_upto(int x, int w) {
   return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
 }
 
-// clamp a 64-bit column bound into [-1, 128] (every bound outside the tile acts the same)
+// clamp a 64-bit column bound into [-1, 128] (every bound outside a tile acts the same)
 __device__ __forceinline__ int clamp_col(long long x) {
   return x < -1 ? -1 : (x > kT ? kT : static_cast<int>(x));
 }
 
-// Is every pair of the block (query positions P0 .. P0+127) x (keys c0 .. c0+127) visible?
-// Conservative: rows past Nq count as visible here (their weights are zero through LSE = +inf).
-__device__ __forceinline__ bool block_full(const MaskSpec& m, int P0, int c0) {
-  const int c1 = c0 + kT - 1, P1 = P0 + kT - 1;
+// Is every pair of the block (query positions P0 .. P0+rows-1) x (keys c0 .. c0+cols-1)
+// visible?  Conservative: rows past Nq count as visible here (their weights are zero through
+// LSE = +inf).
+__device__ __forceinline__ bool block_full(const MaskSpec& m, int P0, int rows, int c0, int cols) {
+  const int c1 = c0 + cols - 1, P1 = P0 + rows - 1;
   if (c1 >= m.Nk) return false;
   if (m.kind == ATTN_MASK_FULL) return true;
   if (c1 > P0) return false;
@@ -128,11 +131,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Row r of a 128 x 128 fp32 accumulator in TMEM -> bf16 row of global memory (times mul).
+// Columns [64 ch, 64 ch + 64) of row r of a 128 x 128 fp32 accumulator in TMEM -> bf16 in
+// global memory (times mul).
 __device__ __forceinline__ void store_acc_row(uint32_t t_acc, float mul, __nv_bfloat16* dst,
-                                              bool valid) {
+                                              bool valid, int ch) {
 #pragma unroll 1
-  for (int cc = 0; cc < 4; ++cc) {
+  for (int cc = 2 * ch; cc < 2 * ch + 2; ++cc) {
     uint32_t a[32];
     dev::tmem_ld32(t_acc + cc * 32, a);
     dev::tmem_wait_ld_regs(a);
@@ -149,11 +153,17 @@ __device__ __forceinline__ void store_acc_row(uint32_t t_acc, float mul, __nv_bf
   }
 }
 
-__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int ch) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 64);
 #pragma unroll
-  for (int i = 0; i < kD / 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = 0; i < 8; ++i) d4[i] = make_uint4(0u, 0u, 0u, 0u);
 }
+
+// Packed bf16 weights of a 64-column sub-step live where each column half was read: columns
+// [0, 32) pack into TMEM columns [0, 16), columns [32, 64) into [32, 48), so neither warp of a
+// lane quarter overwrites scores the other has yet to load.  K-step ks (16 columns) of the
+// accumulating MMA therefore starts at column:
+__device__ __forceinline__ uint32_t packed_col(int ks) { return ks * 8 + (ks >= 2 ? 16 : 0); }
 
 // ------------------------------------------------------------------------------------------
 // 1. D_i = dO_i . O_i and LSE_i * log2(e): one warp per query row
@@ -192,6 +202,19 @@ __global__ void __launch_bounds__(256)
 }
 
 // ------------------------------------------------------------------------------------------
+// The two main kernels run the same software pipeline over sub-steps of 64 rows: sub-step m is
+// half h = m & 1 of tile step m >> 1, and its two score-like products (S and dP, 128 x 64 fp32)
+// go to TMEM buffer m & 1.  The MMA thread issues them two sub-steps ahead, so the tensor core
+// computes sub-step m+1 (and the accumulating products of m-1) while the row warps turn
+// sub-step m into bf16 weights; a buffer is overwritten only by MMAs issued after the
+// accumulating MMAs that read it (tcgen05 MMAs of one thread execute in issue order).
+// Tensor memory: S buffers at columns [0,64) and [64,128), dP buffers at [128,192) and
+// [192,256), accumulators at [256,384) (dV or dQ) and [384,512) (dK).
+// ------------------------------------------------------------------------------------------
+constexpr int kSub = 64;                         // rows of a sub-step (columns of its scores)
+constexpr uint32_t kSubBytes = kSub * 128;       // rows of a sub-step inside one 64-column half
+
+// ------------------------------------------------------------------------------------------
 // 2. dK, dV: one CTA per (b, kv head, key block)
 // ------------------------------------------------------------------------------------------
 struct __align__(1024) SmemKV {
@@ -201,7 +224,7 @@ struct __align__(1024) SmemKV {
   uint8_t dout[2][kTileBytes];
   float lse2[2][kT];  // per stage: the query tile's LSE * log2(e) and D, copied with Q and dO
   float dsum[2][kT];
-  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s, bar_p, bar_done, bar_drain;
+  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_done, bar_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -229,15 +252,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   query_tiles(p.mask, c0, c1, off, p.Nq, qlo, qhi);
   const int nqt = qhi >= qlo ? qhi - qlo + 1 : 0;
   const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qlo + n % nqt
+  const int nsub = 2 * nsteps;
 
   if (tid == 0) {
     dev::mbar_init(dev::smem_u32(&sm.bar_kv), 1);
     for (int s = 0; s < 2; ++s) {
       dev::mbar_init(dev::smem_u32(&sm.bar_qfull[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_qempty[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
     }
-    dev::mbar_init(dev::smem_u32(&sm.bar_s), 1);
-    dev::mbar_init(dev::smem_u32(&sm.bar_p), kT);
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
     dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
@@ -293,9 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ============================= tcgen05.mma issuer ==============================
     if (lane == 0 && nsteps > 0) {
-      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kT, 0, 0);  // both K-major
-      constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);  // A in TMEM, B MN-major
-      const uint32_t t_st = tmem, t_dpt = tmem + 128, t_dv = tmem + 256, t_dk = tmem + 384;
+      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);  // both K-major, N = 64
+      constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);    // A in TMEM, B MN-major
       const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
       const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
       uint64_t dqk[2], dok[2], dqm[2], dom[2];
@@ -305,63 +328,82 @@ __global__ void __launch_bounds__(kThreads, 1)
         dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
         dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
       }
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort);
-      for (int n = 0; ok && n < nsteps; ++n) {
-        const int s = n & 1;
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort))) break;
+      // S^T = K Q_h^T and dP^T = V dO_h^T for sub-step m (queries 64h .. 64h+63 of its tile)
+      auto issue_scores = [&](int m) {
+        const int n = m >> 1, h = m & 1, s = n & 1;
+        if (h == 0 && !wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort))
+          return false;
         dev::tc_fence_after();
-        // S^T = K Q^T and dP^T = V dO^T (the previous step's dV/dK MMAs, which read the P^T
-        // and dS^T these overwrite, were issued earlier and complete first)
+        const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+        const uint32_t hoff = (h * kSubBytes) >> 4;
+        const uint64_t bq = (s ? dqk[1] : dqk[0]) + hoff, bo = (s ? dok[1] : dok[0]) + hoff;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_st, dka + koff, (s ? dqk[1] : dqk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          dev::umma_ss(t_st, dka + koff, bq + koff, idesc_kk, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_dpt, dva + koff, (s ? dok[1] : dok[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          dev::umma_ss(t_dpt, dva + koff, bo + koff, idesc_kk, ks > 0 ? 1u : 0u);
         }
-        dev::umma_commit(dev::smem_u32(&sm.bar_s));
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p), n & 1, abort))) break;
+        dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
+        return true;
+      };
+      // dV += P^T dO_h and dK += dS^T Q_h (K = the 64 queries of the sub-step)
+      auto issue_grads = [&](int m) {
+        const int n = m >> 1, h = m & 1, s = n & 1;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort)) return false;
         dev::tc_fence_after();
-        // dV += P^T dO and dK += dS^T Q (K = the 128 queries of the tile, 16 per MMA)
+        const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+        const uint64_t bo = s ? dom[1] : dom[0], bq = s ? dqm[1] : dqm[0];
 #pragma unroll
-        for (int ks = 0; ks < kT / 16; ++ks) {
-          const uint32_t acc = (n > 0 || ks > 0) ? 1u : 0u;
-          const uint32_t boff = (ks * 16 * 128) >> 4;
-          dev::umma_ts(t_dv, t_st + ks * 8, (s ? dom[1] : dom[0]) + boff, idesc_tm, acc);
-          dev::umma_ts(t_dk, t_dpt + ks * 8, (s ? dqm[1] : dqm[0]) + boff, idesc_tm, acc);
+        for (int ks = 0; ks < kSub / 16; ++ks) {
+          const uint32_t acc = (m > 0 || ks > 0) ? 1u : 0u;
+          const uint32_t boff = (h * kSubBytes + ks * 16 * 128) >> 4;
+          dev::umma_ts(tmem + 256, t_st + packed_col(ks), bo + boff, idesc_tm, acc);
+          dev::umma_ts(tmem + 384, t_dpt + packed_col(ks), bq + boff, idesc_tm, acc);
         }
-        dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));
+        if (h == 1) dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));  // stage s read for good
+        return true;
+      };
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort) && issue_scores(0) &&
+                issue_scores(1);
+      for (int m = 0; ok && m < nsub; ++m) {
+        ok = issue_grads(m);
+        if (ok && m + 2 < nsub) ok = issue_scores(m + 2);
       }
       if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
       wait_drain(dev::smem_u32(&sm.bar_drain), 0);
     }
   } else {
-    // ========================== row workers: one key each ==========================
-    const int r = tid;  // TMEM lane = key c0 + r
+    // ============== row workers: one key each, two warps per key (column halves) ==============
+    const int r = (warp & 3) * 32 + lane;  // TMEM lane = key c0 + r
+    const int ch = warp >> 2;              // this warp's 32 of the 64 columns of a sub-step
     const int j = c0 + r;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_st = tmem + lane_off, t_dpt = t_st + 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.c;
     bool ok = true;
-    for (int n = 0; n < nsteps; ++n) {
-      const int slot = n & 1;
-      const int r0 = (qlo + n % nqt) * kT;
+    for (int m = 0; m < nsub; ++m) {
+      const int n = m >> 1, h = m & 1, s = n & 1;
+      const int r0 = (qlo + n % nqt) * kT + h * kSub;  // first query row of the sub-step
       // the stage's LSE / D vectors came with its Q and dO tiles; the stage cannot be refilled
-      // before this step's P^T and dS^T are released, so its phase is still this step's
-      ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[slot]), (n >> 1) & 1, abort) &&
-           wait_bounded(dev::smem_u32(&sm.bar_s), n & 1, abort);
+      // before this tile's weights are released, so its phase is still this tile's
+      ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort) &&
+           wait_bounded(dev::smem_u32(&sm.bar_s[m & 1]), (m >> 1) & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       dev::tc_fence_after();
+      const uint32_t t_st = tmem + lane_off + (m & 1) * kSub + ch * 32;
+      const uint32_t t_dpt = tmem + lane_off + 128 + (m & 1) * kSub + ch * 32;
+      uint32_t sr[32], dr[32];
+      dev::tmem_ld32(t_st, sr);
+      dev::tmem_ld32(t_dpt, dr);
 
-      // visible query columns of key j in this tile (columns past Nq are zeroed by LSE = +inf)
+      // visible query columns of key j among this warp's 32 (columns past Nq: LSE = +inf)
       const int P0 = r0 + off;
-      const bool full = block_full(p.mask, P0, c0);
-      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
-      if (!full) {
+      uint32_t vis = ~0u;
+      if (!block_full(p.mask, P0, kSub, c0, kT)) {
         int lo = -1, hi = kT;
         if (j >= p.mask.Nk) {
           hi = -1;
@@ -370,58 +412,56 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (p.mask.kind == ATTN_MASK_SLIDING && j >= p.mask.n_sink)
             hi = clamp_col(static_cast<long long>(j) + p.mask.window - 1 - P0);  // p < j + w
         }
-#pragma unroll
-        for (int w = 0; w < 4; ++w) vis[w] = cols_upto(hi, w) & ~cols_upto(lo - 1, w);
+        vis = cols_upto(hi, ch) & ~cols_upto(lo - 1, ch);
       }
-      const float* l2v = sm.lse2[slot];
-      const float* ddv = sm.dsum[slot];
+      const float4* l2v = reinterpret_cast<const float4*>(sm.lse2[s] + h * kSub + ch * 32);
+      const float4* ddv = reinterpret_cast<const float4*>(sm.dsum[s] + h * kSub + ch * 32);
+      dev::tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], dr[32];
-        dev::tmem_ld32(t_st + cc * 32, sr);
-        dev::tmem_ld32(t_dpt + cc * 32, dr);
-        dev::tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
+      uint32_t pk[16], dk16[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
-        uint32_t pk[16], dk16[16];
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const float4 l4 = l2v[e4], d4 = ddv[e4];
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int col = cc * 32 + e;
-          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2v[col]));
-          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2v[col + 1]));
-          p0 = ((vis[cc] >> e) & 1u) ? p0 : 0.f;
-          p1 = ((vis[cc] >> (e + 1)) & 1u) ? p1 : 0.f;
-          const float d0 = p0 * (__uint_as_float(dr[e]) - ddv[col]);
-          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - ddv[col + 1]);
+        for (int e2 = 0; e2 < 4; e2 += 2) {
+          const int e = e4 * 4 + e2;
+          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -lv[e2]));
+          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e2 + 1]));
+          p0 = ((vis >> e) & 1u) ? p0 : 0.f;
+          p1 = ((vis >> (e + 1)) & 1u) ? p1 : 0.f;
+          const float d0 = p0 * (__uint_as_float(dr[e]) - dvv[e2]);
+          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - dvv[e2 + 1]);
           pk[e >> 1] = dev::pack_bf16x2(p0, p1);
           dk16[e >> 1] = dev::pack_bf16x2(d0, d1);
         }
-        // P^T over S^T and dS^T over dP^T, packed two per column: chunk cc fills columns
-        // [16cc, 16cc+16), which chunks 0..cc have already read
-        dev::tmem_st16(t_st + cc * 16, pk);
-        dev::tmem_st16(t_dpt + cc * 16, dk16);
       }
+      // P^T over S^T and dS^T over dP^T, packed into the first 16 of the 32 columns this warp
+      // has just read (see packed_col)
+      dev::tmem_st16(t_st, pk);
+      dev::tmem_st16(t_dpt, dk16);
       dev::tmem_wait_st();
       dev::tc_fence_before();
-      dev::mbar_arrive(dev::smem_u32(&sm.bar_p));
+      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
     }
 
-    // ---- epilogue: dV and scale * dK rows of this CTA's keys, bf16 ----
+    // ---- epilogue: dV and scale * dK rows of this CTA's keys, bf16, a column half per warp ----
     const bool valid = j < p.Nk;
     const size_t krow = static_cast<size_t>(bk) * p.Nk + j;
     __nv_bfloat16* dst_v = p.dv + krow * kD;
     __nv_bfloat16* dst_k = p.dk + krow * kD;
     if (nsteps == 0) {
       if (valid) {
-        store_zero_row(dst_v);
-        store_zero_row(dst_k);
+        store_zero_row(dst_v, ch);
+        store_zero_row(dst_k, ch);
       }
     } else if (ok) {
       ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
       if (__all_sync(0xffffffffu, ok)) {
         dev::tc_fence_after();
-        store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid);
-        store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid);
+        store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid, ch);
+        store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid, ch);
       }
     }
   }
@@ -443,7 +483,7 @@ struct __align__(1024) SmemQ {
   uint8_t dout[kTileBytes];
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
-  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s, bar_p, bar_done, bar_drain;
+  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s[2], bar_p[2], bar_done, bar_drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -470,15 +510,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int last_row = min(r0 + kT, p.Nq) - 1;
   const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kT);
   const int nk = tr.count();
+  const int nsub = 2 * nk;
 
   if (tid == 0) {
     dev::mbar_init(dev::smem_u32(&sm.bar_q), 1);
     for (int s = 0; s < 2; ++s) {
       dev::mbar_init(dev::smem_u32(&sm.bar_kvfull[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_kvempty[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
     }
-    dev::mbar_init(dev::smem_u32(&sm.bar_s), 1);
-    dev::mbar_init(dev::smem_u32(&sm.bar_p), kT);
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
     dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
@@ -531,9 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ============================= tcgen05.mma issuer ==============================
     if (lane == 0 && nk > 0) {
-      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kT, 0, 0);
+      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);
       constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);
-      const uint32_t t_s = tmem, t_dp = tmem + 128, t_dq = tmem + 256;
       const uint64_t dqa = dev::smem_desc(dev::smem_u32(sm.q), 16, 1024, dev::kSwizzle128B);
       const uint64_t doa = dev::smem_desc(dev::smem_u32(sm.dout), 16, 1024, dev::kSwizzle128B);
       uint64_t dkk[2], dvk[2], dkm[2];
@@ -542,55 +582,77 @@ __global__ void __launch_bounds__(kThreads, 1)
         dvk[s] = dev::smem_desc(dev::smem_u32(sm.v[s]), 16, 1024, dev::kSwizzle128B);
         dkm[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
       }
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
-      for (int jj = 0; ok && jj < nk; ++jj) {
-        const int s = jj & 1;
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort))) break;
+      // S = Q K_h^T and dP = dO V_h^T for sub-step m (keys 64h .. 64h+63 of its key tile)
+      auto issue_scores = [&](int m) {
+        const int jj = m >> 1, hh = m & 1, s = jj & 1;
+        if (hh == 0 && !wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort))
+          return false;
         dev::tc_fence_after();
-        // S = Q K^T and dP = dO V^T
+        const uint32_t t_s = tmem + (m & 1) * kSub, t_dp = tmem + 128 + (m & 1) * kSub;
+        const uint32_t hoff = (hh * kSubBytes) >> 4;
+        const uint64_t bk = (s ? dkk[1] : dkk[0]) + hoff, bv = (s ? dvk[1] : dvk[0]) + hoff;
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_s, dqa + koff, (s ? dkk[1] : dkk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          dev::umma_ss(t_s, dqa + koff, bk + koff, idesc_kk, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
           const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_dp, doa + koff, (s ? dvk[1] : dvk[0]) + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          dev::umma_ss(t_dp, doa + koff, bv + koff, idesc_kk, ks > 0 ? 1u : 0u);
         }
-        dev::umma_commit(dev::smem_u32(&sm.bar_s));
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p), jj & 1, abort))) break;
+        dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
+        return true;
+      };
+      // dQ += dS K_h (K = the 64 keys of the sub-step)
+      auto issue_grads = [&](int m) {
+        const int jj = m >> 1, hh = m & 1, s = jj & 1;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort)) return false;
         dev::tc_fence_after();
-        // dQ += dS K (K = the 128 keys of the tile, 16 per MMA)
+        const uint32_t t_s = tmem + (m & 1) * kSub;
+        const uint64_t bk = s ? dkm[1] : dkm[0];
 #pragma unroll
-        for (int ks = 0; ks < kT / 16; ++ks)
-          dev::umma_ts(t_dq, t_s + ks * 8, (s ? dkm[1] : dkm[0]) + ((ks * 16 * 128) >> 4),
-                       idesc_tm, (jj > 0 || ks > 0) ? 1u : 0u);
-        dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));
+        for (int ks = 0; ks < kSub / 16; ++ks)
+          dev::umma_ts(tmem + 256, t_s + packed_col(ks),
+                       bk + ((hh * kSubBytes + ks * 16 * 128) >> 4), idesc_tm,
+                       (m > 0 || ks > 0) ? 1u : 0u);
+        if (hh == 1) dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));  // stage s read for good
+        return true;
+      };
+      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort) && issue_scores(0) &&
+                issue_scores(1);
+      for (int m = 0; ok && m < nsub; ++m) {
+        ok = issue_grads(m);
+        if (ok && m + 2 < nsub) ok = issue_scores(m + 2);
       }
       if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
       wait_drain(dev::smem_u32(&sm.bar_drain), 0);
     }
   } else {
-    // ======================== row workers: one query row each ========================
-    const int r = tid;
+    // ========= row workers: one query row each, two warps per row (column halves) =========
+    const int r = (warp & 3) * 32 + lane;
+    const int ch = warp >> 2;
     const int i = r0 + r;
     const int prow = i + off;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_off, t_dp = t_s + 128;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.c;
     // padding rows (i >= Nq) hold LSE = +inf and D = 0: their weights are zero
     const float l2 = p.lse2[static_cast<size_t>(bh) * p.npad + i];
     const float dd = p.dsum[static_cast<size_t>(bh) * p.npad + i];
     bool ok = true;
-    for (int jj = 0; jj < nk; ++jj) {
-      ok = wait_bounded(dev::smem_u32(&sm.bar_s), jj & 1, abort);
+    for (int m = 0; m < nsub; ++m) {
+      ok = wait_bounded(dev::smem_u32(&sm.bar_s[m & 1]), (m >> 1) & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       dev::tc_fence_after();
-      const int key0 = tr.tile(jj) * kT;
-      uint32_t vis[4] = {~0u, ~0u, ~0u, ~0u};
-      if (!block_full(p.mask, r0 + off, key0)) {
+      const uint32_t t_s = tmem + lane_off + (m & 1) * kSub + ch * 32;
+      const uint32_t t_dp = tmem + lane_off + 128 + (m & 1) * kSub + ch * 32;
+      uint32_t sr[32], dr[32];
+      dev::tmem_ld32(t_s, sr);
+      dev::tmem_ld32(t_dp, dr);
+      const int key0 = tr.tile(m >> 1) * kT + (m & 1) * kSub;  // first key of the sub-step
+      uint32_t vis = ~0u;
+      if (!block_full(p.mask, r0 + off, kT, key0, kSub)) {
         // visible key columns of this row: col <= hi and (col >= lo or col < sk)
         const long long last = p.mask.kind == ATTN_MASK_FULL ? p.mask.Nk - 1
                                                              : min(prow, p.mask.Nk - 1);
@@ -598,45 +660,37 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool sl = p.mask.kind == ATTN_MASK_SLIDING;
         const int lo = sl ? clamp_col(static_cast<long long>(prow) - p.mask.window + 1 - key0) : -1;
         const int sk = sl ? clamp_col(static_cast<long long>(p.mask.n_sink) - key0) : -1;
-#pragma unroll
-        for (int w = 0; w < 4; ++w)
-          vis[w] = cols_upto(hi, w) & (~cols_upto(lo - 1, w) | cols_upto(sk - 1, w));
+        vis = cols_upto(hi, ch) & (~cols_upto(lo - 1, ch) | cols_upto(sk - 1, ch));
       }
+      dev::tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sr[32], dr[32];
-        dev::tmem_ld32(t_s + cc * 32, sr);
-        dev::tmem_ld32(t_dp + cc * 32, dr);
-        dev::tmem_wait_ld();
+      for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
+      uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2));
-          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2));
-          p0 = ((vis[cc] >> e) & 1u) ? p0 : 0.f;
-          p1 = ((vis[cc] >> (e + 1)) & 1u) ? p1 : 0.f;
-          pk[e >> 1] = dev::pack_bf16x2(p0 * (__uint_as_float(dr[e]) - dd),
-                                        p1 * (__uint_as_float(dr[e + 1]) - dd));
-        }
-        dev::tmem_st16(t_s + cc * 16, pk);  // dS over S (see the dK/dV kernel)
+      for (int e = 0; e < 32; e += 2) {
+        float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2));
+        float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2));
+        p0 = ((vis >> e) & 1u) ? p0 : 0.f;
+        p1 = ((vis >> (e + 1)) & 1u) ? p1 : 0.f;
+        pk[e >> 1] = dev::pack_bf16x2(p0 * (__uint_as_float(dr[e]) - dd),
+                                      p1 * (__uint_as_float(dr[e + 1]) - dd));
       }
+      dev::tmem_st16(t_s, pk);  // dS over S (see packed_col)
       dev::tmem_wait_st();
       dev::tc_fence_before();
-      dev::mbar_arrive(dev::smem_u32(&sm.bar_p));
+      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
     }
 
-    // ---- epilogue: scale * dQ row, bf16 ----
+    // ---- epilogue: scale * dQ row, bf16, a column half per warp ----
     const bool valid = i < p.Nq;
     __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
     if (nk == 0) {
-      if (valid) store_zero_row(dst);
+      if (valid) store_zero_row(dst, ch);
     } else if (ok) {
       ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
       if (__all_sync(0xffffffffu, ok)) {
         dev::tc_fence_after();
-        store_acc_row(tmem + lane_off + 256, p.scale, dst, valid);
+        store_acc_row(tmem + lane_off + 256, p.scale, dst, valid, ch);
       }
     }
   }
