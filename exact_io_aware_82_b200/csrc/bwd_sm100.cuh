@@ -25,9 +25,9 @@
 // instead of 5) but needs neither atomics nor a second accumulator set, and the result does not
 // depend on the order in which CTAs finish.
 //
-// Roles of each 320-thread CTA: warps 0-7 are the row workers (warps w and w+4 share TMEM lanes
-// 32(w%4) .. 32(w%4)+31 and split the columns), warp 8 issues every tcgen05.mma from one thread,
-// warp 9 issues the TMA copies from one thread.
+// Roles of each 352-thread CTA: warps 0-7 are the row workers (warps w and w+4 share TMEM lanes
+// 32(w%4) .. 32(w%4)+31 and split the columns), one thread of warp 8 issues the score MMAs, one
+// thread of warp 10 the accumulating MMAs, and one thread of warp 9 the TMA copies.
 // Tensor memory (512 columns): [0,128) S or S^T, [128,256) dP or dP^T, [256,384) dV or dQ,
 // [384,512) dK.  Every wait is bounded (see common.cuh).
 #pragma once
@@ -43,9 +43,10 @@ namespace bwd {
 constexpr int kT = 128;  // tile rows and columns (queries and keys)
 constexpr int kD = 128;  // head dimension
 constexpr int kRowThreads = 256;  // warps 0-7: two warps per TMEM lane quarter
-constexpr int kThreads = kRowThreads + 64;
-constexpr int kMmaWarp = 8;
+constexpr int kThreads = kRowThreads + 96;
+constexpr int kMmaWarp = 8;    // issues the score MMAs (S, dP)
 constexpr int kLoadWarp = 9;
+constexpr int kGradWarp = 10;  // issues the accumulating MMAs (dV, dK or dQ)
 constexpr uint32_t kTileBytes = kT * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kT * 64 * 2;  // one 128-byte-swizzled 64-column half
 constexpr float kLog2e = 1.4426950408889634f;
@@ -204,10 +205,11 @@ __global__ void __launch_bounds__(256)
 // ------------------------------------------------------------------------------------------
 // The two main kernels run the same software pipeline over sub-steps of 64 rows: sub-step m is
 // half h = m & 1 of tile step m >> 1, and its two score-like products (S and dP, 128 x 64 fp32)
-// go to TMEM buffer m & 1.  The MMA thread issues them two sub-steps ahead, so the tensor core
-// computes sub-step m+1 (and the accumulating products of m-1) while the row warps turn
-// sub-step m into bf16 weights; a buffer is overwritten only by MMAs issued after the
-// accumulating MMAs that read it (tcgen05 MMAs of one thread execute in issue order).
+// go to TMEM buffer m & 1.  One thread issues those score MMAs as soon as their buffer is free
+// (the accumulating MMAs of sub-step m-2, which read the bf16 weights stored there, have
+// completed: barrier bar_free), another issues the accumulating MMAs of a sub-step as soon as
+// the row warps have released its weights, so the tensor core computes sub-step m+1 (and the
+// accumulating products of m-1) while the row warps turn sub-step m into bf16 weights.
 // Tensor memory: S buffers at columns [0,64) and [64,128), dP buffers at [128,192) and
 // [192,256), accumulators at [256,384) (dV or dQ) and [384,512) (dK).
 // ------------------------------------------------------------------------------------------
@@ -224,7 +226,8 @@ struct __align__(1024) SmemKV {
   uint8_t dout[2][kTileBytes];
   float lse2[2][kT];  // per stage: the query tile's LSE * log2(e) and D, copied with Q and dO
   float dsum[2][kT];
-  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_done, bar_drain;
+  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_free[2], bar_done;
+  uint64_t bar_drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -261,9 +264,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(dev::smem_u32(&sm.bar_qempty[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
+      dev::mbar_init(dev::smem_u32(&sm.bar_free[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_drain[s]), 1);
     }
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
-    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
     dev::fence_barrier_init();
   }
@@ -314,68 +318,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(bkv, 0);
       for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_qfull[s]), issued, s);
     }
-  } else if (warp == kMmaWarp) {
-    // ============================= tcgen05.mma issuer ==============================
+  } else if (warp == kMmaWarp || warp == kGradWarp) {
+    // ========================= tcgen05.mma issuers (two threads) ==========================
     if (lane == 0 && nsteps > 0) {
       constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);  // both K-major, N = 64
       constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);    // A in TMEM, B MN-major
-      const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
-      const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
-      uint64_t dqk[2], dok[2], dqm[2], dom[2];
-      for (int s = 0; s < 2; ++s) {
-        dqk[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), 16, 1024, dev::kSwizzle128B);
-        dok[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), 16, 1024, dev::kSwizzle128B);
-        dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-        dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+      const int role = warp == kMmaWarp ? 0 : 1;
+      bool ok = true;
+      if (role == 0) {
+        // S^T = K Q_h^T and dP^T = V dO_h^T for sub-step m (queries 64h .. 64h+63 of its tile)
+        const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
+        const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
+        uint64_t dqk[2], dok[2];
+        for (int s = 0; s < 2; ++s) {
+          dqk[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), 16, 1024, dev::kSwizzle128B);
+          dok[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), 16, 1024, dev::kSwizzle128B);
+        }
+        ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort);
+        for (int m = 0; ok && m < nsub; ++m) {
+          const int n = m >> 1, h = m & 1, s = n & 1;
+          // buffer m & 1 is free once the accumulating MMAs of sub-step m - 2 have completed
+          if (m >= 2 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_free[m & 1]),
+                                            ((m >> 1) - 1) & 1, abort)))
+            break;
+          if (h == 0 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort)))
+            break;
+          dev::tc_fence_after();
+          const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+          const uint32_t hoff = (h * kSubBytes) >> 4;
+          const uint64_t bq = (s ? dqk[1] : dqk[0]) + hoff, bo = (s ? dok[1] : dok[0]) + hoff;
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+            dev::umma_ss(t_st, dka + koff, bq + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+            dev::umma_ss(t_dpt, dva + koff, bo + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
+        }
+      } else {
+        // dV += P^T dO_h and dK += dS^T Q_h (K = the 64 queries of the sub-step)
+        uint64_t dqm[2], dom[2];
+        for (int s = 0; s < 2; ++s) {
+          dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+          dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        }
+        for (int m = 0; ok && m < nsub; ++m) {
+          const int n = m >> 1, h = m & 1, s = n & 1;
+          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort))) break;
+          dev::tc_fence_after();
+          const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+          const uint64_t bo = s ? dom[1] : dom[0], bq = s ? dqm[1] : dqm[0];
+#pragma unroll
+          for (int ks = 0; ks < kSub / 16; ++ks) {
+            const uint32_t acc = (m > 0 || ks > 0) ? 1u : 0u;
+            const uint32_t boff = (h * kSubBytes + ks * 16 * 128) >> 4;
+            dev::umma_ts(tmem + 256, t_st + packed_col(ks), bo + boff, idesc_tm, acc);
+            dev::umma_ts(tmem + 384, t_dpt + packed_col(ks), bq + boff, idesc_tm, acc);
+          }
+          dev::umma_commit(dev::smem_u32(&sm.bar_free[m & 1]));
+          if (h == 1) dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));  // stage s read for good
+        }
+        // the accumulators are final once this thread's MMAs have completed (every score MMA
+        // completed before the row warps released the weights these read)
+        if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       }
-      // S^T = K Q_h^T and dP^T = V dO_h^T for sub-step m (queries 64h .. 64h+63 of its tile)
-      auto issue_scores = [&](int m) {
-        const int n = m >> 1, h = m & 1, s = n & 1;
-        if (h == 0 && !wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort))
-          return false;
-        dev::tc_fence_after();
-        const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
-        const uint32_t hoff = (h * kSubBytes) >> 4;
-        const uint64_t bq = (s ? dqk[1] : dqk[0]) + hoff, bo = (s ? dok[1] : dok[0]) + hoff;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_st, dka + koff, bq + koff, idesc_kk, ks > 0 ? 1u : 0u);
-        }
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_dpt, dva + koff, bo + koff, idesc_kk, ks > 0 ? 1u : 0u);
-        }
-        dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
-        return true;
-      };
-      // dV += P^T dO_h and dK += dS^T Q_h (K = the 64 queries of the sub-step)
-      auto issue_grads = [&](int m) {
-        const int n = m >> 1, h = m & 1, s = n & 1;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort)) return false;
-        dev::tc_fence_after();
-        const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
-        const uint64_t bo = s ? dom[1] : dom[0], bq = s ? dqm[1] : dqm[0];
-#pragma unroll
-        for (int ks = 0; ks < kSub / 16; ++ks) {
-          const uint32_t acc = (m > 0 || ks > 0) ? 1u : 0u;
-          const uint32_t boff = (h * kSubBytes + ks * 16 * 128) >> 4;
-          dev::umma_ts(tmem + 256, t_st + packed_col(ks), bo + boff, idesc_tm, acc);
-          dev::umma_ts(tmem + 384, t_dpt + packed_col(ks), bq + boff, idesc_tm, acc);
-        }
-        if (h == 1) dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));  // stage s read for good
-        return true;
-      };
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort) && issue_scores(0) &&
-                issue_scores(1);
-      for (int m = 0; ok && m < nsub; ++m) {
-        ok = issue_grads(m);
-        if (ok && m + 2 < nsub) ok = issue_scores(m + 2);
-      }
-      if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
-      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
-      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain[role]));
+      wait_drain(dev::smem_u32(&sm.bar_drain[role]), 0);
     }
   } else {
     // ============== row workers: one key each, two warps per key (column halves) ==============
@@ -483,7 +495,8 @@ struct __align__(1024) SmemQ {
   uint8_t dout[kTileBytes];
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
-  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s[2], bar_p[2], bar_done, bar_drain;
+  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s[2], bar_p[2], bar_free[2], bar_done;
+  uint64_t bar_drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -519,9 +532,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(dev::smem_u32(&sm.bar_kvempty[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
+      dev::mbar_init(dev::smem_u32(&sm.bar_free[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_drain[s]), 1);
     }
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
-    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
     dev::fence_barrier_init();
   }
@@ -569,65 +583,70 @@ __global__ void __launch_bounds__(kThreads, 1)
       wait_drain(bq, 0);
       for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_kvfull[s]), issued, s);
     }
-  } else if (warp == kMmaWarp) {
-    // ============================= tcgen05.mma issuer ==============================
+  } else if (warp == kMmaWarp || warp == kGradWarp) {
+    // ========================= tcgen05.mma issuers (two threads) ==========================
     if (lane == 0 && nk > 0) {
       constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);
       constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);
-      const uint64_t dqa = dev::smem_desc(dev::smem_u32(sm.q), 16, 1024, dev::kSwizzle128B);
-      const uint64_t doa = dev::smem_desc(dev::smem_u32(sm.dout), 16, 1024, dev::kSwizzle128B);
-      uint64_t dkk[2], dvk[2], dkm[2];
-      for (int s = 0; s < 2; ++s) {
-        dkk[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), 16, 1024, dev::kSwizzle128B);
-        dvk[s] = dev::smem_desc(dev::smem_u32(sm.v[s]), 16, 1024, dev::kSwizzle128B);
-        dkm[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-      }
-      // S = Q K_h^T and dP = dO V_h^T for sub-step m (keys 64h .. 64h+63 of its key tile)
-      auto issue_scores = [&](int m) {
-        const int jj = m >> 1, hh = m & 1, s = jj & 1;
-        if (hh == 0 && !wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort))
-          return false;
-        dev::tc_fence_after();
-        const uint32_t t_s = tmem + (m & 1) * kSub, t_dp = tmem + 128 + (m & 1) * kSub;
-        const uint32_t hoff = (hh * kSubBytes) >> 4;
-        const uint64_t bk = (s ? dkk[1] : dkk[0]) + hoff, bv = (s ? dvk[1] : dvk[0]) + hoff;
-#pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_s, dqa + koff, bk + koff, idesc_kk, ks > 0 ? 1u : 0u);
+      const int role = warp == kMmaWarp ? 0 : 1;
+      bool ok = true;
+      if (role == 0) {
+        // S = Q K_h^T and dP = dO V_h^T for sub-step m (keys 64h .. 64h+63 of its key tile)
+        const uint64_t dqa = dev::smem_desc(dev::smem_u32(sm.q), 16, 1024, dev::kSwizzle128B);
+        const uint64_t doa = dev::smem_desc(dev::smem_u32(sm.dout), 16, 1024, dev::kSwizzle128B);
+        uint64_t dkk[2], dvk[2];
+        for (int s = 0; s < 2; ++s) {
+          dkk[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), 16, 1024, dev::kSwizzle128B);
+          dvk[s] = dev::smem_desc(dev::smem_u32(sm.v[s]), 16, 1024, dev::kSwizzle128B);
         }
+        ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
+        for (int m = 0; ok && m < nsub; ++m) {
+          const int jj = m >> 1, hh = m & 1, s = jj & 1;
+          if (m >= 2 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_free[m & 1]),
+                                            ((m >> 1) - 1) & 1, abort)))
+            break;
+          if (hh == 0 &&
+              !(ok = wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort)))
+            break;
+          dev::tc_fence_after();
+          const uint32_t t_s = tmem + (m & 1) * kSub, t_dp = tmem + 128 + (m & 1) * kSub;
+          const uint32_t hoff = (hh * kSubBytes) >> 4;
+          const uint64_t bk = (s ? dkk[1] : dkk[0]) + hoff, bv = (s ? dvk[1] : dvk[0]) + hoff;
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(t_dp, doa + koff, bv + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+            dev::umma_ss(t_s, dqa + koff, bk + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+            dev::umma_ss(t_dp, doa + koff, bv + koff, idesc_kk, ks > 0 ? 1u : 0u);
+          }
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
         }
-        dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
-        return true;
-      };
-      // dQ += dS K_h (K = the 64 keys of the sub-step)
-      auto issue_grads = [&](int m) {
-        const int jj = m >> 1, hh = m & 1, s = jj & 1;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort)) return false;
-        dev::tc_fence_after();
-        const uint32_t t_s = tmem + (m & 1) * kSub;
-        const uint64_t bk = s ? dkm[1] : dkm[0];
+      } else {
+        // dQ += dS K_h (K = the 64 keys of the sub-step)
+        uint64_t dkm[2];
+        for (int s = 0; s < 2; ++s)
+          dkm[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        for (int m = 0; ok && m < nsub; ++m) {
+          const int jj = m >> 1, hh = m & 1, s = jj & 1;
+          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort))) break;
+          dev::tc_fence_after();
+          const uint32_t t_s = tmem + (m & 1) * kSub;
+          const uint64_t bk = s ? dkm[1] : dkm[0];
 #pragma unroll
-        for (int ks = 0; ks < kSub / 16; ++ks)
-          dev::umma_ts(tmem + 256, t_s + packed_col(ks),
-                       bk + ((hh * kSubBytes + ks * 16 * 128) >> 4), idesc_tm,
-                       (m > 0 || ks > 0) ? 1u : 0u);
-        if (hh == 1) dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));  // stage s read for good
-        return true;
-      };
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort) && issue_scores(0) &&
-                issue_scores(1);
-      for (int m = 0; ok && m < nsub; ++m) {
-        ok = issue_grads(m);
-        if (ok && m + 2 < nsub) ok = issue_scores(m + 2);
+          for (int ks = 0; ks < kSub / 16; ++ks)
+            dev::umma_ts(tmem + 256, t_s + packed_col(ks),
+                         bk + ((hh * kSubBytes + ks * 16 * 128) >> 4), idesc_tm,
+                         (m > 0 || ks > 0) ? 1u : 0u);
+          dev::umma_commit(dev::smem_u32(&sm.bar_free[m & 1]));
+          if (hh == 1) dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));  // stage s read for good
+        }
+        if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       }
-      if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
-      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
-      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain[role]));
+      wait_drain(dev::smem_u32(&sm.bar_drain[role]), 0);
     }
   } else {
     // ========= row workers: one query row each, two warps per row (column halves) =========
