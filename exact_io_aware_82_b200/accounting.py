@@ -19,7 +19,7 @@ are not credited.
 
 from __future__ import annotations
 
-MASK_FULL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2
+MASK_FULL, MASK_CAUSAL, MASK_SLIDING, MASK_LOCAL_GLOBAL = 0, 1, 2, 3
 
 
 def _sum_min_w(lo: int, hi: int, w: int) -> int:
@@ -52,6 +52,8 @@ def visible_pairs(Nq: int, Nk: int, mask_kind: int, window: int = 0, n_sink: int
         if a > p_hi:
             return 0
         return (a + 1 + p_hi + 1) * (p_hi - a + 1) // 2
+    if mask_kind == MASK_LOCAL_GLOBAL:
+        return _local_global_pairs(Nq, Nk, window, n_sink)
     if mask_kind != MASK_SLIDING:
         raise ValueError("mask_kind")
     w, s = window, n_sink
@@ -97,3 +99,20 @@ def attn_bwd_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int, wi
     score, dP, and the dV, dK, dQ contributions), 2 * d each, i.e. 10 * d = 2.5 x the forward.
     The extra score and dP recomputation of a split dQ kernel is not credited."""
     return 10 * d * B * Hq * visible_pairs(Nq, Nk, mask_kind, window, n_sink)
+
+
+def _local_global_pairs(Nq: int, Nk: int, w: int, g: int) -> int:
+    """Bidirectional window of w keys on each side plus g global tokens, counted row by row:
+    a global row (0 <= p < g) sees all Nk keys; another row sees the window [p - w, p + w]
+    clipped to the keys, plus the global keys outside it."""
+    import numpy as np
+
+    p = np.arange(Nq, dtype=np.int64) + (Nk - Nq)
+    G = min(g, Nk)
+    lo = np.maximum(p - w, 0)
+    hi = np.minimum(p + w, Nk - 1)
+    win = np.maximum(hi - lo + 1, 0)
+    inter = np.where(hi >= lo, np.maximum(np.minimum(hi, G - 1) - lo + 1, 0), 0)
+    rows = win + (G - inter)
+    rows = np.where((p >= 0) & (p < g), Nk, rows)
+    return int(rows.sum())

@@ -21,6 +21,12 @@
  *    sparse attention and sliding window sections; "Attention Research", section 4), read as
  *    the causal left window of w keys including the diagonal; always-visible sink tokens
  *    ("Attention Research", section 4), read as key positions 0..n_sink-1, still causal.
+ *  - Local + global (Longformer; "Chapter 3.1 - The Cost of Attention", section 3: a window of
+ *    neighbours on either side plus a few global tokens that attend to, and are attended by,
+ *    every token; "Quadratic Complexity Bottleneck", sliding window: W tokens to the left and
+ *    right): not causal; key j is visible to position p iff |p - j| <= w, or j is a global
+ *    token, or p is one.  The global tokens are positions 0..n_global-1 (n_global is passed in
+ *    n_sink); a query row is global iff 0 <= p < n_global.
  *  - GQA ("Quadratic Complexity Bottleneck", grouped-query attention): query heads are
  *    partitioned into Hkv contiguous groups of G = Hq / Hkv; query head h reads kv head h / G.
  *  - Causal alignment when Nq != Nk (the pages are silent): bottom-right, query row i sits at
@@ -41,6 +47,7 @@
 #define ORACLE_MASK_FULL 0
 #define ORACLE_MASK_CAUSAL 1
 #define ORACLE_MASK_SLIDING 2
+#define ORACLE_MASK_LOCAL_GLOBAL 3
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -53,6 +60,11 @@ int oracle_num_threads(void) {
 /* Visibility of key j to the query at absolute key position p (see header comment). */
 int oracle_visible(int64_t p, int64_t j, int mask_kind, int64_t window, int64_t n_sink) {
     if (mask_kind == ORACLE_MASK_FULL) return 1;
+    if (mask_kind == ORACLE_MASK_LOCAL_GLOBAL) {
+        if (j < n_sink) return 1;            /* global key */
+        if (p >= 0 && p < n_sink) return 1;  /* global query */
+        return j >= p - window && j <= p + window;
+    }
     if (j > p) return 0; /* causal */
     if (mask_kind == ORACLE_MASK_CAUSAL) return 1;
     if (j > p - window) return 1; /* inside the window: p - w < j <= p */
@@ -64,8 +76,9 @@ static int check_args(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mask_ki
                       int n_sink) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Nq < 0 || Nk < 0 || d < 1) return -1;
     if (Hq % Hkv != 0) return -1;
-    if (mask_kind < 0 || mask_kind > 2) return -1;
+    if (mask_kind < 0 || mask_kind > 3) return -1;
     if (mask_kind == ORACLE_MASK_SLIDING && window < 1) return -1;
+    if (mask_kind == ORACLE_MASK_LOCAL_GLOBAL && window < 0) return -1;
     if (n_sink < 0) return -1;
     return 0;
 }

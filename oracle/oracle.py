@@ -14,7 +14,7 @@ import subprocess
 
 import numpy as np
 
-MASK_FULL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2
+MASK_FULL, MASK_CAUSAL, MASK_SLIDING, MASK_LOCAL_GLOBAL = 0, 1, 2, 3
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")

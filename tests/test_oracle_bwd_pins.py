@@ -57,6 +57,8 @@ FD_CASES = [
     (7, 7, 3, SLIDING, 2, 2, 4, 2, 0.6),         # window + sinks, GQA with two kv heads
     (5, 5, 2, SLIDING, 1, 0, 2, 2, -0.8),        # diagonal only, negative scale
     (4, 6, 3, FULL, 0, 0, 4, 2, -0.5),
+    (7, 7, 3, O.MASK_LOCAL_GLOBAL, 1, 1, 2, 1, 0.8),  # bidirectional window + a global token
+    (5, 8, 2, O.MASK_LOCAL_GLOBAL, 2, 0, 1, 1, 0.7),
 ]
 
 

@@ -30,6 +30,11 @@ MUTANTS = {
     "top_left_causal": ("i + (int64_t)Nk - Nq, mask_kind", "i, mask_kind"),
     "wrong_value_row": ("o[t] += pj * V[j * (int64_t)d + t];", "o[t] += pj * V[(Nk - 1 - j) * (int64_t)d + t];"),
     "unnormalised": ("double pj = s[j] / l;", "double pj = s[j];"),
+    "local_one_sided": ("return j >= p - window && j <= p + window;", "return j >= p - window && j <= p;"),
+    "local_window_edge": ("return j >= p - window && j <= p + window;",
+                          "return j > p - window && j <= p + window;"),
+    "local_no_global_query": ("if (p >= 0 && p < n_sink) return 1;  /* global query */", ""),
+    "local_no_global_key": ("if (j < n_sink) return 1;            /* global key */", ""),
 }
 
 
@@ -52,6 +57,7 @@ def _checks():
     yield "brute_causal_rect", brute(3, 6, 2, CAUSAL, 0, 0)
     yield "brute_sliding_sinks", brute(7, 7, 3, SLIDING, 2, 2)
     yield "brute_gqa", brute(3, 4, 2, CAUSAL, 0, 0, Hq=4, Hkv=2)
+    yield "brute_local_global", brute(7, 7, 3, O.MASK_LOCAL_GLOBAL, 1, 1)
 
     def zero_q():
         Nq = Nk = 9

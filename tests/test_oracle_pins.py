@@ -20,7 +20,7 @@ import synth
 from exact_io_aware_82_b200 import accounting as acc
 from oracle import oracle as O
 
-FULL, CAUSAL, SLIDING = O.MASK_FULL, O.MASK_CAUSAL, O.MASK_SLIDING
+FULL, CAUSAL, SLIDING, LOCAL = O.MASK_FULL, O.MASK_CAUSAL, O.MASK_SLIDING, O.MASK_LOCAL_GLOBAL
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_figures.json")
 
 
@@ -32,6 +32,12 @@ def visible_set(p, Nk, mask, w, s):
     """Mask as a set, written from the set definitions (not from the oracle's predicate)."""
     if mask == FULL:
         return set(range(Nk))
+    if mask == LOCAL:
+        # Longformer: w neighbours on either side; s global tokens (positions 0..s-1) that see
+        # every key and are seen by every query
+        if 0 <= p < s:
+            return set(range(Nk))
+        return set(j for j in range(Nk) if abs(p - j) <= w) | set(range(min(s, Nk)))
     past = set(range(0, min(p, Nk - 1) + 1)) if p >= 0 else set()
     if mask == CAUSAL:
         return past
@@ -45,7 +51,8 @@ def visible_set(p, Nk, mask, w, s):
 # --------------------------------------------------------------------------------------------
 @pytest.mark.parametrize("mask,w,s,Nq,Nk", [
     (FULL, 0, 0, 7, 11), (CAUSAL, 0, 0, 9, 9), (CAUSAL, 0, 0, 5, 12), (CAUSAL, 0, 0, 12, 5),
-    (SLIDING, 3, 0, 10, 10), (SLIDING, 4, 2, 13, 13), (SLIDING, 2, 3, 6, 15)])
+    (SLIDING, 3, 0, 10, 10), (SLIDING, 4, 2, 13, 13), (SLIDING, 2, 3, 6, 15),
+    (LOCAL, 2, 0, 11, 11), (LOCAL, 1, 2, 12, 12), (LOCAL, 3, 1, 6, 14), (LOCAL, 2, 2, 14, 6)])
 def test_zero_query_gives_mean_of_visible_values(mask, w, s, Nq, Nk):
     d = 5
     q = np.zeros((1, 2, Nq, d))
@@ -85,7 +92,8 @@ def test_one_hot_lookup():
 # --------------------------------------------------------------------------------------------
 # P3  row-stochastic weights; V = I exposes P itself
 # --------------------------------------------------------------------------------------------
-@pytest.mark.parametrize("mask,w,s", [(FULL, 0, 0), (CAUSAL, 0, 0), (SLIDING, 3, 2)])
+@pytest.mark.parametrize("mask,w,s", [(FULL, 0, 0), (CAUSAL, 0, 0), (SLIDING, 3, 2), (LOCAL, 2, 1),
+                                      (LOCAL, 0, 0)])
 def test_weights_are_row_stochastic_and_masked(mask, w, s):
     n = 12
     q, k = rnd(4, 0, (1, 1, n, n)), rnd(4, 1, (1, 1, n, n))
@@ -169,7 +177,8 @@ def _decimal_attention(q, k, v, Nq, Nk, d, mask, w, s, scale):
 @pytest.mark.parametrize("Nq,Nk,d,mask,w,s", [
     (4, 4, 3, FULL, 0, 0), (5, 5, 4, CAUSAL, 0, 0), (3, 6, 2, CAUSAL, 0, 0), (6, 3, 2, CAUSAL, 0, 0),
     (6, 6, 3, SLIDING, 2, 0), (6, 6, 4, SLIDING, 2, 1), (5, 6, 3, SLIDING, 1, 2),
-    (6, 6, 3, SLIDING, 6, 0), (1, 6, 4, FULL, 0, 0)])
+    (6, 6, 3, SLIDING, 6, 0), (1, 6, 4, FULL, 0, 0), (7, 7, 3, LOCAL, 1, 1), (5, 8, 2, LOCAL, 2, 2),
+    (8, 5, 3, LOCAL, 1, 0)])
 def test_brute_force_decimal(Nq, Nk, d, mask, w, s):
     q, k, v = rnd(7, 0, (1, 1, Nq, d)), rnd(7, 1, (1, 1, Nk, d)), rnd(7, 2, (1, 1, Nk, d))
     scale = 1.0 / math.sqrt(d)
@@ -218,6 +227,21 @@ def test_mask_reductions():
     of, lf = O.attention(q, k, v, FULL)
     np.testing.assert_allclose(of[:, :, -1], oc[:, :, -1], atol=1e-15)
     np.testing.assert_allclose(lf[:, :, -1], lc[:, :, -1], atol=1e-15)
+    # local + global: a window covering every key, or every token global, is the full mask;
+    # w = 0 without globals is the diagonal; one global token at 0 makes row 0 a full row and
+    # column 0 visible to every row
+    for w, g in ((n, 0), (n + 3, 2), (0, n), (1, n + 1)):
+        ol, ll = O.attention(q, k, v, LOCAL, w, g)
+        np.testing.assert_array_equal(ol, of)
+        np.testing.assert_array_equal(ll, lf)
+    o0, l0 = O.attention(q, k, v, LOCAL, 0, 0)
+    np.testing.assert_allclose(o0, v, atol=1e-15)
+    np.testing.assert_allclose(l0, np.einsum("bhid,bhid->bhi", q, k) / math.sqrt(d), atol=1e-13)
+    og, lg = O.attention(q, k, v, LOCAL, 0, 1)
+    np.testing.assert_array_equal(og[:, :, 0], of[:, :, 0])
+    np.testing.assert_allclose(lg[:, :, 1:], np.logaddexp(
+        np.einsum("bhid,bhd->bhi", q[:, :, 1:], k[:, :, 0]) / math.sqrt(d),
+        np.einsum("bhid,bhid->bhi", q[:, :, 1:], k[:, :, 1:]) / math.sqrt(d)), atol=1e-13)
 
 
 # --------------------------------------------------------------------------------------------
@@ -274,7 +298,8 @@ def test_linearity_in_v():
 @pytest.mark.parametrize("Nq,Nk", [(1, 1), (7, 7), (5, 12), (12, 5), (128, 128), (129, 300)])
 @pytest.mark.parametrize("mask,w,s", [(FULL, 0, 0), (CAUSAL, 0, 0), (SLIDING, 1, 0),
                                       (SLIDING, 4, 0), (SLIDING, 4, 3), (SLIDING, 50, 60),
-                                      (SLIDING, 400, 4)])
+                                      (SLIDING, 400, 4), (LOCAL, 0, 0), (LOCAL, 3, 0), (LOCAL, 3, 2),
+                                      (LOCAL, 40, 70), (LOCAL, 200, 5)])
 def test_pair_counts_closed_form(Nq, Nk, mask, w, s):
     brute = sum(len(visible_set(i + Nk - Nq, Nk, mask, w, s)) for i in range(Nq))
     assert O.visible_pairs(Nq, Nk, mask, w, s) == brute
