@@ -36,8 +36,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "attention fwd TFLOP/s & % BF16 TC peak (prefill); decode HBM GB/s & % peak"
-FULL, CAUSAL, SLIDING = 0, 1, 2
-MASK_NAMES = {FULL: "full", CAUSAL: "causal", SLIDING: "sliding"}
+FULL, CAUSAL, SLIDING, LOCAL_GLOBAL = 0, 1, 2, 3
+MASK_NAMES = {FULL: "full", CAUSAL: "causal", SLIDING: "sliding", LOCAL_GLOBAL: "local+global"}
 
 WORKLOADS = {
     "full_b1_h1_n256_d64_f32": dict(kind="fwd_f32", B=1, Hq=1, Hkv=1, N=256, d=64, mask=FULL,
@@ -56,6 +56,10 @@ WORKLOADS = {
                                              d=128, mask=CAUSAL, window=0, n_sink=0, seed=6,
                                              lens=[4096, 3584, 3072, 2816, 2560, 2304, 2048, 1792,
                                                    1664, 1536, 1536, 1280, 1280, 1024, 1024, 1152]),
+    # bidirectional (Longformer) window of 2048 keys on each side + 4 global tokens
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": dict(kind="fwd", B=1, Hq=32, Hkv=8, N=32768,
+                                                         d=128, mask=LOCAL_GLOBAL, window=2048,
+                                                         n_sink=4, seed=9),
     # backward pass of the headline workload (dQ, dK, dV from the forward's O and LSE)
     "bwd_causal_b4_h16_n2048_d128": dict(kind="bwd", B=4, Hq=16, Hkv=16, N=2048, d=128,
                                          mask=CAUSAL, window=0, n_sink=0, seed=8),
@@ -160,6 +164,8 @@ def config_of(name, w, n_gpus):
         c.update({"n": w["N"]})
     if w["mask"] == SLIDING:
         c.update({"window": w["window"], "n_sink": w["n_sink"]})
+    if w["mask"] == LOCAL_GLOBAL:
+        c.update({"window_each_side": w["window"], "n_global": w["n_sink"]})
     c["inputs"] = "fp32" if w["kind"] == "fwd_f32" else "bf16"
     c["l2"] = "flushed before every timed step (256 MiB write)"
     c["parallelism"] = "replicas x%d (independent batch per GPU, no collective)" % n_gpus

@@ -14,7 +14,7 @@ import ctypes
 import math
 import os
 
-MASK_FULL, MASK_CAUSAL, MASK_SLIDING = 0, 1, 2
+MASK_FULL, MASK_CAUSAL, MASK_SLIDING, MASK_LOCAL_GLOBAL = 0, 1, 2, 3
 ATTN_OK = 0
 ATTN_ERR_INVALID_ARG = -1
 ATTN_ERR_UNSUPPORTED = -2

@@ -126,8 +126,9 @@ int check_fwd_args(const void* q, const void* k, const void* v, const void* o, i
   if ((!q_empty && (q == nullptr || o == nullptr)) || (!kv_empty && (k == nullptr || v == nullptr)))
     return ATTN_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_SLIDING) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_LOCAL_GLOBAL) return ATTN_ERR_INVALID_ARG;
   if (mask_kind == ATTN_MASK_SLIDING && window < 1) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_LOCAL_GLOBAL && window < 0) return ATTN_ERR_INVALID_ARG;
   if (n_sink < 0) return ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
   return ATTN_OK;
@@ -136,8 +137,9 @@ int check_fwd_args(const void* q, const void* k, const void* v, const void* o, i
 MaskSpec make_mask(int mask_kind, int window, int n_sink, int Nk) {
   MaskSpec m;
   m.kind = mask_kind;
-  m.window = mask_kind == ATTN_MASK_SLIDING ? window : 0;
-  m.n_sink = mask_kind == ATTN_MASK_SLIDING ? n_sink : 0;
+  const bool windowed = mask_kind == ATTN_MASK_SLIDING || mask_kind == ATTN_MASK_LOCAL_GLOBAL;
+  m.window = windowed ? window : 0;
+  m.n_sink = windowed ? n_sink : 0;
   m.Nk = Nk;
   return m;
 }
@@ -587,7 +589,9 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
-  bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + 7) / 8), 256, 0, st>>>(
+  bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
+                                               bwd::kPrepRowsPerBlock),
+                         256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
       dsum, Nq, p.npad, prow);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;

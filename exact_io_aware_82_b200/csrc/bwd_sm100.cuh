@@ -71,47 +71,44 @@ struct Params {
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
-// Columns 32w .. 32w+31 of a tile that are <= x, as bits (bit i = column 32w + i).
-__device__ __forceinline__ uint32_t cols_upto(int x, int w) {
-  const int k = x - 32 * w;
-  return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
-}
-
-// clamp a 64-bit column bound into [-1, 128] (every bound outside a tile acts the same)
-__device__ __forceinline__ int clamp_col(long long x) {
-  return x < -1 ? -1 : (x > kT ? kT : static_cast<int>(x));
-}
-
-// Is every pair of the block (query positions P0 .. P0+rows-1) x (keys c0 .. c0+cols-1)
-// visible?  Conservative: rows past Nq count as visible here (their weights are zero through
-// LSE = +inf).
-__device__ __forceinline__ bool block_full(const MaskSpec& m, int P0, int rows, int c0, int cols) {
-  const int c1 = c0 + cols - 1, P1 = P0 + rows - 1;
-  if (c1 >= m.Nk) return false;
-  if (m.kind == ATTN_MASK_FULL) return true;
-  if (c1 > P0) return false;
-  if (m.kind == ATTN_MASK_CAUSAL) return true;
-  return (static_cast<long long>(c0) > static_cast<long long>(P1) - m.window) || (c1 < m.n_sink);
-}
-
 __device__ __forceinline__ int floor_div128(long long a) {
   return static_cast<int>(a >= 0 ? a / kT : -((-a + kT - 1) / kT));
 }
 
-// Query tiles [lo, hi] whose rows see at least one key of [c0, c1] (off = Nk - Nq; query row i
-// sits at key position i + off).  Empty when lo > hi.
-__device__ __forceinline__ void query_tiles(const MaskSpec& m, int c0, int c1, int off, int Nq,
-                                            int& lo, int& hi) {
+// Query tiles whose rows see at least one key of [c0, c1] (off = Nk - Nq; query row i sits at
+// key position i + off), as a TileRange: tiles [0, ns) (the global rows of the local + global
+// mask), then [lo, hi].
+__device__ __forceinline__ TileRange query_tiles(const MaskSpec& m, int c0, int c1, int off,
+                                                 int Nq) {
   const int nqt = (Nq + kT - 1) / kT;
-  lo = 0;
-  hi = nqt - 1;
-  if (m.kind == ATTN_MASK_FULL) return;
+  TileRange r{0, 0, nqt - 1};
+  if (m.kind == ATTN_MASK_FULL) return r;
+  if (m.kind == ATTN_MASK_LOCAL_GLOBAL) {
+    if (c0 < m.n_sink) return r;  // a global key is seen by every row
+    // rows p in [c0 - w, c1 + w], and the global rows 0 <= p < n_global (i < n_global - off)
+    const long long g_rows = static_cast<long long>(m.n_sink) - off;
+    const int g_tiles = g_rows <= 0 ? 0 : min(nqt, static_cast<int>((g_rows + kT - 1) / kT));
+    r.lo = max(0, floor_div128(static_cast<long long>(c0) - m.window - off));
+    r.hi = min(r.hi, floor_div128(static_cast<long long>(c1) + m.window - off));
+    if (r.lo > r.hi) {  // no window row: the global rows only
+      r.ns = g_tiles;
+      r.lo = g_tiles;
+      r.hi = g_tiles - 1;
+    } else if (g_tiles >= r.lo) {
+      r.lo = 0;
+      r.hi = max(r.hi, g_tiles - 1);
+    } else {
+      r.ns = g_tiles;
+    }
+    return r;
+  }
   // causal: p = i + off >= key  ->  i >= c0 - off for the block's first key
-  lo = max(0, floor_div128(static_cast<long long>(c0) - off));
+  r.lo = max(0, floor_div128(static_cast<long long>(c0) - off));
   // window: p < key + w for keys past the sinks (a block holding a sink key is seen by every
   // later row)
   if (m.kind == ATTN_MASK_SLIDING && c0 >= m.n_sink)
-    hi = min(hi, floor_div128(static_cast<long long>(c1) + m.window - 1 - off));
+    r.hi = min(r.hi, floor_div128(static_cast<long long>(c1) + m.window - 1 - off));
+  return r;
 }
 
 // Producer drain: wait until the last copy issued into stage s (of `issued` copies alternating
@@ -167,38 +164,57 @@ __device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int ch) {
 __device__ __forceinline__ uint32_t packed_col(int ks) { return ks * 8 + (ks >= 2 ? 16 : 0); }
 
 // ------------------------------------------------------------------------------------------
-// 1. D_i = dO_i . O_i and LSE_i * log2(e): one warp per query row
+// 1. D_i = dO_i . O_i and LSE_i * log2(e) per (padded) query row
 // ------------------------------------------------------------------------------------------
+constexpr int kPrepRowsPerBlock = 64;  // 8 warps x 8 rows
+
 __global__ void __launch_bounds__(256)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                     const float* __restrict__ lse, float* __restrict__ lse2,
                     float* __restrict__ dsum, int Nq, int npad, long long padded_rows) {
-  // padded row index -> (b*Hq + h, i); rows i >= Nq only get the padding values
-  const long long prow = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (prow >= padded_rows) return;
-  const long long bh = prow / npad;
-  const int i = static_cast<int>(prow % npad);
-  if (i >= Nq) {
-    if (lane == 0) {
-      dsum[prow] = 0.f;
-      lse2[prow] = pos_inf();
-    }
-    return;
-  }
-  const long long row = bh * Nq + i;
-  const uint2 a = *reinterpret_cast<const uint2*>(o + row * kD + lane * 4);
-  const uint2 g = *reinterpret_cast<const uint2*>(dout + row * kD + lane * 4);
-  float acc = __uint_as_float(a.x << 16) * __uint_as_float(g.x << 16);
-  acc = fmaf(__uint_as_float(a.x & 0xffff0000u), __uint_as_float(g.x & 0xffff0000u), acc);
-  acc = fmaf(__uint_as_float(a.y << 16), __uint_as_float(g.y << 16), acc);
-  acc = fmaf(__uint_as_float(a.y & 0xffff0000u), __uint_as_float(g.y & 0xffff0000u), acc);
+  // a half-warp per row (16 lanes x 16 bytes = one 256-byte row of O and of dO); each warp
+  // takes 8 consecutive padded rows, every load issued before the first use
+  const int lane = threadIdx.x & 31, sub = lane >> 4, sl = lane & 15;
+  const long long base = static_cast<long long>(blockIdx.x) * kPrepRowsPerBlock +
+                         (threadIdx.x >> 5) * 8;
+  uint4 a[4], g[4];
+  long long src[4];
 #pragma unroll
-  for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-  if (lane == 0) {
-    dsum[prow] = acc;
-    const float l = lse[row];
-    lse2[prow] = (l == -pos_inf()) ? pos_inf() : l * kLog2e;
+  for (int it = 0; it < 4; ++it) {
+    const long long prow = base + 2 * it + sub;
+    src[it] = -1;
+    if (prow < padded_rows) {
+      const int i = static_cast<int>(prow % npad);
+      if (i < Nq) src[it] = (prow / npad) * Nq + i;
+    }
+    a[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(o + src[it] * kD + sl * 8)
+                         : make_uint4(0u, 0u, 0u, 0u);
+    g[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(dout + src[it] * kD + sl * 8)
+                         : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const uint32_t aw[4] = {a[it].x, a[it].y, a[it].z, a[it].w};
+    const uint32_t gw[4] = {g[it].x, g[it].y, g[it].z, g[it].w};
+    float acc = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(gw[w] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(gw[w] & 0xffff0000u), acc);
+    }
+#pragma unroll
+    for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+    const long long prow = base + 2 * it + sub;
+    if (sl == 0 && prow < padded_rows) {
+      if (src[it] >= 0) {
+        dsum[prow] = acc;
+        const float l = lse[src[it]];
+        lse2[prow] = (l == -pos_inf()) ? pos_inf() : l * kLog2e;
+      } else {  // padding row past Nq
+        dsum[prow] = 0.f;
+        lse2[prow] = pos_inf();
+      }
+    }
   }
 }
 
@@ -251,10 +267,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bk / p.Hkv, hk = bk % p.Hkv;
   const int c0 = kb * kT, c1 = min(c0 + kT, p.Nk) - 1;
   const int off = p.Nk - p.Nq;
-  int qlo, qhi;
-  query_tiles(p.mask, c0, c1, off, p.Nq, qlo, qhi);
-  const int nqt = qhi >= qlo ? qhi - qlo + 1 : 0;
-  const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qlo + n % nqt
+  const TileRange qr = query_tiles(p.mask, c0, c1, off, p.Nq);
+  const int nqt = qr.count();
+  const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qr.tile(n % nqt)
   const int nsub = 2 * nsteps;
 
   if (tid == 0) {
@@ -301,7 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = n & 1;
         if (!wait_bounded(dev::smem_u32(&sm.bar_qempty[s]), ((n >> 1) & 1) ^ 1, abort)) break;
         const int hq = hk * p.G + n / nqt;
-        const int r0 = (qlo + n % nqt) * kT;
+        const int r0 = qr.tile(n % nqt) * kT;
         const uint32_t bq = dev::smem_u32(&sm.bar_qfull[s]);
         const size_t vrow = static_cast<size_t>(b * p.Hq + hq) * p.npad + r0;
         dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes + 2 * kT * 4);
@@ -399,7 +414,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int m = 0; m < nsub; ++m) {
       const int n = m >> 1, h = m & 1, s = n & 1;
-      const int r0 = (qlo + n % nqt) * kT + h * kSub;  // first query row of the sub-step
+      const int r0 = qr.tile(n % nqt) * kT + h * kSub;  // first query row of the sub-step
       // the stage's LSE / D vectors came with its Q and dO tiles; the stage cannot be refilled
       // before this tile's weights are released, so its phase is still this tile's
       ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort) &&
@@ -412,19 +427,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_ld32(t_st, sr);
       dev::tmem_ld32(t_dpt, dr);
 
-      // visible query columns of key j among this warp's 32 (columns past Nq: LSE = +inf)
+      // visible query columns of key j among this warp's 32 (columns past Nq: LSE = +inf):
+      // [lo, hi], and for the local + global mask also the global rows [glo, ghi]
       const int P0 = r0 + off;
       uint32_t vis = ~0u;
-      if (!block_full(p.mask, P0, kSub, c0, kT)) {
-        int lo = -1, hi = kT;
+      if (!block_visible(p.mask, P0, kSub, c0, kT)) {
+        int lo = -1, hi = kT, glo = 0, ghi = -1;
         if (j >= p.mask.Nk) {
           hi = -1;
+        } else if (p.mask.kind == ATTN_MASK_LOCAL_GLOBAL) {
+          if (j >= p.mask.n_sink) {  // a global key is seen by every row
+            lo = clamp_col(static_cast<long long>(j) - p.mask.window - P0);  // p >= j - w
+            hi = clamp_col(static_cast<long long>(j) + p.mask.window - P0);  // p <= j + w
+            glo = clamp_col(-static_cast<long long>(P0));                  // p >= 0
+            ghi = clamp_col(static_cast<long long>(p.mask.n_sink) - 1 - P0);  // p < n_global
+          }
         } else if (p.mask.kind != ATTN_MASK_FULL) {
           lo = clamp_col(static_cast<long long>(j) - P0);  // p >= j
           if (p.mask.kind == ATTN_MASK_SLIDING && j >= p.mask.n_sink)
             hi = clamp_col(static_cast<long long>(j) + p.mask.window - 1 - P0);  // p < j + w
         }
-        vis = cols_upto(hi, ch) & ~cols_upto(lo - 1, ch);
+        vis = (cols_upto(hi, ch) & ~cols_upto(lo - 1, ch)) |
+              (cols_upto(ghi, ch) & ~cols_upto(glo - 1, ch));
       }
       const float4* l2v = reinterpret_cast<const float4*>(sm.lse2[s] + h * kSub + ch * 32);
       const float4* ddv = reinterpret_cast<const float4*>(sm.dsum[s] + h * kSub + ch * 32);
@@ -671,15 +695,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_ld32(t_dp, dr);
       const int key0 = tr.tile(m >> 1) * kT + (m & 1) * kSub;  // first key of the sub-step
       uint32_t vis = ~0u;
-      if (!block_full(p.mask, r0 + off, kT, key0, kSub)) {
-        // visible key columns of this row: col <= hi and (col >= lo or col < sk)
-        const long long last = p.mask.kind == ATTN_MASK_FULL ? p.mask.Nk - 1
-                                                             : min(prow, p.mask.Nk - 1);
-        const int hi = clamp_col(last - key0);
-        const bool sl = p.mask.kind == ATTN_MASK_SLIDING;
-        const int lo = sl ? clamp_col(static_cast<long long>(prow) - p.mask.window + 1 - key0) : -1;
-        const int sk = sl ? clamp_col(static_cast<long long>(p.mask.n_sink) - key0) : -1;
-        vis = cols_upto(hi, ch) & (~cols_upto(lo - 1, ch) | cols_upto(sk - 1, ch));
+      if (!block_visible(p.mask, r0 + off, kT, key0, kSub)) {
+        // visible key columns of this row: (lo <= col <= hi) or col < sk
+        int hi, lo, sk;
+        row_cols(p.mask, prow, key0, hi, lo, sk);
+        vis = row_bits(hi, lo, sk, ch);
       }
       dev::tmem_wait_ld();
 #pragma unroll

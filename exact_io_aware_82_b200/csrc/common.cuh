@@ -53,17 +53,83 @@ __device__ __forceinline__ bool wait_drain(uint32_t bar, uint32_t parity) {
 // Mask shared by every kernel.  p = key position of the query row (i + Nk - Nq), j = key index.
 struct MaskSpec {
   int kind;    // ATTN_MASK_*
-  int window;  // sliding window width w (keys p-w+1 .. p)
-  int n_sink;  // always-visible sink keys 0 .. n_sink-1 (still causal)
+  int window;  // sliding: window width w (keys p-w+1 .. p); local+global: w keys on each side
+  int n_sink;  // sliding: always-visible sink keys 0 .. n_sink-1 (still causal);
+               // local+global: the global tokens 0 .. n_sink-1 (as keys and as queries)
   int Nk;      // keys >= Nk are padding
 };
+
+__host__ __device__ __forceinline__ bool is_global_row(const MaskSpec& m, int p) {
+  return p >= 0 && p < m.n_sink;
+}
 
 __device__ __forceinline__ bool key_visible(const MaskSpec& m, int p, int j) {
   if (j >= m.Nk) return false;
   if (m.kind == ATTN_MASK_FULL) return true;
+  if (m.kind == ATTN_MASK_LOCAL_GLOBAL) {
+    if (j < m.n_sink || is_global_row(m, p)) return true;
+    const long long d = static_cast<long long>(p) - j;
+    return d <= m.window && -d <= m.window;
+  }
   if (j > p) return false;
   if (m.kind == ATTN_MASK_CAUSAL) return true;
   return (j > p - m.window) || (j < m.n_sink);
+}
+
+// Columns 32w .. 32w+31 of a 128-column tile that are <= x, as bits (bit i = column 32w + i).
+__device__ __forceinline__ uint32_t cols_upto(int x, int w) {
+  const int k = x - 32 * w;
+  return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
+}
+
+// clamp a 64-bit column bound into [-1, 128] (every bound outside a tile acts the same)
+__host__ __device__ __forceinline__ int clamp_col(long long x) {
+  return x < -1 ? -1 : (x > 128 ? 128 : static_cast<int>(x));
+}
+
+// Visible keys of the query at position p among the columns key0 .. key0+127 of a tile:
+// (lo <= col <= hi) or col < sk, bounds clamped to [-1, 128].  Sliding-window sinks stop at the
+// causal bound; global keys of the local + global mask do not.
+__device__ __forceinline__ void row_cols(const MaskSpec& m, int p, int key0, int& hi, int& lo,
+                                         int& sk) {
+  const long long kNone = -(1ll << 40);
+  long long last = m.Nk - 1, first = kNone, sink = kNone;
+  if (m.kind == ATTN_MASK_CAUSAL) {
+    last = p < last ? p : last;
+  } else if (m.kind == ATTN_MASK_SLIDING) {
+    last = p < last ? p : last;
+    first = static_cast<long long>(p) - m.window + 1;
+    sink = m.n_sink < last + 1 ? m.n_sink : last + 1;
+  } else if (m.kind == ATTN_MASK_LOCAL_GLOBAL && !is_global_row(m, p)) {
+    const long long right = static_cast<long long>(p) + m.window;
+    last = right < last ? right : last;
+    first = static_cast<long long>(p) - m.window;
+    sink = m.n_sink < m.Nk ? m.n_sink : m.Nk;
+  }
+  hi = clamp_col(last - key0);
+  lo = clamp_col(first - key0);
+  sk = clamp_col(sink - key0);
+}
+
+// The 32 columns 32w .. 32w+31 of that set, as bits.
+__device__ __forceinline__ uint32_t row_bits(int hi, int lo, int sk, int w) {
+  return (cols_upto(hi, w) & ~cols_upto(lo - 1, w)) | cols_upto(sk - 1, w);
+}
+
+// Is every pair of the block (query positions P0 .. P0+rows-1) x (keys c0 .. c0+cols-1)
+// visible?  Conservative: rows past Nq count as visible (callers zero or skip them).
+__host__ __device__ __forceinline__ bool block_visible(const MaskSpec& m, int P0, int rows, int c0,
+                                                      int cols) {
+  const long long c1 = static_cast<long long>(c0) + cols - 1;
+  const long long P1 = static_cast<long long>(P0) + rows - 1;
+  if (c1 >= m.Nk) return false;
+  if (m.kind == ATTN_MASK_FULL) return true;
+  if (m.kind == ATTN_MASK_LOCAL_GLOBAL)
+    return c1 < m.n_sink || (P0 >= 0 && P1 < m.n_sink) ||
+           (c0 >= P1 - m.window && c1 <= P0 + static_cast<long long>(m.window));
+  if (c1 > P0) return false;
+  if (m.kind == ATTN_MASK_CAUSAL) return true;
+  return (c0 > P1 - m.window) || (c1 < m.n_sink);
 }
 
 // Range of key tiles (of `tile` keys) a block of query positions [p_lo, p_hi] must visit:
@@ -82,6 +148,35 @@ __host__ __device__ inline TileRange key_tiles(const MaskSpec& m, int p_lo, int 
   if (m.kind == ATTN_MASK_FULL) {
     r.lo = 0;
     r.hi = last_key / tile;
+    return r;
+  }
+  if (m.kind == ATTN_MASK_LOCAL_GLOBAL) {
+    // a global row sees every key; otherwise the window tiles and the global-key tiles
+    const int g_lo = p_lo > 0 ? p_lo : 0, g_hi = p_hi < m.n_sink - 1 ? p_hi : m.n_sink - 1;
+    if (g_lo <= g_hi) {
+      r.hi = last_key / tile;
+      return r;
+    }
+    const int g_keys = m.n_sink < m.Nk ? m.n_sink : m.Nk;
+    const int g_tiles = (g_keys + tile - 1) / tile;
+    long long first = static_cast<long long>(p_lo) - m.window;
+    long long last = static_cast<long long>(p_hi) + m.window;
+    if (first < 0) first = 0;
+    if (last > last_key) last = last_key;
+    if (first > last) {  // no window key: the global keys only
+      r.ns = g_tiles;
+      r.lo = g_tiles;
+      r.hi = g_tiles - 1;
+      return r;
+    }
+    r.lo = static_cast<int>(first / tile);
+    r.hi = static_cast<int>(last / tile);
+    if (g_tiles >= r.lo) {  // global tiles run into the window: one contiguous range
+      r.lo = 0;
+      if (g_tiles - 1 > r.hi) r.hi = g_tiles - 1;
+    } else {
+      r.ns = g_tiles;
+    }
     return r;
   }
   if (p_hi < 0) return r;  // every row precedes the first key

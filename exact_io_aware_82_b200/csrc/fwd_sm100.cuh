@@ -83,18 +83,7 @@ constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base
 // Is every (row, key) of the 128x128 block of query tile rows [P0, P0+127] x keys of tile kt
 // visible?  Conservative (uses all 128 rows even past Nq).
 __device__ __forceinline__ bool tile_is_full(const MaskSpec& m, int P0, int kt) {
-  const int c0 = kt * kBN, c1 = c0 + kBN - 1, P1 = P0 + kBM - 1;
-  if (c1 >= m.Nk) return false;
-  if (m.kind == ATTN_MASK_FULL) return true;
-  if (c1 > P0) return false;
-  if (m.kind == ATTN_MASK_CAUSAL) return true;
-  return (c0 > P1 - m.window) || (c1 < m.n_sink);
-}
-
-// Columns 32w .. 32w+31 of a tile that are <= x, as bits (bit i = column 32w + i).
-__device__ __forceinline__ uint32_t cols_upto(int x, int w) {
-  const int k = x - 32 * w;
-  return k < 0 ? 0u : (k >= 31 ? 0xffffffffu : (2u << k) - 1u);
+  return block_visible(m, P0, kBM, kt * kBN, kBN);
 }
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
@@ -382,17 +371,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_wait_ld_regs(r);
 
       if (!tile_is_full(mask, P0, kt)) {
-        // visible columns of this row inside the tile: col <= hi and (col >= lo or col < sk),
+        // visible columns of this row inside the tile: (lo <= col <= hi) or col < sk,
         // as a 128-bit set built with shifts, then one bit test and select per column (no
         // per-column branches, whatever the compiler knows about hi, lo and sk)
-        const int hi = min(mask.kind == ATTN_MASK_FULL ? mask.Nk - 1 : prow, mask.Nk - 1) - key0;
-        const bool sl = mask.kind == ATTN_MASK_SLIDING;
-        const int lo = sl ? prow - mask.window + 1 - key0 : -(1 << 30);
-        const int sk = sl ? mask.n_sink - key0 : -(1 << 30);
+        int hi, lo, sk;
+        row_cols(mask, prow, key0, hi, lo, sk);
         uint32_t vis[4];
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-          vis[w] = cols_upto(hi, w) & (~cols_upto(lo - 1, w) | cols_upto(sk - 1, w));
+          vis[w] = row_bits(hi, lo, sk, w);
 #pragma unroll
         for (int e = 0; e < 128; ++e)
           r[e] = ((vis[e >> 5] >> (e & 31)) & 1u) ? r[e] : __float_as_uint(masked);

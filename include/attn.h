@@ -22,6 +22,11 @@
  *                      keys including the diagonal ("Quadratic Complexity Bottleneck",
  *                      sliding-window attention) plus n_sink always-visible sink tokens at key
  *                      positions 0..n_sink-1 ("Attention Research", section 4).
+ *   ATTN_MASK_LOCAL_GLOBAL  not causal: key j visible iff |p_i - j| <= window (window keys on
+ *                      each side), or j < n_sink, or 0 <= p_i < n_sink: the first n_sink
+ *                      tokens are global, they see and are seen by every token (Longformer;
+ *                      "Chapter 3.1 - The Cost of Attention", section 3; "Quadratic Complexity
+ *                      Bottleneck", sliding window: W tokens to the left and right).
  * Rows with no visible key get O = 0 and LSE = -inf.
  * GQA ("Quadratic Complexity Bottleneck", grouped-query attention): Hq = G * Hkv and query head
  * h reads kv head hk = h / G (contiguous groups); Hkv = 1 is multi-query attention.
@@ -60,7 +65,12 @@ extern "C" {
 /* Same object as cudaStream_t (NULL = the legacy default stream). */
 typedef struct CUstream_st *attn_stream_t;
 
-enum attn_mask_kind { ATTN_MASK_FULL = 0, ATTN_MASK_CAUSAL = 1, ATTN_MASK_SLIDING = 2 };
+enum attn_mask_kind {
+  ATTN_MASK_FULL = 0,
+  ATTN_MASK_CAUSAL = 1,
+  ATTN_MASK_SLIDING = 2,
+  ATTN_MASK_LOCAL_GLOBAL = 3
+};
 
 enum attn_status {
   ATTN_OK = 0,
@@ -86,8 +96,9 @@ ATTN_API const char *attn_last_error_detail(void);
  *   q, o   bf16 [B][Hq][Nq][d];  k, v  bf16 [B][Hkv][Nk][d];  lse fp32 [B][Hq][Nq] or NULL.
  *   B >= 0, Nq >= 0, Nk >= 0 (B = 0 or Nq = 0: nothing to do; Nk = 0: O = 0, LSE = -inf),
  *   Hq >= 1, Hkv >= 1, Hq % Hkv == 0, d == 128.
- *   mask_kind in attn_mask_kind; window >= 1 for ATTN_MASK_SLIDING (ignored otherwise);
- *   n_sink >= 0 (used by ATTN_MASK_SLIDING only); scale finite (1/sqrt(d) in the usual case).
+ *   mask_kind in attn_mask_kind; window >= 1 for ATTN_MASK_SLIDING, >= 0 for
+ *   ATTN_MASK_LOCAL_GLOBAL (ignored otherwise); n_sink >= 0 (sinks or global tokens, used by
+ *   those two masks only); scale finite (1/sqrt(d) in the usual case).
  *   All pointers 16-byte aligned.  Accumulation is fp32; O is rounded to bf16 once.
  */
 ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, float *lse, int B, int Hq,

@@ -67,9 +67,11 @@ def test_invalid_arguments_are_rejected(lib, f32):
     assert fwd(lib, Hq=0, f32=f32) == E
     assert fwd(lib, Hkv=0, f32=f32) == E
     assert fwd(lib, Hq=3, Hkv=2, f32=f32) == E
-    assert fwd(lib, mask=3, f32=f32) == E
+    assert fwd(lib, mask=4, f32=f32) == E
     assert fwd(lib, mask=-1, f32=f32) == E
     assert fwd(lib, mask=2, w=0, f32=f32) == E
+    assert fwd(lib, mask=3, w=-1, f32=f32) == E
+    assert fwd(lib, mask=3, w=2, s=-1, f32=f32) == E
     assert fwd(lib, mask=2, w=4, s=-1, f32=f32) == E
     assert fwd(lib, scale=float("nan"), f32=f32) == E
     assert fwd(lib, scale=float("inf"), f32=f32) == E
