@@ -82,16 +82,19 @@ DECODE = "decode_b64_h32_kv8_n32768_d128"
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the sources of that
 # kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
-    "causal_b4_h16_n2048_d128": {"bytes": 141631488, "src": "c1646697c270d7e4"},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 471216640, "src": "c1646697c270d7e4"},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 690882560, "src": "c1646697c270d7e4"},
-    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1290109184, "src": "c1646697c270d7e4"},
+    "causal_b4_h16_n2048_d128": {"bytes": 140389376, "src": "5252e77825f07a1a"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 455650304, "src": "5252e77825f07a1a"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 677068032, "src": "5252e77825f07a1a"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293632000, "src": "5252e77825f07a1a"},
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 827440128, "src": "5252e77825f07a1a"},
+    # the backward step's three kernels together (prep + dK/dV + dQ)
+    "bwd_causal_b4_h16_n2048_d128": {"bytes": 470214400, "src": "bc71c31cb46971e0"},
     # captured on the 8-sequence cases; the cache is read once per sequence, so the
     # 64-sequence launch moves 8x that
-    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1078274048, "src": "5e2d19b554ce67c9"},
-    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1078274048, "src": "5e2d19b554ce67c9"},
-    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1078672128, "src": "5e2d19b554ce67c9"},
-    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1078672128, "src": "5e2d19b554ce67c9"},
+    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1080556288, "src": "47499156659e5257"},
+    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1080556288, "src": "47499156659e5257"},
+    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1078285568, "src": "47499156659e5257"},
+    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1078285568, "src": "47499156659e5257"},
 }
 
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
@@ -99,11 +102,14 @@ NCU_TRAFFIC = {
 FAMILY_SOURCES = {
     "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
+    "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
 }
 
 
 def family_of(w):
-    return "decode" if w["kind"] in ("decode", "decode_paged") else "prefill"
+    if w["kind"] in ("decode", "decode_paged"):
+        return "decode"
+    return "bwd" if w["kind"] == "bwd" else "prefill"
 
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
