@@ -60,6 +60,9 @@ WORKLOADS = {
     "local_global_b1_h32_kv8_n32768_w2048_g4_d128": dict(kind="fwd", B=1, Hq=32, Hkv=8, N=32768,
                                                          d=128, mask=LOCAL_GLOBAL, window=2048,
                                                          n_sink=4, seed=9),
+    # the headline workload with E4M3 (FP8) Q, K, V and per-(b, head) scales
+    "fp8_causal_b4_h16_n2048_d128": dict(kind="fwd_fp8", B=4, Hq=16, Hkv=16, N=2048, d=128,
+                                         mask=CAUSAL, window=0, n_sink=0, seed=10),
     # backward pass of the headline workload (dQ, dK, dV from the forward's O and LSE)
     "bwd_causal_b4_h16_n2048_d128": dict(kind="bwd", B=4, Hq=16, Hkv=16, N=2048, d=128,
                                          mask=CAUSAL, window=0, n_sink=0, seed=8),
@@ -100,7 +103,7 @@ NCU_TRAFFIC = {
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
 # up grids and tensor maps)
 FAMILY_SOURCES = {
-    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
     "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
 }
@@ -172,7 +175,8 @@ def config_of(name, w, n_gpus):
         c.update({"window": w["window"], "n_sink": w["n_sink"]})
     if w["mask"] == LOCAL_GLOBAL:
         c.update({"window_each_side": w["window"], "n_global": w["n_sink"]})
-    c["inputs"] = "fp32" if w["kind"] == "fwd_f32" else "bf16"
+    c["inputs"] = {"fwd_f32": "fp32", "fwd_fp8": "e4m3 codes, fp32 scale per (b, head)"}.get(
+        w["kind"], "bf16")
     c["l2"] = "flushed before every timed step (256 MiB write)"
     c["parallelism"] = "replicas x%d (independent batch per GPU, no collective)" % n_gpus
     return c
@@ -291,6 +295,17 @@ class Workload:
             sl = torch.full((B,), N, dtype=torch.int32, device="cuda")
             self.inputs = [q, k, v, bt, sl]
             self.lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        elif w["kind"] == "fwd_fp8":
+            # E4M3 codes with per-(b, head) scales, drawn on the host
+            xs, scs = [], []
+            for tid, shape in ((synth.Q_ID, (B, Hq, N, d)), (synth.K_ID, (B, Hkv, N, d)),
+                               (synth.V_ID, (B, Hkv, N, d))):
+                codes, sc = synth.normal_e4m3(seed, tid, shape)
+                xs.append(torch.from_numpy(codes).cuda())
+                scs.append(torch.from_numpy(sc).cuda())
+            self.inputs = xs + scs
+            self.lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
+            self.o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device="cuda")
         elif w["kind"] == "bwd":
             # the forward's outputs for these inputs are inputs of the backward step
             q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, N, d), dt, "cuda")
@@ -312,7 +327,8 @@ class Workload:
             self.inputs = [q, k, v]
             lse_shape = (B, Hq) if w["kind"] == "decode" else (B, Hq, nq)
             self.lse = torch.empty(lse_shape, dtype=torch.float32, device="cuda")
-        self.o = torch.empty_like(self.inputs[0])
+        if w["kind"] != "fwd_fp8":
+            self.o = torch.empty_like(self.inputs[0])
         # what a step hands back to its caller (read back in the end-to-end timing)
         self.outputs = self.grads if w["kind"] == "bwd" else [self.o, self.lse]
         if w["kind"] in ("decode", "decode_paged"):
@@ -326,6 +342,9 @@ class Workload:
         o, lse = self.o, self.lse
         if w["kind"] == "decode":
             A.attn_decode(x[0], x[1], x[2], o=o, lse=lse, workspace=self.ws)
+        elif w["kind"] == "fwd_fp8":
+            A.attn_fwd_fp8(x[0], x[1], x[2], x[3], x[4], x[5], o=o, lse=lse, mask_kind=w["mask"],
+                           window=w["window"], n_sink=w["n_sink"])
         elif w["kind"] == "bwd":
             g = self.grads
             A.attn_bwd(x[0], x[1], x[2], x[3], x[4], x[5], mask_kind=w["mask"], window=w["window"],
@@ -446,13 +465,17 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
         bound, peak, punit = "hbm", peaks["hbm_gbs"], "GB/s"
     else:
         bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        if w["kind"] == "fwd_fp8":
+            # no FP8 GEMM was measured: the bf16 figure times the nominal ratio 4.5 / 2.25
+            peak = round(2.0 * peaks["bf16_tflops"], 1)
         if w["kind"] == "fwd_f32":
             bound, peak = "fp32-fma", None
     tr = NCU_TRAFFIC.get(name)
     traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash(family_of(w)) else None
     roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic,
-            "peak_source": peak_kind + (" burst" if bound == "tensor" else "")}
+            "peak_source": peak_kind + (" burst" if bound == "tensor" else "")
+            + (" bf16 x 2 (nominal FP8 / BF16 ratio)" if w["kind"] == "fwd_fp8" else "")}
 
     # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
     host_in = [t.cpu().pin_memory() for t in wl.inputs]
@@ -503,6 +526,9 @@ def oracle_sample(name, budget_s, seed=0, host=None):
     def draw(tid, shape):
         if w["kind"] == "fwd_f32":
             return synth.normal_f32(w["seed"], tid, shape).astype(np.float64)
+        if w["kind"] == "fwd_fp8":
+            codes, sc = synth.normal_e4m3(w["seed"], tid, shape)
+            return synth.e4m3_bits_to_f32(codes).astype(np.float64) * sc.astype(np.float64)[..., None, None]
         return synth.bf16_bits_to_f32(synth.normal_bf16_bits(w["seed"], tid, shape)).astype(np.float64)
 
     if w["kind"] == "fwd_varlen":
@@ -715,7 +741,8 @@ def main():
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(r["ms_per_step"], 5), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None,
-                "dtype": "f32" if w["kind"] == "fwd_f32" else "bf16",
+                "dtype": {"fwd_f32": "f32", "fwd_fp8": "e4m3 (fp32 accumulate, bf16 out)"}.get(
+                    w["kind"], "bf16"),
                 "data": "synthetic (iid N(0,1), seeded counter-based generator)",
                 "config": config_of(name, w, world), "roofline": r["roofline"], "e2e": r["e2e"],
                 "gpu_launches": r["launches"], "clocks": r["clocks"]}

@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
            "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc",
-           "attn_fwd_varlen", "attn_decode_paged", "attn_bwd", "attn_bwd_workspace_bytes")
+           "attn_fwd_varlen", "attn_decode_paged", "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_fp8")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
 DECODE_NOALLOC_MAX_BYTES = 32 << 20
@@ -75,6 +75,8 @@ def lib():
         L.attn_fwd_varlen.restype = i
         L.attn_decode_paged.argtypes = [vp] * 7 + [i] * 8 + [f, i, vp, ctypes.c_size_t, vp]
         L.attn_decode_paged.restype = i
+        L.attn_fwd_fp8.argtypes = [vp] * 8 + [i] * 9 + [f, vp]
+        L.attn_fwd_fp8.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i] * 3
         L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.attn_bwd.argtypes = [vp] * 9 + [i] * 9 + [f, vp, ctypes.c_size_t, vp]
@@ -173,6 +175,39 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, l
                                int(max_seqlen_q), d, int(mask_kind), int(window), int(n_sink),
                                scale, _stream_ptr(stream))
     _raise(rc, "attn_fwd_varlen")
+    return o, lse
+
+
+def attn_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o=None, lse=None,
+                 mask_kind=MASK_FULL, window=0, n_sink=0, scale=None, return_lse=True,
+                 stream=None):
+    """E4M3 forward: q [B,Hq,Nq,d], k, v [B,Hkv,Nk,d] as uint8 (or float8_e4m3fn) codes;
+    descale_q [B,Hq], descale_k / descale_v [B,Hkv] fp32 CUDA tensors.  Returns (o bf16, lse)."""
+    import torch
+
+    def codes(t, n):
+        if not isinstance(t, torch.Tensor):
+            raise TypeError("%s must be a torch.Tensor" % n)
+        if t.dtype == getattr(torch, "float8_e4m3fn", None):
+            t = t.view(torch.uint8)
+        _check(t, n, torch.uint8, 4)
+        return t
+
+    q, k, v = codes(q, "q"), codes(k, "k"), codes(v, "v")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    _check(descale_q, "descale_q", torch.float32, 2)
+    _check(descale_k, "descale_k", torch.float32, 2)
+    _check(descale_v, "descale_v", torch.float32, 2)
+    if o is None:
+        o = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(descale_q),
+                            _ptr(descale_k), _ptr(descale_v), B, Hq, Hkv, Nq, Nk, d,
+                            int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
+    _raise(rc, "attn_fwd_fp8")
     return o, lse
 
 

@@ -70,9 +70,10 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    void (*kernels[4])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
-        fwd::fwd_bf16_sm100_kernel<false, true>, fwd::fwd_bf16_sm100_kernel<true, true>};
+        fwd::fwd_bf16_sm100_kernel<false, true>,  fwd::fwd_bf16_sm100_kernel<true, true>,
+        fwd::fwd_fp8_sm100_kernel<false>,         fwd::fwd_fp8_sm100_kernel<true>};
     for (auto* kern : kernels) {
       const int rc = cuda_status(cudaFuncSetAttribute(
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
@@ -171,6 +172,22 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// 3-D tiled TMA map over [heads][rows][128] E4M3 codes (one byte each), read as boxes of the full
+// 128-byte row width x 128 rows x 1 head with the 128-byte swizzle.
+int encode_map_e4m3(CUtensorMap* map, const void* base, int rows, int heads) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD),
+                                 static_cast<cuuint64_t>(rows) * fwd::kD};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -412,6 +429,58 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
     fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
     fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                 const float* descale_q, const float* descale_k, const float* descale_v, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                 float scale, attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  const bool q_empty = B == 0 || Nq == 0, kv_empty = B == 0 || Nk == 0;
+  if (!q_empty && (descale_q == nullptr || (!kv_empty && (descale_k == nullptr ||
+                                                          descale_v == nullptr))))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != fwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (q_empty) return ATTN_OK;
+  if (Nk == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq * Nq, d, st);
+  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
+      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  fwd::Params p;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.c = scale * kLog2e;
+  if (p.c == 0.f) p.c = 1e-30f;
+  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.cu_q = nullptr;
+  p.cu_k = nullptr;
+  p.descale_q = descale_q;
+  p.descale_k = descale_k;
+  p.descale_v = descale_v;
+  const dim3 grid(static_cast<unsigned>(units));
+  if (scale < 0.f)
+    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  else
+    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "dev/ptx_f8.cuh"
 
 namespace attn {
 namespace fwd {
@@ -54,6 +55,11 @@ static_assert(kThreads * kRegsLaunch <= 65536, "launch register budget");
 constexpr uint32_t kTileBytes = kBM * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column half
 constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
+// E4M3 operands (kFp8): P is scaled by kPScaleF8 before it is rounded to E4M3 and the running
+// maximum is refreshed whenever it grows by more than 1 (log2 units), so scaled P stays below
+// 2 * 128 = 256 <= 448 (the largest E4M3 value) while small weights keep 128x more range.
+constexpr float kPScaleF8 = 128.0f;
+constexpr float kRescaleThresholdF8 = 1.0f;
 
 struct Params {
   int B, Hq, Hkv, Nq, Nk, G;  // packed variable-length mode: B = number of sequences,
@@ -65,6 +71,10 @@ struct Params {
   int num_qblocks;
   __nv_bfloat16* o;
   float* lse;
+  // E4M3 operands only: per (b, head) factors that turn the codes into values
+  const float* descale_q;  // [B][Hq]
+  const float* descale_k;  // [B][Hkv]
+  const float* descale_v;  // [B][Hkv]
 };
 
 struct __align__(1024) Smem {
@@ -94,11 +104,14 @@ __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); 
 // attention is block diagonal, reset at every sequence boundary given by cu_seqlens); tensors
 // are token-major, Q/O [total_q][Hq][d], K/V [total_k][Hkv][d], LSE [total_q][Hq], and each
 // sequence is masked on its own (p_i = i + Nk_s - Nq_s).  Otherwise the dense [B][H][N][d] form.
-template <bool kNeg, bool kVarlen>
-__global__ void __launch_bounds__(kThreads, 1)
-    fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
-                          const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+// kFp8: Q, K, V hold E4M3 codes (a 128 x 128 tile is 16 KB, one 128-byte-wide TMA box) and both
+// products run as kind::f8f6f4 MMAs, P being rounded to E4M3 (times kPScaleF8) in TMEM.
+template <bool kNeg, bool kVarlen, bool kFp8>
+__device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
+                                          const CUtensorMap& tm_v, const Params& p) {
+  constexpr int kHalves = kFp8 ? 1 : 2;                          // TMA boxes per tile
+  constexpr uint32_t kTile = kFp8 ? kTileBytes / 2 : kTileBytes;  // bytes of one tile
+  constexpr float kThreshold = kFp8 ? kRescaleThresholdF8 : kRescaleThreshold;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
@@ -184,9 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool q_issued = false;
       if (nk > 0) {
         const uint32_t bq = dev::smem_u32(&sm.bar_q);
-        dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes);
+        dev::mbar_arrive_expect_tx(bq, 2 * kTile);
         for (int t = 0; t < 2; ++t)
-          for (int half = 0; half < 2; ++half)
+          for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
                                q_base + r0 + t * kBM, h);
@@ -200,8 +213,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = ((j >> 1) & 1) ^ 1;
           if (!wait_bounded(dev::smem_u32(&sm.bar_kempty[s]), ph, abort)) break;
           const uint32_t bk = dev::smem_u32(&sm.bar_kfull[s]);
-          dev::mbar_arrive_expect_tx(bk, kTileBytes);
-          for (int half = 0; half < 2; ++half)
+          dev::mbar_arrive_expect_tx(bk, kTile);
+          for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
                                k_base + kt * kBN, h / p.G);
@@ -211,8 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ++k_issued;
           if (!wait_bounded(dev::smem_u32(&sm.bar_vempty[s]), ph, abort)) break;
           const uint32_t bv = dev::smem_u32(&sm.bar_vfull[s]);
-          dev::mbar_arrive_expect_tx(bv, kTileBytes);
-          for (int half = 0; half < 2; ++half)
+          dev::mbar_arrive_expect_tx(bv, kTile);
+          for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
                                k_base + kt * kBN, h / p.G);
@@ -236,8 +249,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ============================ tcgen05.mma issuer =============================
     if (lane == 0 && nk > 0) {
-      constexpr uint32_t idesc_s = dev::idesc_bf16_f32(kBM, kBN, 0, 0);  // Q, K both K-major
-      constexpr uint32_t idesc_o = dev::idesc_bf16_f32(kBM, kD, 0, 1);   // P (TMEM), V MN-major
+      // Q, K both K-major; P (TMEM), V MN-major
+      constexpr uint32_t idesc_s = kFp8 ? dev::idesc_e4m3_f32(kBM, kBN, 0, 0)
+                                        : dev::idesc_bf16_f32(kBM, kBN, 0, 0);
+      constexpr uint32_t idesc_o = kFp8 ? dev::idesc_e4m3_f32(kBM, kD, 0, 1)
+                                        : dev::idesc_bf16_f32(kBM, kD, 0, 1);
       const uint32_t q_base[2] = {dev::smem_u32(sm.q[0]), dev::smem_u32(sm.q[1])};
       const uint32_t tm_s[2] = {tmem + 0, tmem + 128};
       const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
@@ -256,19 +272,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t a0 = t ? dq[1] : dq[0];
         const uint64_t b0 = s ? dk[1] : dk[0];
         const uint32_t d = t ? tm_s[1] : tm_s[0];
+        if constexpr (kFp8) {
+          // K = 32 one-byte elements (32 bytes) per MMA, all inside one 128-byte swizzle row
 #pragma unroll
-        for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-          dev::umma_ss(d, a0 + koff, b0 + koff, idesc_s, ks > 0 ? 1u : 0u);
+          for (int ks = 0; ks < kD / 32; ++ks)
+            dev::umma_ss_f8(d, a0 + ks * 2, b0 + ks * 2, idesc_s, ks > 0 ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < kD / 16; ++ks) {
+            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+            dev::umma_ss(d, a0 + koff, b0 + koff, idesc_s, ks > 0 ? 1u : 0u);
+          }
         }
       };
       auto issue_pv = [&](int t, int s, bool acc) {
         const uint64_t b0 = s ? dv[1] : dv[0];
         const uint32_t d = t ? tm_o[1] : tm_o[0];
         const uint32_t a = t ? tm_s[1] : tm_s[0];
+        if constexpr (kFp8) {
+          // 32 keys per MMA: 8 TMEM columns of packed E4M3 P, 32 rows (4 KB) of V
 #pragma unroll
-        for (int ks = 0; ks < kBN / 16; ++ks)
-          dev::umma_ts(d, a + ks * 8, b0 + ((ks * 16 * 128) >> 4), idesc_o, (acc || ks > 0) ? 1u : 0u);
+          for (int ks = 0; ks < kBN / 32; ++ks)
+            dev::umma_ts_f8(d, a + ks * 8, b0 + ((ks * 32 * 128) >> 4), idesc_o,
+                            (acc || ks > 0) ? 1u : 0u);
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < kBN / 16; ++ks)
+            dev::umma_ts(d, a + ks * 8, b0 + ((ks * 16 * 128) >> 4), idesc_o,
+                         (acc || ks > 0) ? 1u : 0u);
+        }
       };
 
       // K_j lives in k[j & 1] (phase (j >> 1) & 1 of its barriers), V_j likewise in v[j & 1]
@@ -348,7 +380,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_o = tmem + lane_off + 256 + t * 128;
     const int P0 = r0 + t * kBM + off;  // key position of the tile's first row
     const int prow = P0 + row;          // key position of this thread's row
-    const float c = p.c;
+    // scores in log2 units: c = scale * log2(e), times the Q and K descale factors for E4M3
+    const float c = kFp8 ? p.c * __ldg(p.descale_q + bh) * __ldg(p.descale_k + bkv) : p.c;
     const float masked = kNeg ? pos_inf() : neg_inf();
     float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
@@ -408,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float tmax = (mx == masked) ? neg_inf() : mx * c;
       const float m_new = fmaxf(m_ref, tmax);
       float alpha = 1.f;
-      if (m_new > m_ref + kRescaleThreshold) {
+      if (m_new > m_ref + kThreshold) {
         alpha = dev::ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
         m_ref = m_new;
       }
@@ -428,21 +461,39 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
 
-      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t; the row sum
-      // accumulates in 8 independent packed pairs
+      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t (E4M3: four
+      // codes of kPScaleF8 * P per column over the first 32); the row sum accumulates in 8
+      // independent packed pairs
       float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+        if constexpr (kFp8) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const int col = half * 64 + e;
-          const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
-          const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
-          acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
-          pk[e >> 1] = dev::pack_bf16x2(p0, p1);
+          for (int e = 0; e < 64; e += 4) {
+            const int col = half * 64 + e;
+            const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
+            const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
+            const float p2 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 2]), c, -m_use));
+            const float p3 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 3]), c, -m_use));
+            acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
+            acc[((e >> 1) + 1) & 3] = dev::add2(acc[((e >> 1) + 1) & 3], make_float2(p2, p3));
+            pk[e >> 2] = dev::pack_e4m3x4(p0 * kPScaleF8, p1 * kPScaleF8, p2 * kPScaleF8,
+                                          p3 * kPScaleF8);
+          }
+          dev::tmem_st16(t_s + half * 16, pk);
+        } else {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const int col = half * 64 + e;
+            const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
+            const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
+            acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
+            pk[e >> 1] = dev::pack_bf16x2(p0, p1);
+          }
+          dev::tmem_st32(t_s + half * 32, pk);
         }
-        dev::tmem_st32(t_s + half * 32, pk);
       }
       acc[0] = dev::add2(acc[0], acc[1]);
       acc[2] = dev::add2(acc[2], acc[3]);
@@ -461,7 +512,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tc_fence_after();
       const int grow = r0 + t * kBM + row;
       const bool valid = grow < nq;
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      // E4M3: undo the scale of P and apply the V descale factor
+      const float o_mul = kFp8 ? __ldg(p.descale_v + bkv) / kPScaleF8 : 1.f;
+      const float inv_l = l > 0.f ? o_mul / l : 0.f;
       const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + h
                                   : static_cast<size_t>(bh) * p.Nq + grow;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
@@ -501,6 +554,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tc_fence_after();
     dev::tmem_dealloc(tmem, 512);
   }
+}
+
+// bf16 Q, K, V (dense or packed variable-length)
+template <bool kNeg, bool kVarlen>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  fwd_sm100<kNeg, kVarlen, false>(tm_q, tm_k, tm_v, p);
+}
+
+// E4M3 Q, K, V with per-(b, head) descale factors (dense)
+template <bool kNeg>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                         const __grid_constant__ CUtensorMap tm_k,
+                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  fwd_sm100<kNeg, false, true>(tm_q, tm_k, tm_v, p);
 }
 
 }  // namespace fwd

@@ -124,6 +124,22 @@ ATTN_API int attn_fwd_varlen(const void *q, const void *k, const void *v, void *
                              attn_stream_t stream);
 
 /*
+ * attn_fwd_fp8 - attn_fwd on E4M3 (8-bit floating point) Q, K, V ("Attention Research",
+ * section 2: FlashAttention-3's FP8 path, and FP8/FP4 attention numerics as remaining work).
+ *   q bytes [B][Hq][Nq][d], k, v bytes [B][Hkv][Nk][d]: E4M3 codes (1 sign, 4 exponent bits
+ *   with bias 7, 3 mantissa bits, largest finite 448); element (b, h, i, t) of Q stands for
+ *   descale_q[b*Hq + h] * E4M3(q[b][h][i][t]), likewise K and V with descale_k, descale_v
+ *   [B][Hkv] (device fp32 arrays, every factor > 0).  o bf16 [B][Hq][Nq][d], lse fp32 or NULL.
+ *   Both products run on the tensor cores as E4M3 x E4M3 with fp32 accumulation; the weights P
+ *   (times 128) are rounded to E4M3 for the P V product, the row sums stay fp32.  Masks,
+ *   scale and the other rules as attn_fwd (dense layout only).
+ */
+ATTN_API int attn_fwd_fp8(const void *q, const void *k, const void *v, void *o, float *lse,
+                          const float *descale_q, const float *descale_k, const float *descale_v,
+                          int B, int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind, int window,
+                          int n_sink, float scale, attn_stream_t stream);
+
+/*
  * attn_fwd_f32 - the same operation on fp32 Q, K, V, O (fp32 arithmetic throughout).
  *   d in {64, 128}; all other arguments and rules as attn_fwd.
  */

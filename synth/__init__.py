@@ -84,6 +84,55 @@ def normal_bf16_bits(seed: int, tensor_id: int, shape) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------------------------
+# FP8 E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities, largest
+# finite 448, code 0x7F / 0xFF is NaN) for the FP8 workloads' inputs.
+# --------------------------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def _e4m3_magnitudes() -> np.ndarray:
+    """Values of the non-negative finite codes 0x00 .. 0x7E, increasing with the code."""
+    codes = np.arange(0x7F, dtype=np.int64)
+    e, m = codes >> 3, codes & 7
+    return np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+
+
+def f32_to_e4m3_bits(x: np.ndarray) -> np.ndarray:
+    """Round to the nearest E4M3 value (ties to an even code), saturating at +-448; uint8 codes."""
+    x = np.asarray(x, dtype=np.float64)
+    mags = _e4m3_magnitudes()
+    a = np.minimum(np.abs(x), E4M3_MAX)
+    i = np.clip(np.searchsorted(mags, a), 1, len(mags) - 1)
+    lo, hi = mags[i - 1], mags[i]
+    down, up = a - lo, hi - a
+    code = np.where(down < up, i - 1, np.where(up < down, i, np.where((i - 1) % 2 == 0, i - 1, i)))
+    code = np.where(a >= E4M3_MAX, 0x7E, code)
+    return (code | np.where(np.signbit(x), 0x80, 0)).astype(np.uint8)
+
+
+def e4m3_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """Exact values of E4M3 codes (NaN codes are not produced by f32_to_e4m3_bits)."""
+    b = np.asarray(bits, dtype=np.uint8).astype(np.int64)
+    mag = np.append(_e4m3_magnitudes(), np.nan)[b & 0x7F]
+    return np.where(b & 0x80, -mag, mag).astype(np.float32)
+
+
+def normal_e4m3(seed: int, tensor_id: int, shape, head_axes: int = 2):
+    """iid N(0,1) (as ``normal_f32``) quantised to E4M3 with one scale per slice over the first
+    ``head_axes`` axes (per (b, head)): scale = amax / 448, code = E4M3(x / scale).
+
+    Returns (codes uint8 of ``shape``, scales float32 of shape[:head_axes]); the represented
+    values are scale * e4m3_bits_to_f32(codes)."""
+    x = normal_f32(seed, tensor_id, shape).astype(np.float64)
+    lead = tuple(shape[:head_axes])
+    flat = x.reshape(lead + (-1,))
+    amax = np.abs(flat).max(axis=-1)
+    scales = (np.maximum(amax, 1e-30) / E4M3_MAX).astype(np.float32)
+    codes = f32_to_e4m3_bits(flat / scales.astype(np.float64)[..., None])
+    return codes.reshape(shape), scales
+
+
+# --------------------------------------------------------------------------------------------
 # torch implementation of the same counter-based stream (used to fill large device buffers
 # directly on the GPU; equality with the numpy stream is checked on the CPU by the tests).
 # --------------------------------------------------------------------------------------------

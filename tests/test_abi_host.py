@@ -138,3 +138,16 @@ def test_bwd_workspace_size():
     assert A.attn_bwd_workspace_bytes(4, 16, 2048) == 2 * 4 * 16 * 2048 * 4
     assert A.attn_bwd_workspace_bytes(1, 2, 300) == 2 * 1 * 2 * 384 * 4  # rows padded to 128
     assert A.attn_bwd_workspace_bytes(0, 2, 300) == 0
+
+
+def test_fp8_invalid_arguments_are_rejected(lib):
+    E = A.ATTN_ERR_INVALID_ARG
+
+    def fp8(q=P, k=P, v=P, o=P, dq=P, dk=P, dv=P, mask=1, w=0, s=0, scale=0.1, d=128):
+        return lib.attn_fwd_fp8(q, k, v, o, N, dq, dk, dv, 1, 2, 1, 4, 4, d, mask, w, s, scale, N)
+
+    for name in ("q", "k", "v", "o", "dq", "dk", "dv"):
+        assert fp8(**{name: N}) == E, name
+    assert fp8(mask=5) == E
+    assert fp8(scale=float("inf")) == E
+    assert fp8(d=64) == A.ATTN_ERR_UNSUPPORTED

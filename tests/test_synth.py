@@ -43,3 +43,37 @@ def test_streams_are_distinct_and_normal():
     assert abs(np.corrcoef(q, k)[0, 1]) < 0.01 and abs(np.corrcoef(q, q3)[0, 1]) < 0.01
     # tails of N(0,1): P(|z| > 3) = 0.0027
     assert abs(np.mean(np.abs(q) > 3.0) - 0.0027) < 0.0006
+
+
+def test_e4m3_codes_round_trip_and_order():
+    codes = np.arange(256, dtype=np.uint8)
+    finite = codes[(codes & 0x7F) != 0x7F]
+    vals = synth.e4m3_bits_to_f32(finite)
+    assert np.array_equal(synth.f32_to_e4m3_bits(vals)[vals != 0], finite[vals != 0])
+    mags = synth.e4m3_bits_to_f32(np.arange(0x7F, dtype=np.uint8)).astype(np.float64)
+    assert np.all(np.diff(mags) > 0)
+    # published anchors of the format: smallest subnormal, smallest normal, one, largest finite
+    assert mags[1] == 2.0 ** -9 and mags[8] == 2.0 ** -6 and mags[0x38] == 1.0 and mags[-1] == 448.0
+
+
+def test_e4m3_rounding_matches_torch():
+    import torch
+
+    rng = np.random.default_rng(5)
+    x = np.concatenate([rng.standard_normal(20000) * 30, rng.uniform(-448, 448, 20000),
+                        rng.standard_normal(5000) * 1e-3]).astype(np.float32)
+    ours = synth.f32_to_e4m3_bits(x)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    assert synth.f32_to_e4m3_bits(np.array([1000.0, -1e9]))[0] == 0x7E  # saturates at 448
+
+
+def test_normal_e4m3_per_head_scales():
+    codes, scales = synth.normal_e4m3(3, synth.Q_ID, (2, 3, 50, 16))
+    assert codes.shape == (2, 3, 50, 16) and scales.shape == (2, 3)
+    x = synth.normal_f32(3, synth.Q_ID, (2, 3, 50, 16)).astype(np.float64)
+    deq = synth.e4m3_bits_to_f32(codes).astype(np.float64) * scales[..., None, None]
+    # every element within half an E4M3 step (relative 2^-4) of the drawn value, amax exact-ish
+    rel = np.abs(deq - x) / np.maximum(np.abs(x), 2.0 ** -6 * scales.max())
+    assert rel.max() <= 2.0 ** -4 + 1e-6
+    assert np.all(np.abs(synth.e4m3_bits_to_f32(codes)).reshape(2, 3, -1).max(axis=-1) == 448.0)
