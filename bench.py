@@ -85,11 +85,12 @@ DECODE = "decode_b64_h32_kv8_n32768_d128"
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the sources of that
 # kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
-    "causal_b4_h16_n2048_d128": {"bytes": 140389376, "src": "5252e77825f07a1a"},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 455650304, "src": "5252e77825f07a1a"},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 677068032, "src": "5252e77825f07a1a"},
-    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293632000, "src": "5252e77825f07a1a"},
-    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 827440128, "src": "5252e77825f07a1a"},
+    "causal_b4_h16_n2048_d128": {"bytes": 145144064, "src": "59bdcb2a74df9252"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 471887360, "src": "59bdcb2a74df9252"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 686198016, "src": "59bdcb2a74df9252"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293224960, "src": "59bdcb2a74df9252"},
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 828471040, "src": "59bdcb2a74df9252"},
+    "fp8_causal_b4_h16_n2048_d128": {"bytes": 53103360, "src": "59bdcb2a74df9252"},
     # the backward step's three kernels together (prep + dK/dV + dQ)
     "bwd_causal_b4_h16_n2048_d128": {"bytes": 470214400, "src": "bc71c31cb46971e0"},
     # captured on the 8-sequence cases; the cache is read once per sequence, so the
