@@ -1,5 +1,7 @@
-// bf16 exact attention forward for sm_100a: TMA -> shared memory -> tcgen05.mma (TMEM
+// Exact attention forward for sm_100a: TMA -> shared memory -> tcgen05.mma (TMEM
 // accumulators) -> online softmax in registers -> P back to TMEM -> tcgen05.mma for P V.
+// Operands are bf16 (fwd_bf16_sm100_kernel, dense or packed variable-length) or E4M3 codes with
+// per-(b, head) scales (fwd_fp8_sm100_kernel); every mask of common.cuh is supported.
 //
 // The method: "FlashAttention and sparse attention" (grasp.study), section 1 (tiling, kernel
 // fusion, online softmax: running max and running sum, earlier partial results rescaled when
