@@ -59,3 +59,13 @@ def test_reference_arm_does_nothing_on_other_ranks():
     class Args:
         workload, warmup, steps, gpus = None, 3, 5, 2
     assert bench.run_reference(Args(), rank=1, world=2) == 0
+
+
+def test_kernel_hash_ignores_comments_and_layout():
+    import bench
+
+    code = "int f(int a) {\n  return a + 1;  // one more\n}\n/* note */"
+    assert bench.code_tokens(code) == bench.code_tokens("int f(int a) { return a + 1; }")
+    assert bench.code_tokens(code) != bench.code_tokens("int f(int a) { return a + 2; }")
+    for fam in bench.FAMILY_SOURCES:
+        assert len(bench.kernel_sources_hash(fam)) == 16

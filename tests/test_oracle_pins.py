@@ -317,6 +317,13 @@ def test_pair_counts_at_workload_sizes():
     assert acc.attn_flops(4, 16, 2048, 2048, 128, CAUSAL) == 68753031168
     assert acc.attn_flops(2, 32, 8192, 8192, 128, CAUSAL) == 1099645845504
     assert acc.decode_bytes(64, 32, 8, 32768, 128) == 8589934592 + 2 * 128 * 2 * 64 * 32 + 4 * 64 * 32
+    # local + global workload: the row-wise count against the oracle's enumeration
+    assert acc.visible_pairs(32768, 32768, LOCAL, 2048, 4) == 130299884
+    assert O.visible_pairs(32768, 32768, LOCAL, 2048, 4) == 130299884
+    # backward: five products of 2*d per visible pair, 2.5x the forward
+    assert acc.attn_bwd_flops(4, 16, 2048, 2048, 128, CAUSAL) == 171882577920
+    assert 2 * acc.attn_bwd_flops(4, 16, 2048, 2048, 128, CAUSAL) == 5 * acc.attn_flops(
+        4, 16, 2048, 2048, 128, CAUSAL)
     # paged: plus one int32 block-table entry per 16-key page and one int32 length per sequence
     assert acc.decode_paged_bytes(64, 32, 8, 32768, 128, 16) == \
         acc.decode_bytes(64, 32, 8, 32768, 128) + 4 * 64 * 2048 + 4 * 64
