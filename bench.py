@@ -327,7 +327,8 @@ class Workload:
                                 n_sink=w["n_sink"])
             self.inputs = [q, k, v, o, lse, dout]
             self.grads = [torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)]
-            self.ws = torch.empty(A.attn_bwd_workspace_bytes(B, Hq, N), dtype=torch.uint8,
+            self.ws = torch.empty(A.attn_bwd_workspace_bytes(B, Hq, N, N, w["mask"], w["window"],
+                                                             w["n_sink"]), dtype=torch.uint8,
                                   device="cuda")
             self.launches_per_step = 3
         else:

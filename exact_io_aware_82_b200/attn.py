@@ -77,7 +77,7 @@ def lib():
         L.attn_decode_paged.restype = i
         L.attn_fwd_fp8.argtypes = [vp] * 8 + [i] * 9 + [f, vp]
         L.attn_fwd_fp8.restype = i
-        L.attn_bwd_workspace_bytes.argtypes = [i] * 3
+        L.attn_bwd_workspace_bytes.argtypes = [i] * 7
         L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.attn_bwd.argtypes = [vp] * 9 + [i] * 9 + [f, vp, ctypes.c_size_t, vp]
         L.attn_bwd.restype = i
@@ -232,8 +232,9 @@ def attn_fwd_f32(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sin
     return o, lse
 
 
-def attn_bwd_workspace_bytes(B, Hq, Nq) -> int:
-    return int(lib().attn_bwd_workspace_bytes(B, Hq, Nq))
+def attn_bwd_workspace_bytes(B, Hq, Nq, Nk, mask_kind=MASK_FULL, window=0, n_sink=0) -> int:
+    return int(lib().attn_bwd_workspace_bytes(B, Hq, Nq, Nk, int(mask_kind), int(window),
+                                              int(n_sink)))
 
 
 def attn_bwd(q, k, v, o, lse, dout, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None,
@@ -255,8 +256,9 @@ def attn_bwd(q, k, v, o, lse, dout, mask_kind=MASK_FULL, window=0, n_sink=0, sca
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     if workspace is None:
-        workspace = torch.empty(max(attn_bwd_workspace_bytes(B, Hq, Nq), 16), dtype=torch.uint8,
-                                device=q.device)
+        workspace = torch.empty(max(attn_bwd_workspace_bytes(B, Hq, Nq, Nk, mask_kind, window,
+                                                             n_sink), 16),
+                                dtype=torch.uint8, device=q.device)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
                         _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, int(mask_kind), int(window),

@@ -112,10 +112,28 @@ int configure_bwd(DeviceInfo* info) {
   return ATTN_OK;
 }
 
-// Backward workspace: LSE * log2(e) and D per query row, rows padded to whole 128-row tiles.
-size_t bwd_ws_bytes(int B, int Hq, int Nq) {
-  const size_t npad = static_cast<size_t>((Nq + bwd::kT - 1) / bwd::kT) * bwd::kT;
-  return 2 * static_cast<size_t>(B) * Hq * npad * sizeof(float);
+// Backward workspace, in this order: LSE * log2(e) and D per query row (fp32, rows padded to
+// whole 128-row tiles); the dS block offsets of the key blocks (int32, num_kblocks + 1); the
+// dS^T blocks (bf16 128 x 128, one per visible (key block, query tile) pair and query head).
+struct BwdLayout {
+  size_t npad, pairs, off_bytes, ds_offset, total;
+};
+
+BwdLayout bwd_layout(int B, int Hq, int Nq, int Nk, const MaskSpec& m) {
+  BwdLayout L{};
+  const int nqt = (Nq + bwd::kT - 1) / bwd::kT, nkb = (Nk + bwd::kT - 1) / bwd::kT;
+  L.npad = static_cast<size_t>(nqt) * bwd::kT;
+  size_t pairs = 0;
+  for (int kb = 0; kb < nkb; ++kb) {
+    const int c0 = kb * bwd::kT, c1 = (c0 + bwd::kT < Nk ? c0 + bwd::kT : Nk) - 1;
+    pairs += static_cast<size_t>(bwd::query_tiles(m, c0, c1, Nk - Nq, Nq).count());
+  }
+  L.pairs = pairs;
+  const size_t vec = 2 * static_cast<size_t>(B) * Hq * L.npad * sizeof(float);
+  L.off_bytes = (static_cast<size_t>(nkb) + 1) * sizeof(int);
+  L.ds_offset = (vec + L.off_bytes + 255) & ~size_t(255);
+  L.total = L.ds_offset + static_cast<size_t>(B) * Hq * pairs * bwd::kT * bwd::kT * 2;
+  return L;
 }
 
 // Common argument rules of the forward entry points.
@@ -592,9 +610,14 @@ int attn_decode_paged(const void* q, const void* k_cache, const void* v_cache, v
                     workspace, workspace_bytes, st, info, &pg);
 }
 
-size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq) {
-  if (B < 1 || Hq < 1 || Nq < 0) return 0;
-  return bwd_ws_bytes(B, Hq, Nq);
+size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int Nk, int mask_kind, int window,
+                                int n_sink) {
+  if (B < 1 || Hq < 1 || Nq < 0 || Nk < 0) return 0;
+  if (mask_kind < ATTN_MASK_FULL || mask_kind > ATTN_MASK_LOCAL_GLOBAL || n_sink < 0 ||
+      (mask_kind == ATTN_MASK_SLIDING && window < 1) ||
+      (mask_kind == ATTN_MASK_LOCAL_GLOBAL && window < 0))
+    return 0;
+  return bwd_layout(B, Hq, Nq, Nk, make_mask(mask_kind, window, n_sink, Nk)).total;
 }
 
 int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -629,7 +652,11 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   const long long units_q = static_cast<long long>(nqt) * B * Hq;
   const long long units_kv = static_cast<long long>(nkb) * B * Hkv;
   if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
-  if (workspace == nullptr || workspace_bytes < bwd_ws_bytes(B, Hq, Nq) || !aligned16(workspace))
+  const MaskSpec mask = make_mask(mask_kind, window, n_sink, Nk);
+  const BwdLayout L = bwd_layout(B, Hq, Nq, Nk, mask);
+  if (static_cast<double>(B) * Hq * static_cast<double>(L.pairs) > 2147483647.0)
+    return ATTN_ERR_UNSUPPORTED;  // dS block index of the dQ kernel's tensor map
+  if (workspace == nullptr || workspace_bytes < L.total || !aligned16(workspace))
     return ATTN_ERR_WORKSPACE;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;  // the tensor-map encoder
   if ((rc = configure_bwd(info)) != ATTN_OK) return rc;
@@ -644,7 +671,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   p.Nq = Nq;
   p.Nk = Nk;
   p.G = Hq / Hkv;
-  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.mask = mask;
   p.scale = scale;
   p.c = scale * kLog2e;
   p.num_kblocks = nkb;
@@ -657,18 +684,35 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   p.dq = static_cast<__nv_bfloat16*>(dq);
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.ds_off = reinterpret_cast<int*>(dsum + static_cast<size_t>(B) * Hq * p.npad);
+  p.ds = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + L.ds_offset);
+  p.ds_pairs = static_cast<long long>(L.pairs);
+  // dS^T blocks as a 3-D tensor (queries, keys, block) for the dQ kernel's TMA loads
+  CUtensorMap tds;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(bwd::kT), static_cast<cuuint64_t>(bwd::kT),
+                                static_cast<cuuint64_t>(B) * Hq * (L.pairs > 0 ? L.pairs : 1)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(bwd::kT) * 2,
+                                   static_cast<cuuint64_t>(bwd::kT) * bwd::kT * 2};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    if (g_encode(&tds, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.ds, dims, strides, box, estride,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_UNSUPPORTED;
+  }
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
   bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
                                                bwd::kPrepRowsPerBlock),
                          256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
-      dsum, Nq, p.npad, prow);
+      dsum, Nq, p.npad, prow, mask, nkb, p.ds_off);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(units_kv), bwd::kThreads, bwd::kSmemKVBytes, st>>>(
       tq, tk, tv, tdo, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
-      tq, tk, tv, tdo, p);
+      tds, tk, p);
   return cuda_status(cudaGetLastError());
 }
 

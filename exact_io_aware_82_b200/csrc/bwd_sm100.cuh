@@ -19,11 +19,14 @@
 //     the row warps (one TMEM lane = one key each) turn them into P^T and dS^T (bf16, written
 //     back over S^T and dP^T); then dV += P^T dO and dK += dS^T Q with P^T / dS^T as the A operand
 //     read from TMEM.
-//  3. bwd_dq_kernel: one CTA per (b, query head, 128-row query tile), walking the key tiles the
-//     tile sees: S = Q K^T, dP = dO V^T, dS in TMEM (bf16), dQ += dS K.
-// Splitting dQ from dK/dV recomputes S and dP once more (7 MMA tiles per visible tile pair
-// instead of 5) but needs neither atomics nor a second accumulator set, and the result does not
-// depend on the order in which CTAs finish.
+//     It also writes each (key block, query tile) block of dS^T (bf16, the values its own
+//     dK MMA used) to a workspace slot.
+//  3. bwd_dq_kernel: one CTA per (b, query head, 128-row query tile) computes dQ = scale dS K as
+//     a plain tensor-core product over the dS^T blocks of the tile's key tiles: no recomputation
+//     and no softmax, so it is bound by reading dS (2 bytes per visible pair).
+// Handing dS over through HBM instead of recomputing it (or of atomically adding dQ partials)
+// costs a write and a read of dS but keeps every product on the tensor core exactly once, and
+// the result does not depend on the order in which CTAs finish.
 //
 // Roles of each 352-thread CTA: warps 0-7 are the row workers (warps w and w+4 share TMEM lanes
 // 32(w%4) .. 32(w%4)+31 and split the columns), one thread of warp 8 issues the score MMAs, one
@@ -64,22 +67,38 @@ struct Params {
   int num_kblocks;    // ceil(Nk / 128)
   int num_qtiles;     // ceil(Nq / 128)
   int npad;           // num_qtiles * 128: row stride of lse2 and dsum
+  // dS^T handed from the dK/dV kernel to the dQ kernel: slot (b*Hq + h) * ds_pairs + ds_off[kb] +
+  // (index of the query tile in key block kb's query-tile range) holds the 128 x 128 bf16 block
+  // (keys x queries) of that pair
+  __nv_bfloat16* ds;
+  int* ds_off;         // [num_kblocks + 1], written by the prep kernel
+  long long ds_pairs;  // ds_off[num_kblocks]: blocks per (b, query head)
 };
+
+// Index of query tile qt in key block kb's query-tile range, or -1 if the range misses it.
+__host__ __device__ __forceinline__ int pair_index(const TileRange& r, int qt) {
+  if (qt < r.ns) return qt;
+  if (qt >= r.lo && qt <= r.hi) return r.ns + (qt - r.lo);
+  return -1;
+}
 
 // ------------------------------------------------------------------------------------------
 // helpers
 // ------------------------------------------------------------------------------------------
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
 
-__device__ __forceinline__ int floor_div128(long long a) {
+__host__ __device__ __forceinline__ int imin(int a, int b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int imax(int a, int b) { return a > b ? a : b; }
+
+__host__ __device__ __forceinline__ int floor_div128(long long a) {
   return static_cast<int>(a >= 0 ? a / kT : -((-a + kT - 1) / kT));
 }
 
 // Query tiles whose rows see at least one key of [c0, c1] (off = Nk - Nq; query row i sits at
 // key position i + off), as a TileRange: tiles [0, ns) (the global rows of the local + global
 // mask), then [lo, hi].
-__device__ __forceinline__ TileRange query_tiles(const MaskSpec& m, int c0, int c1, int off,
-                                                 int Nq) {
+__host__ __device__ __forceinline__ TileRange query_tiles(const MaskSpec& m, int c0, int c1,
+                                                          int off, int Nq) {
   const int nqt = (Nq + kT - 1) / kT;
   TileRange r{0, 0, nqt - 1};
   if (m.kind == ATTN_MASK_FULL) return r;
@@ -87,27 +106,27 @@ __device__ __forceinline__ TileRange query_tiles(const MaskSpec& m, int c0, int 
     if (c0 < m.n_sink) return r;  // a global key is seen by every row
     // rows p in [c0 - w, c1 + w], and the global rows 0 <= p < n_global (i < n_global - off)
     const long long g_rows = static_cast<long long>(m.n_sink) - off;
-    const int g_tiles = g_rows <= 0 ? 0 : min(nqt, static_cast<int>((g_rows + kT - 1) / kT));
-    r.lo = max(0, floor_div128(static_cast<long long>(c0) - m.window - off));
-    r.hi = min(r.hi, floor_div128(static_cast<long long>(c1) + m.window - off));
+    const int g_tiles = g_rows <= 0 ? 0 : imin(nqt, static_cast<int>((g_rows + kT - 1) / kT));
+    r.lo = imax(0, floor_div128(static_cast<long long>(c0) - m.window - off));
+    r.hi = imin(r.hi, floor_div128(static_cast<long long>(c1) + m.window - off));
     if (r.lo > r.hi) {  // no window row: the global rows only
       r.ns = g_tiles;
       r.lo = g_tiles;
       r.hi = g_tiles - 1;
     } else if (g_tiles >= r.lo) {
       r.lo = 0;
-      r.hi = max(r.hi, g_tiles - 1);
+      r.hi = imax(r.hi, g_tiles - 1);
     } else {
       r.ns = g_tiles;
     }
     return r;
   }
   // causal: p = i + off >= key  ->  i >= c0 - off for the block's first key
-  r.lo = max(0, floor_div128(static_cast<long long>(c0) - off));
+  r.lo = imax(0, floor_div128(static_cast<long long>(c0) - off));
   // window: p < key + w for keys past the sinks (a block holding a sink key is seen by every
   // later row)
   if (m.kind == ATTN_MASK_SLIDING && c0 >= m.n_sink)
-    r.hi = min(r.hi, floor_div128(static_cast<long long>(c1) + m.window - 1 - off));
+    r.hi = imin(r.hi, floor_div128(static_cast<long long>(c1) + m.window - 1 - off));
   return r;
 }
 
@@ -171,7 +190,18 @@ constexpr int kPrepRowsPerBlock = 64;  // 8 warps x 8 rows
 __global__ void __launch_bounds__(256)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                     const float* __restrict__ lse, float* __restrict__ lse2,
-                    float* __restrict__ dsum, int Nq, int npad, long long padded_rows) {
+                    float* __restrict__ dsum, int Nq, int npad, long long padded_rows,
+                    MaskSpec mask, int num_kblocks, int* __restrict__ ds_off) {
+  // the dS block offsets of the key blocks (a running count of their query tiles)
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    int acc = 0;
+    for (int kb = 0; kb < num_kblocks; ++kb) {
+      ds_off[kb] = acc;
+      const int c0 = kb * kT, c1 = imin(c0 + kT, mask.Nk) - 1;
+      acc += query_tiles(mask, c0, c1, mask.Nk - Nq, Nq).count();
+    }
+    ds_off[num_kblocks] = acc;
+  }
   // a half-warp per row (16 lanes x 16 bytes = one 256-byte row of O and of dO); each warp
   // takes 8 consecutive padded rows, every load issued before the first use
   const int lane = threadIdx.x & 31, sub = lane >> 4, sl = lane & 15;
@@ -411,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int j = c0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.c;
+    const long long ds_base = nsteps > 0 ? p.ds_off[kb] : 0;
     bool ok = true;
     for (int m = 0; m < nsub; ++m) {
       const int n = m >> 1, h = m & 1, s = n & 1;
@@ -477,6 +508,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // has just read (see packed_col)
       dev::tmem_st16(t_st, pk);
       dev::tmem_st16(t_dpt, dk16);
+      {
+        // the same bf16 dS^T values into this (key block, query tile) block for the dQ kernel:
+        // row r (key), columns 64h + 32ch .. +31 (queries)
+        const int hq = hk * p.G + n / nqt;
+        const long long slot = static_cast<long long>(b * p.Hq + hq) * p.ds_pairs + ds_base + n % nqt;
+        uint4* dst = reinterpret_cast<uint4*>(p.ds + slot * (kT * kT) + r * kT + h * kSub + ch * 32);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4)
+          dst[v4] = make_uint4(dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
+      }
       dev::tmem_wait_st();
       dev::tc_fence_before();
       dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
@@ -512,25 +553,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// 3. dQ: one CTA per (b, query head, query tile)
+// 3. dQ = scale dS K: one CTA per (b, query head, query tile), over the dS^T blocks the dK/dV
+//    kernel wrote.  dS^T blocks and K tiles stream through a 3-stage ring; one thread issues
+//    the MMAs (A = dS read MN-major from the [keys][queries] block, B = K MN-major); dQ
+//    accumulates in 128 TMEM columns; warps 0-7 store it.
 // ------------------------------------------------------------------------------------------
+constexpr int kDqStages = 3;
+
 struct __align__(1024) SmemQ {
-  uint8_t q[kTileBytes];
-  uint8_t dout[kTileBytes];
-  uint8_t k[2][kTileBytes];
-  uint8_t v[2][kTileBytes];
-  uint64_t bar_q, bar_kvfull[2], bar_kvempty[2], bar_s[2], bar_p[2], bar_free[2], bar_done;
-  uint64_t bar_drain[2];
+  uint8_t ds[kDqStages][kTileBytes];
+  uint8_t k[kDqStages][kTileBytes];
+  uint64_t bar_full[kDqStages], bar_empty[kDqStages], bar_done, bar_drain;
   uint32_t tmem_base;
   int abort;
+  int any;  // set by the MMA thread: at least one dS block contributed
 };
 constexpr size_t kSmemQBytes = sizeof(SmemQ) + 1024;
 
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v,
-                  const __grid_constant__ CUtensorMap tm_do, const Params p) {
+    bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_ds,
+                  const __grid_constant__ CUtensorMap tm_k, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   SmemQ& sm = *reinterpret_cast<SmemQ*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~uintptr_t(1023));
@@ -547,30 +589,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int last_row = min(r0 + kT, p.Nq) - 1;
   const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kT);
   const int nk = tr.count();
-  const int nsub = 2 * nk;
+  // step jj uses key tile tr.tile(jj) if this query tile is in that key block's range (a pair
+  // outside it has no visible entry and no dS block); every role walks the same list
+  auto pair_slot = [&](int jj, int& kt) -> long long {
+    kt = tr.tile(jj);
+    const int c0 = kt * kT, c1 = min(c0 + kT, p.Nk) - 1;
+    const int idx = pair_index(query_tiles(p.mask, c0, c1, off, p.Nq), qt);
+    if (idx < 0) return -1;
+    return static_cast<long long>(bh) * p.ds_pairs + p.ds_off[kt] + idx;
+  };
 
   if (tid == 0) {
-    dev::mbar_init(dev::smem_u32(&sm.bar_q), 1);
-    for (int s = 0; s < 2; ++s) {
-      dev::mbar_init(dev::smem_u32(&sm.bar_kvfull[s]), 1);
-      dev::mbar_init(dev::smem_u32(&sm.bar_kvempty[s]), 1);
-      dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
-      dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
-      dev::mbar_init(dev::smem_u32(&sm.bar_free[s]), 1);
-      dev::mbar_init(dev::smem_u32(&sm.bar_drain[s]), 1);
+    for (int s = 0; s < kDqStages; ++s) {
+      dev::mbar_init(dev::smem_u32(&sm.bar_full[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_empty[s]), 1);
     }
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
+    sm.any = 0;
     dev::fence_barrier_init();
   }
   if (warp == kLoadWarp && lane == 0) {
-    dev::tma_prefetch_desc(&tm_q);
+    dev::tma_prefetch_desc(&tm_ds);
     dev::tma_prefetch_desc(&tm_k);
-    dev::tma_prefetch_desc(&tm_v);
-    dev::tma_prefetch_desc(&tm_do);
   }
   if (warp == kMmaWarp) {
-    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 128);
     dev::tmem_relinquish();
   }
   dev::tc_fence_before();
@@ -581,155 +626,74 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kLoadWarp) {
     // ================================ TMA producer ================================
-    if (lane == 0 && nk > 0) {
-      const uint32_t bq = dev::smem_u32(&sm.bar_q);
-      dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes);
-      for (int half = 0; half < 2; ++half) {
-        dev::tma_load_3d(dev::smem_u32(sm.q) + half * kHalfBytes, &tm_q, bq, half * 64, r0, bh);
-        dev::tma_load_3d(dev::smem_u32(sm.dout) + half * kHalfBytes, &tm_do, bq, half * 64, r0,
-                         bh);
-      }
-      int issued = 0;
+    if (lane == 0) {
+      int u = 0;
       for (int jj = 0; jj < nk; ++jj) {
-        const int s = jj & 1;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_kvempty[s]), ((jj >> 1) & 1) ^ 1, abort)) break;
-        const int key0 = tr.tile(jj) * kT;
-        const uint32_t bk = dev::smem_u32(&sm.bar_kvfull[s]);
-        dev::mbar_arrive_expect_tx(bk, 2 * kTileBytes);
+        int kt;
+        const long long slot = pair_slot(jj, kt);
+        if (slot < 0) continue;
+        const int s = u % kDqStages;
+        if (!wait_bounded(dev::smem_u32(&sm.bar_empty[s]), ((u / kDqStages) & 1) ^ 1, abort))
+          break;
+        const uint32_t bf = dev::smem_u32(&sm.bar_full[s]);
+        dev::mbar_arrive_expect_tx(bf, 2 * kTileBytes);
         for (int half = 0; half < 2; ++half) {
-          dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64, key0,
-                           bkv);
-          dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bk, half * 64, key0,
-                           bkv);
+          dev::tma_load_3d(dev::smem_u32(sm.ds[s]) + half * kHalfBytes, &tm_ds, bf, half * 64, 0,
+                           static_cast<int>(slot));
+          dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bf, half * 64,
+                           kt * kT, bkv);
         }
-        ++issued;
+        ++u;
       }
-      wait_drain(bq, 0);
-      for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_kvfull[s]), issued, s);
+      // drain: the last copy into each stage has landed
+      for (int s = 0; s < kDqStages; ++s) {
+        const int last = (u - 1 - s) >= 0 ? (u - 1 - s) / kDqStages * kDqStages + s : -1;
+        if (last >= 0) wait_drain(dev::smem_u32(&sm.bar_full[s]), (last / kDqStages) & 1);
+      }
     }
-  } else if (warp == kMmaWarp || warp == kGradWarp) {
-    // ========================= tcgen05.mma issuers (two threads) ==========================
-    if (lane == 0 && nk > 0) {
-      constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);
-      constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);
-      const int role = warp == kMmaWarp ? 0 : 1;
+  } else if (warp == kMmaWarp) {
+    // ============================= tcgen05.mma issuer ==============================
+    if (lane == 0) {
+      constexpr uint32_t idesc = dev::idesc_bf16_f32(kT, kD, 1, 1);  // A and B MN-major
       bool ok = true;
-      if (role == 0) {
-        // S = Q K_h^T and dP = dO V_h^T for sub-step m (keys 64h .. 64h+63 of its key tile)
-        const uint64_t dqa = dev::smem_desc(dev::smem_u32(sm.q), 16, 1024, dev::kSwizzle128B);
-        const uint64_t doa = dev::smem_desc(dev::smem_u32(sm.dout), 16, 1024, dev::kSwizzle128B);
-        uint64_t dkk[2], dvk[2];
-        for (int s = 0; s < 2; ++s) {
-          dkk[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), 16, 1024, dev::kSwizzle128B);
-          dvk[s] = dev::smem_desc(dev::smem_u32(sm.v[s]), 16, 1024, dev::kSwizzle128B);
-        }
-        ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
-        for (int m = 0; ok && m < nsub; ++m) {
-          const int jj = m >> 1, hh = m & 1, s = jj & 1;
-          if (m >= 2 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_free[m & 1]),
-                                            ((m >> 1) - 1) & 1, abort)))
-            break;
-          if (hh == 0 &&
-              !(ok = wait_bounded(dev::smem_u32(&sm.bar_kvfull[s]), (jj >> 1) & 1, abort)))
-            break;
-          dev::tc_fence_after();
-          const uint32_t t_s = tmem + (m & 1) * kSub, t_dp = tmem + 128 + (m & 1) * kSub;
-          const uint32_t hoff = (hh * kSubBytes) >> 4;
-          const uint64_t bk = (s ? dkk[1] : dkk[0]) + hoff, bv = (s ? dvk[1] : dvk[0]) + hoff;
+      int u = 0;
+      for (int jj = 0; ok && jj < nk; ++jj) {
+        int kt;
+        if (pair_slot(jj, kt) < 0) continue;
+        const int s = u % kDqStages;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_full[s]), (u / kDqStages) & 1, abort))) break;
+        dev::tc_fence_after();
+        const uint64_t da = dev::smem_desc(dev::smem_u32(sm.ds[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        const uint64_t db = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-            dev::umma_ss(t_s, dqa + koff, bk + koff, idesc_kk, ks > 0 ? 1u : 0u);
-          }
-#pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-            dev::umma_ss(t_dp, doa + koff, bv + koff, idesc_kk, ks > 0 ? 1u : 0u);
-          }
-          dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
-        }
-      } else {
-        // dQ += dS K_h (K = the 64 keys of the sub-step)
-        uint64_t dkm[2];
-        for (int s = 0; s < 2; ++s)
-          dkm[s] = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-        for (int m = 0; ok && m < nsub; ++m) {
-          const int jj = m >> 1, hh = m & 1, s = jj & 1;
-          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort))) break;
-          dev::tc_fence_after();
-          const uint32_t t_s = tmem + (m & 1) * kSub;
-          const uint64_t bk = s ? dkm[1] : dkm[0];
-#pragma unroll
-          for (int ks = 0; ks < kSub / 16; ++ks)
-            dev::umma_ts(tmem + 256, t_s + packed_col(ks),
-                         bk + ((hh * kSubBytes + ks * 16 * 128) >> 4), idesc_tm,
-                         (m > 0 || ks > 0) ? 1u : 0u);
-          dev::umma_commit(dev::smem_u32(&sm.bar_free[m & 1]));
-          if (hh == 1) dev::umma_commit(dev::smem_u32(&sm.bar_kvempty[s]));  // stage s read for good
-        }
-        if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
+        for (int ks = 0; ks < kT / 16; ++ks)  // 16 keys (2 KB of each block) per MMA
+          dev::umma_ss(tmem, da + ((ks * 2048) >> 4), db + ((ks * 2048) >> 4), idesc,
+                       (u > 0 || ks > 0) ? 1u : 0u);
+        dev::umma_commit(dev::smem_u32(&sm.bar_empty[s]));
+        ++u;
       }
-      dev::umma_commit(dev::smem_u32(&sm.bar_drain[role]));
-      wait_drain(dev::smem_u32(&sm.bar_drain[role]), 0);
+      if (ok && u > 0) dev::umma_commit(dev::smem_u32(&sm.bar_done));
+      dev::umma_commit(dev::smem_u32(&sm.bar_drain));
+      wait_drain(dev::smem_u32(&sm.bar_drain), 0);
+      sm.any = (ok && u > 0) ? 1 : 0;
     }
-  } else {
-    // ========= row workers: one query row each, two warps per row (column halves) =========
+  }
+  // every MMA has completed (the MMA thread drained them) and sm.any is published
+  __syncthreads();
+  if (warp < 8) {
+    // ======================= store: scale * dQ, a column half per warp =======================
     const int r = (warp & 3) * 32 + lane;
     const int ch = warp >> 2;
     const int i = r0 + r;
-    const int prow = i + off;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const float c = p.c;
-    // padding rows (i >= Nq) hold LSE = +inf and D = 0: their weights are zero
-    const float l2 = p.lse2[static_cast<size_t>(bh) * p.npad + i];
-    const float dd = p.dsum[static_cast<size_t>(bh) * p.npad + i];
-    bool ok = true;
-    for (int m = 0; m < nsub; ++m) {
-      ok = wait_bounded(dev::smem_u32(&sm.bar_s[m & 1]), (m >> 1) & 1, abort);
-      if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      dev::tc_fence_after();
-      const uint32_t t_s = tmem + lane_off + (m & 1) * kSub + ch * 32;
-      const uint32_t t_dp = tmem + lane_off + 128 + (m & 1) * kSub + ch * 32;
-      uint32_t sr[32], dr[32];
-      dev::tmem_ld32(t_s, sr);
-      dev::tmem_ld32(t_dp, dr);
-      const int key0 = tr.tile(m >> 1) * kT + (m & 1) * kSub;  // first key of the sub-step
-      uint32_t vis = ~0u;
-      if (!block_visible(p.mask, r0 + off, kT, key0, kSub)) {
-        // visible key columns of this row: (lo <= col <= hi) or col < sk
-        int hi, lo, sk;
-        row_cols(p.mask, prow, key0, hi, lo, sk);
-        vis = row_bits(hi, lo, sk, ch);
-      }
-      dev::tmem_wait_ld();
-#pragma unroll
-      for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
-      uint32_t pk[16];
-#pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -l2));
-        float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -l2));
-        p0 = ((vis >> e) & 1u) ? p0 : 0.f;
-        p1 = ((vis >> (e + 1)) & 1u) ? p1 : 0.f;
-        pk[e >> 1] = dev::pack_bf16x2(p0 * (__uint_as_float(dr[e]) - dd),
-                                      p1 * (__uint_as_float(dr[e + 1]) - dd));
-      }
-      dev::tmem_st16(t_s, pk);  // dS over S (see packed_col)
-      dev::tmem_wait_st();
-      dev::tc_fence_before();
-      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
-    }
-
-    // ---- epilogue: scale * dQ row, bf16, a column half per warp ----
     const bool valid = i < p.Nq;
     __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
-    if (nk == 0) {
-      if (valid) store_zero_row(dst, ch);
-    } else if (ok) {
-      ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
-      if (__all_sync(0xffffffffu, ok)) {
+    if (!sm.any) {
+      if (valid && !*abort) store_zero_row(dst, ch);
+    } else {
+      if (wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort)) {
         dev::tc_fence_after();
-        store_acc_row(tmem + lane_off + 256, p.scale, dst, valid, ch);
+        store_acc_row(tmem + lane_off, p.scale, dst, valid, ch);
       }
     }
   }
@@ -739,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, 512);
+    dev::tmem_dealloc(tmem, 128);
   }
 }
 

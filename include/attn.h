@@ -158,12 +158,17 @@ ATTN_API int attn_fwd_f32(const float *q, const float *k, const float *v, float 
  *   lse  fp32 [B][Hq][Nq], the forward's LSE for the same inputs, mask and scale (required).
  *   d == 128; mask, window, n_sink, scale as attn_fwd.  dq, dk, dv are fully written (rows and
  *   keys that see nothing get zeros).
- *   workspace: device scratch of at least attn_bwd_workspace_bytes(B, Hq, Nq) bytes, 16-byte
- *   aligned, overwritten before it is read.
+ *   workspace: device scratch of at least attn_bwd_workspace_bytes(B, Hq, Nq, Nk, mask_kind,
+ *   window, n_sink) bytes, 16-byte aligned, overwritten before it is read.  Besides two fp32
+ *   values per query row it holds dS, the weight gradient, as bf16 for every 128 x 128 (query
+ *   tile, key block) pair that has a visible entry: the dK/dV kernel writes it, the dQ kernel
+ *   reads it (about 2 bytes per visible pair and query head, e.g. 285 MB for B=4, H=16,
+ *   causal n=2048).
  * Errors: as attn_fwd; ATTN_ERR_WORKSPACE for a missing or short workspace.  Three kernels are
  * queued on `stream`; the result does not depend on their scheduling (no atomics).
  */
-ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq, int Nk, int mask_kind, int window,
+                                         int n_sink);
 
 ATTN_API int attn_bwd(const void *q, const void *k, const void *v, const void *o, const float *lse,
                       const void *dout, void *dq, void *dk, void *dv, int B, int Hq, int Hkv,

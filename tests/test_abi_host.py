@@ -135,9 +135,20 @@ def test_bwd_invalid_arguments_are_rejected(lib):
 
 
 def test_bwd_workspace_size():
-    assert A.attn_bwd_workspace_bytes(4, 16, 2048) == 2 * 4 * 16 * 2048 * 4
-    assert A.attn_bwd_workspace_bytes(1, 2, 300) == 2 * 1 * 2 * 384 * 4  # rows padded to 128
-    assert A.attn_bwd_workspace_bytes(0, 2, 300) == 0
+    def expect(B, Hq, Nq, Nk, pairs):
+        npad = (Nq + 127) // 128 * 128
+        vec = 2 * B * Hq * npad * 4
+        off = ((Nk + 127) // 128 + 1) * 4
+        return (vec + off + 255) // 256 * 256 + B * Hq * pairs * 128 * 128 * 2
+
+    # causal n = 2048: key block kb is seen by query tiles kb .. 15, 136 pairs per head
+    assert A.attn_bwd_workspace_bytes(4, 16, 2048, 2048, A.MASK_CAUSAL) == expect(4, 16, 2048, 2048, 136)
+    # full, 300 x 300: 3 key blocks x 3 query tiles
+    assert A.attn_bwd_workspace_bytes(1, 2, 300, 300, A.MASK_FULL) == expect(1, 2, 300, 300, 9)
+    # window of one key: each key block meets its own query tile only
+    assert A.attn_bwd_workspace_bytes(1, 2, 512, 512, A.MASK_SLIDING, 1, 0) == expect(1, 2, 512, 512, 4)
+    assert A.attn_bwd_workspace_bytes(0, 2, 300, 300, A.MASK_FULL) == 0
+    assert A.attn_bwd_workspace_bytes(1, 2, 300, 300, A.MASK_SLIDING, 0, 0) == 0  # bad window
 
 
 def test_fp8_invalid_arguments_are_rejected(lib):
