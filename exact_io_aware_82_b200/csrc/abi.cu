@@ -649,7 +649,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
     return ATTN_OK;
   }
   const int nqt = (Nq + bwd::kT - 1) / bwd::kT, nkb = (Nk + bwd::kT - 1) / bwd::kT;
-  const long long units_q = static_cast<long long>(nqt) * B * Hq;
+  const long long units_q = static_cast<long long>((nqt + 1) / 2) * B * Hq;  // query-tile pairs
   const long long units_kv = static_cast<long long>(nkb) * B * Hkv;
   if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   const MaskSpec mask = make_mask(mask_kind, window, n_sink, Nk);

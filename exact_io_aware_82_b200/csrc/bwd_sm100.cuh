@@ -553,10 +553,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// 3. dQ = scale dS K: one CTA per (b, query head, query tile), over the dS^T blocks the dK/dV
-//    kernel wrote.  dS^T blocks and K tiles stream through a 3-stage ring; one thread issues
-//    the MMAs (A = dS read MN-major from the [keys][queries] block, B = K MN-major); dQ
-//    accumulates in 128 TMEM columns; warps 0-7 store it.
+// 3. dQ = scale dS K over the dS^T blocks the dK/dV kernel wrote.  One CTA per (b, query head,
+//    pair of query tiles): tile qt = nqt-1-i (heavy under a causal mask) and tile i (light), so
+//    CTAs carry similar work and each pays its set-up once for two tiles.  dS^T blocks and K
+//    tiles stream through a 3-stage ring (the first tile's blocks, then the second's); one thread
+//    issues the MMAs (A = dS read MN-major from the [keys][queries] block, B = K MN-major) into
+//    one 128-column TMEM accumulator per tile; warps 0-7 store the results.
 // ------------------------------------------------------------------------------------------
 constexpr int kDqStages = 3;
 
@@ -566,7 +568,7 @@ struct __align__(1024) SmemQ {
   uint64_t bar_full[kDqStages], bar_empty[kDqStages], bar_done, bar_drain;
   uint32_t tmem_base;
   int abort;
-  int any;  // set by the MMA thread: at least one dS block contributed
+  int any;  // set by the MMA thread: bit t = some dS block contributed to tile t
 };
 constexpr size_t kSmemQBytes = sizeof(SmemQ) + 1024;
 
@@ -578,23 +580,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                                         ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // heaviest query tiles (causal) first
   const int nbh = p.B * p.Hq;
-  const int qt = p.num_qtiles - 1 - static_cast<int>(blockIdx.x) / nbh;
+  const int pi = static_cast<int>(blockIdx.x) / nbh;
   const int bh = blockIdx.x % nbh;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bkv = b * p.Hkv + h / p.G;
-  const int r0 = qt * kT;
   const int off = p.Nk - p.Nq;
-  const int last_row = min(r0 + kT, p.Nq) - 1;
-  const TileRange tr = key_tiles(p.mask, r0 + off, last_row + off, kT);
-  const int nk = tr.count();
-  // step jj uses key tile tr.tile(jj) if this query tile is in that key block's range (a pair
-  // outside it has no visible entry and no dS block); every role walks the same list
-  auto pair_slot = [&](int jj, int& kt) -> long long {
-    kt = tr.tile(jj);
+  int qts[2] = {p.num_qtiles - 1 - pi, pi};
+  const int ntiles = qts[0] == qts[1] ? 1 : 2;
+  TileRange trs[2];
+  int nks[2] = {0, 0};
+  for (int t = 0; t < ntiles; ++t) {
+    const int r0 = qts[t] * kT, last_row = min(r0 + kT, p.Nq) - 1;
+    trs[t] = key_tiles(p.mask, r0 + off, last_row + off, kT);
+    nks[t] = trs[t].count();
+  }
+  const int nsteps = nks[0] + (ntiles > 1 ? nks[1] : 0);
+  // step jj: tile t = jj < nks[0] ? 0 : 1 and its key tile; a pair outside the key block's
+  // query-tile range has no visible entry and no dS block (slot -1); every role walks the same
+  // list
+  auto step_slot = [&](int jj, int& t, int& kt) -> long long {
+    t = jj < nks[0] ? 0 : 1;
+    kt = t ? trs[1].tile(jj - nks[0]) : trs[0].tile(jj);
     const int c0 = kt * kT, c1 = min(c0 + kT, p.Nk) - 1;
-    const int idx = pair_index(query_tiles(p.mask, c0, c1, off, p.Nq), qt);
+    const int idx = pair_index(query_tiles(p.mask, c0, c1, off, p.Nq), t ? qts[1] : qts[0]);
     if (idx < 0) return -1;
     return static_cast<long long>(bh) * p.ds_pairs + p.ds_off[kt] + idx;
   };
@@ -615,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tma_prefetch_desc(&tm_k);
   }
   if (warp == kMmaWarp) {
-    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 128);
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 256);
     dev::tmem_relinquish();
   }
   dev::tc_fence_before();
@@ -628,9 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ================================ TMA producer ================================
     if (lane == 0) {
       int u = 0;
-      for (int jj = 0; jj < nk; ++jj) {
-        int kt;
-        const long long slot = pair_slot(jj, kt);
+      for (int jj = 0; jj < nsteps; ++jj) {
+        int t, kt;
+        const long long slot = step_slot(jj, t, kt);
         if (slot < 0) continue;
         const int s = u % kDqStages;
         if (!wait_bounded(dev::smem_u32(&sm.bar_empty[s]), ((u / kDqStages) & 1) ^ 1, abort))
@@ -656,44 +665,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = dev::idesc_bf16_f32(kT, kD, 1, 1);  // A and B MN-major
       bool ok = true;
-      int u = 0;
-      for (int jj = 0; ok && jj < nk; ++jj) {
-        int kt;
-        if (pair_slot(jj, kt) < 0) continue;
+      int u = 0, used[2] = {0, 0};
+      for (int jj = 0; ok && jj < nsteps; ++jj) {
+        int t, kt;
+        if (step_slot(jj, t, kt) < 0) continue;
         const int s = u % kDqStages;
         if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_full[s]), (u / kDqStages) & 1, abort))) break;
         dev::tc_fence_after();
         const uint64_t da = dev::smem_desc(dev::smem_u32(sm.ds[s]), kHalfBytes, 1024, dev::kSwizzle128B);
         const uint64_t db = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        const int first = t ? used[1] == 0 : used[0] == 0;
 #pragma unroll
         for (int ks = 0; ks < kT / 16; ++ks)  // 16 keys (2 KB of each block) per MMA
-          dev::umma_ss(tmem, da + ((ks * 2048) >> 4), db + ((ks * 2048) >> 4), idesc,
-                       (u > 0 || ks > 0) ? 1u : 0u);
+          dev::umma_ss(tmem + t * 128, da + ((ks * 2048) >> 4), db + ((ks * 2048) >> 4), idesc,
+                       (!first || ks > 0) ? 1u : 0u);
         dev::umma_commit(dev::smem_u32(&sm.bar_empty[s]));
+        if (t) ++used[1]; else ++used[0];
         ++u;
       }
       if (ok && u > 0) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
       wait_drain(dev::smem_u32(&sm.bar_drain), 0);
-      sm.any = (ok && u > 0) ? 1 : 0;
+      sm.any = ok ? (used[0] > 0 ? 1 : 0) | (used[1] > 0 ? 2 : 0) : 0;
     }
   }
   // every MMA has completed (the MMA thread drained them) and sm.any is published
   __syncthreads();
   if (warp < 8) {
-    // ======================= store: scale * dQ, a column half per warp =======================
+    // =================== store: scale * dQ of each tile, a column half per warp ===================
     const int r = (warp & 3) * 32 + lane;
     const int ch = warp >> 2;
-    const int i = r0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const bool valid = i < p.Nq;
-    __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
-    if (!sm.any) {
-      if (valid && !*abort) store_zero_row(dst, ch);
-    } else {
-      if (wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort)) {
-        dev::tc_fence_after();
-        store_acc_row(tmem + lane_off, p.scale, dst, valid, ch);
+    const int flags = sm.any;
+    bool ready = false;
+    if (flags) {
+      ready = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
+      if (ready) dev::tc_fence_after();
+    }
+    for (int t = 0; t < ntiles; ++t) {
+      const int i = qts[t] * kT + r;
+      const bool valid = i < p.Nq;
+      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
+      if (!(flags & (1 << t))) {
+        if (valid && !*abort) store_zero_row(dst, ch);
+      } else if (ready) {
+        store_acc_row(tmem + lane_off + t * 128, p.scale, dst, valid, ch);
       }
     }
   }
@@ -703,7 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, 128);
+    dev::tmem_dealloc(tmem, 256);
   }
 }
 
