@@ -75,10 +75,18 @@ struct Params {
   long long ds_pairs;  // ds_off[num_kblocks]: blocks per (b, query head)
 };
 
-// Index of query tile qt in key block kb's query-tile range, or -1 if the range misses it.
-__host__ __device__ __forceinline__ int pair_index(const TileRange& r, int qt) {
-  if (qt < r.ns) return qt;
-  if (qt >= r.lo && qt <= r.hi) return r.ns + (qt - r.lo);
+// Query tiles of one key block: [s0, ns) (the global rows of the local + global mask, when
+// they are apart from the rest), then [lo, hi]; the two ranges never overlap.
+struct QueryTiles {
+  int s0, ns, lo, hi;
+  __host__ __device__ int count() const { return (ns - s0) + (hi < lo ? 0 : hi - lo + 1); }
+  __host__ __device__ int tile(int j) const { return j < ns - s0 ? s0 + j : lo + (j - (ns - s0)); }
+};
+
+// Index of query tile qt in key block kb's query tiles, or -1 if they miss it.
+__host__ __device__ __forceinline__ int pair_index(const QueryTiles& r, int qt) {
+  if (qt >= r.s0 && qt < r.ns) return qt - r.s0;
+  if (qt >= r.lo && qt <= r.hi) return (r.ns - r.s0) + (qt - r.lo);
   return -1;
 }
 
@@ -95,29 +103,33 @@ __host__ __device__ __forceinline__ int floor_div128(long long a) {
 }
 
 // Query tiles whose rows see at least one key of [c0, c1] (off = Nk - Nq; query row i sits at
-// key position i + off), as a TileRange: tiles [0, ns) (the global rows of the local + global
-// mask), then [lo, hi].
-__host__ __device__ __forceinline__ TileRange query_tiles(const MaskSpec& m, int c0, int c1,
-                                                          int off, int Nq) {
+// key position i + off).
+__host__ __device__ __forceinline__ QueryTiles query_tiles(const MaskSpec& m, int c0, int c1,
+                                                           int off, int Nq) {
   const int nqt = (Nq + kT - 1) / kT;
-  TileRange r{0, 0, nqt - 1};
+  QueryTiles r{0, 0, 0, nqt - 1};
   if (m.kind == ATTN_MASK_FULL) return r;
   if (m.kind == ATTN_MASK_LOCAL_GLOBAL) {
     if (c0 < m.n_sink) return r;  // a global key is seen by every row
-    // rows p in [c0 - w, c1 + w], and the global rows 0 <= p < n_global (i < n_global - off)
-    const long long g_rows = static_cast<long long>(m.n_sink) - off;
-    const int g_tiles = g_rows <= 0 ? 0 : imin(nqt, static_cast<int>((g_rows + kT - 1) / kT));
+    // the window rows: positions p in [c0 - w, c1 + w]
     r.lo = imax(0, floor_div128(static_cast<long long>(c0) - m.window - off));
     r.hi = imin(r.hi, floor_div128(static_cast<long long>(c1) + m.window - off));
+    // the global rows: positions 0 <= p < n_global, i.e. rows [max(0, -off), n_global - off)
+    // of [0, Nq); they end no later than the window rows do
+    const long long g0 = off < 0 ? -static_cast<long long>(off) : 0;
+    long long g1 = static_cast<long long>(m.n_sink) - off;
+    if (g1 > Nq) g1 = Nq;
+    if (g0 >= g1) return r;  // no global row
+    const int ga = static_cast<int>(g0 / kT), gb = static_cast<int>((g1 - 1) / kT);
     if (r.lo > r.hi) {  // no window row: the global rows only
-      r.ns = g_tiles;
-      r.lo = g_tiles;
-      r.hi = g_tiles - 1;
-    } else if (g_tiles >= r.lo) {
-      r.lo = 0;
-      r.hi = imax(r.hi, g_tiles - 1);
-    } else {
-      r.ns = g_tiles;
+      r.lo = ga;
+      r.hi = gb;
+    } else if (gb + 1 >= r.lo) {  // touching or overlapping: one range
+      r.lo = imin(r.lo, ga);
+      r.hi = imax(r.hi, gb);
+    } else {  // global tiles first, apart from the window tiles
+      r.s0 = ga;
+      r.ns = gb + 1;
     }
     return r;
   }
@@ -297,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int b = bk / p.Hkv, hk = bk % p.Hkv;
   const int c0 = kb * kT, c1 = min(c0 + kT, p.Nk) - 1;
   const int off = p.Nk - p.Nq;
-  const TileRange qr = query_tiles(p.mask, c0, c1, off, p.Nq);
+  const QueryTiles qr = query_tiles(p.mask, c0, c1, off, p.Nq);
   const int nqt = qr.count();
   const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qr.tile(n % nqt)
   const int nsub = 2 * nsteps;

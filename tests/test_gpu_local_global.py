@@ -75,7 +75,8 @@ def test_local_global_packed_sequences():
 
 
 @pytest.mark.parametrize("Nq,Nk,w,g,Hq,Hkv", [(700, 700, 64, 2, 4, 1), (300, 450, 50, 1, 2, 2),
-                                              (450, 300, 30, 0, 2, 2), (513, 513, 0, 130, 2, 1)])
+                                              (450, 300, 30, 0, 2, 2), (513, 513, 0, 130, 2, 1),
+                                              (1100, 900, 100, 4, 2, 1)])
 def test_local_global_backward(Nq, Nk, w, g, Hq, Hkv):
     d = 128
     (q, k, v), (q64, k64, v64) = bf16_inputs(94, 1, Hq, Hkv, Nq, Nk, d)
