@@ -104,17 +104,51 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
 
 
-def _check(t, name, dtype, ndim):
+def _check(t, name, dtype, ndim, shape=None):
+    """Type, dtype, rank, contiguity and (if given) exact shape of one tensor argument."""
     import torch
 
     if not isinstance(t, torch.Tensor):
         raise TypeError("%s must be a torch.Tensor" % name)
-    if t.device.type != "cuda":
-        raise ValueError("%s must be a CUDA tensor" % name)
     if t.dtype != dtype:
         raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
     if t.dim() != ndim or not t.is_contiguous():
         raise ValueError("%s must be a contiguous %d-d tensor" % (name, ndim))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _check_out(t, name, dtype, shape):
+    """An optional output / gradient tensor: None, or exactly the tensor the library writes."""
+    if t is not None:
+        _check(t, name, dtype, len(shape), shape)
+
+
+def _check_workspace(ws, nbytes):
+    import torch
+
+    if ws is None:
+        return
+    _check(ws, "workspace", torch.uint8, 1)
+    if ws.numel() < nbytes:
+        raise ValueError("workspace holds %d bytes, the call needs %d" % (ws.numel(), nbytes))
+
+
+def _device(stream, **tensors):
+    """The one CUDA device that every given tensor (and the stream, if any) lives on.
+
+    The library launches on the calling thread's current device with raw pointers, so a tensor
+    on another device must be refused here rather than handed to a kernel."""
+    devs = {t.device for t in tensors.values() if t is not None}
+    if len(devs) != 1:
+        raise ValueError("all tensors must be on one device, got %s" % ", ".join(
+            "%s on %s" % (n, t.device) for n, t in tensors.items() if t is not None))
+    dev = devs.pop()
+    if dev.type != "cuda":
+        raise ValueError("tensors must be CUDA tensors, got %s" % dev)
+    if stream is not None and stream.device != dev:
+        raise ValueError("stream is on %s, the tensors on %s" % (stream.device, dev))
+    return dev
 
 
 def _raise(rc, where):
@@ -130,17 +164,23 @@ def attn_fwd(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sink=0,
     """
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.bfloat16, 4)
+    _check(q, "q", torch.bfloat16, 4)
     B, Hq, Nq, d = q.shape
+    _check(k, "k", torch.bfloat16, 4)
     Hkv, Nk = k.shape[1], k.shape[2]
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
-                        int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
+    _check(k, "k", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check_out(o, "o", torch.bfloat16, (B, Hq, Nq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, Nq))
+    dev = _device(stream, q=q, k=k, v=v, o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                            int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
     _raise(rc, "attn_fwd")
     return o, lse
 
@@ -156,24 +196,31 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, o=None, l
     """
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.bfloat16, 3)
-    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (cu_seqlens_k, "cu_seqlens_k")):
-        _check(t, n, torch.int32, 1)
+    _check(q, "q", torch.bfloat16, 3)
     total_q, Hq, d = q.shape
+    _check(k, "k", torch.bfloat16, 3)
     total_k, Hkv = k.shape[0], k.shape[1]
+    _check(k, "k", torch.bfloat16, 3, (total_k, Hkv, d))
+    _check(v, "v", torch.bfloat16, 3, (total_k, Hkv, d))
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32, 1)
     num_seqs = cu_seqlens_q.numel() - 1
-    if cu_seqlens_k.numel() != num_seqs + 1:
-        raise ValueError("cu_seqlens_q and cu_seqlens_k must have the same length")
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((total_q, Hq), dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens_q),
-                               _ptr(cu_seqlens_k), num_seqs, Hq, Hkv, total_q, total_k,
-                               int(max_seqlen_q), d, int(mask_kind), int(window), int(n_sink),
-                               scale, _stream_ptr(stream))
+    if num_seqs < 0:
+        raise ValueError("cu_seqlens_q needs num_seqs + 1 >= 1 offsets")
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32, 1, (num_seqs + 1,))
+    _check_out(o, "o", torch.bfloat16, (total_q, Hq, d))
+    _check_out(lse, "lse", torch.float32, (total_q, Hq))
+    dev = _device(stream, q=q, k=k, v=v, cu_seqlens_q=cu_seqlens_q, cu_seqlens_k=cu_seqlens_k,
+                  o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((total_q, Hq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                   _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), num_seqs, Hq, Hkv,
+                                   total_q, total_k, int(max_seqlen_q), d, int(mask_kind),
+                                   int(window), int(n_sink), scale, _stream_ptr(stream))
     _raise(rc, "attn_fwd_varlen")
     return o, lse
 
@@ -196,17 +243,25 @@ def attn_fwd_fp8(q, k, v, descale_q, descale_k, descale_v, o=None, lse=None,
     q, k, v = codes(q, "q"), codes(k, "k"), codes(v, "v")
     B, Hq, Nq, d = q.shape
     Hkv, Nk = k.shape[1], k.shape[2]
-    _check(descale_q, "descale_q", torch.float32, 2)
-    _check(descale_k, "descale_k", torch.float32, 2)
-    _check(descale_v, "descale_v", torch.float32, 2)
-    if o is None:
-        o = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q.device)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(descale_q),
-                            _ptr(descale_k), _ptr(descale_v), B, Hq, Hkv, Nq, Nk, d,
-                            int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
+    _check(k, "k", torch.uint8, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.uint8, 4, (B, Hkv, Nk, d))
+    _check(descale_q, "descale_q", torch.float32, 2, (B, Hq))
+    _check(descale_k, "descale_k", torch.float32, 2, (B, Hkv))
+    _check(descale_v, "descale_v", torch.float32, 2, (B, Hkv))
+    _check_out(o, "o", torch.bfloat16, (B, Hq, Nq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, Nq))
+    dev = _device(stream, q=q, k=k, v=v, descale_q=descale_q, descale_k=descale_k,
+                  descale_v=descale_v, o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=dev)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_fwd_fp8(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(descale_q),
+                                _ptr(descale_k), _ptr(descale_v), B, Hq, Hkv, Nq, Nk, d,
+                                int(mask_kind), int(window), int(n_sink), scale,
+                                _stream_ptr(stream))
     _raise(rc, "attn_fwd_fp8")
     return o, lse
 
@@ -216,18 +271,24 @@ def attn_fwd_f32(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sin
     """Exact attention forward on fp32 tensors (same shapes and rules as attn_fwd)."""
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.float32, 4)
+    _check(q, "q", torch.float32, 4)
     B, Hq, Nq, d = q.shape
+    _check(k, "k", torch.float32, 4)
     Hkv, Nk = k.shape[1], k.shape[2]
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk,
-                            d, int(mask_kind), int(window), int(n_sink), scale,
-                            _stream_ptr(stream))
+    _check(k, "k", torch.float32, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.float32, 4, (B, Hkv, Nk, d))
+    _check_out(o, "o", torch.float32, (B, Hq, Nq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, Nq))
+    dev = _device(stream, q=q, k=k, v=v, o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_fwd_f32(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq,
+                                Nk, d, int(mask_kind), int(window), int(n_sink), scale,
+                                _stream_ptr(stream))
     _raise(rc, "attn_fwd_f32")
     return o, lse
 
@@ -245,24 +306,34 @@ def attn_bwd(q, k, v, o, lse, dout, mask_kind=MASK_FULL, window=0, n_sink=0, sca
     """
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
-        _check(t, n, torch.bfloat16, 4)
-    _check(lse, "lse", torch.float32, 3)
+    _check(q, "q", torch.bfloat16, 4)
     B, Hq, Nq, d = q.shape
+    _check(k, "k", torch.bfloat16, 4)
     Hkv, Nk = k.shape[1], k.shape[2]
-    if o.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, Hq, Nq):
-        raise ValueError("o and dout must have the shape of q, lse [B, Hq, Nq]")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    if workspace is None:
-        workspace = torch.empty(max(attn_bwd_workspace_bytes(B, Hq, Nq, Nk, mask_kind, window,
-                                                             n_sink), 16),
-                                dtype=torch.uint8, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
-                        _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, int(mask_kind), int(window),
-                        int(n_sink), scale, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(k, "k", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(o, "o", torch.bfloat16, 4, (B, Hq, Nq, d))
+    _check(dout, "dout", torch.bfloat16, 4, (B, Hq, Nq, d))
+    _check(lse, "lse", torch.float32, 3, (B, Hq, Nq))
+    _check_out(dq, "dq", torch.bfloat16, (B, Hq, Nq, d))
+    _check_out(dk, "dk", torch.bfloat16, (B, Hkv, Nk, d))
+    _check_out(dv, "dv", torch.bfloat16, (B, Hkv, Nk, d))
+    _check_workspace(workspace, 0)
+    dev = _device(stream, q=q, k=k, v=v, o=o, lse=lse, dout=dout, dq=dq, dk=dk, dv=dv,
+                  workspace=workspace)
+    with torch.cuda.device(dev):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        if workspace is None:
+            workspace = torch.empty(max(attn_bwd_workspace_bytes(B, Hq, Nq, Nk, mask_kind, window,
+                                                                 n_sink), 16),
+                                    dtype=torch.uint8, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), _ptr(dq),
+                            _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, int(mask_kind),
+                            int(window), int(n_sink), scale, _ptr(workspace), workspace.numel(),
+                            _stream_ptr(stream))
     _raise(rc, "attn_bwd")
     return dq, dk, dv
 
@@ -275,6 +346,16 @@ def attn_decode_num_splits(B, Hq, Hkv, Nk, d) -> int:
     return int(lib().attn_decode_num_splits(B, Hq, Hkv, Nk, d))
 
 
+def _decode_query(q):
+    import torch
+
+    _check(q, "q", torch.bfloat16, 4)
+    B, Hq, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    return B, Hq, d
+
+
 def attn_decode(q, k, v, o=None, lse=None, scale=None, num_splits=0, workspace=None,
                 return_lse=True, stream=None):
     """Split-K decode: q [B,Hq,1,d] bf16 against the cache k/v [B,Hkv,Nk,d] bf16.
@@ -284,23 +365,27 @@ def attn_decode(q, k, v, o=None, lse=None, scale=None, num_splits=0, workspace=N
     """
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.bfloat16, 4)
-    B, Hq, one, d = q.shape
-    if one != 1:
-        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    B, Hq, d = _decode_query(q)
+    _check(k, "k", torch.bfloat16, 4)
     Hkv, Nk = k.shape[1], k.shape[2]
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    if workspace is None:
-        nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits)
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk, d,
-                           scale, int(num_splits), _ptr(workspace), workspace.numel(),
-                           _stream_ptr(stream))
+    _check(k, "k", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check_out(o, "o", torch.bfloat16, (B, Hq, 1, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq))
+    _check_workspace(workspace, 0)
+    dev = _device(stream, q=q, k=k, v=v, o=o, lse=lse, workspace=workspace)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        if workspace is None:
+            nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, Nk, d, num_splits)
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk, d,
+                               scale, int(num_splits), _ptr(workspace), workspace.numel(),
+                               _stream_ptr(stream))
     _raise(rc, "attn_decode")
     return o, lse
 
@@ -315,33 +400,36 @@ def attn_decode_paged(q, k_cache, v_cache, block_table, seq_lens, max_seq_len, o
     """
     import torch
 
-    _check(q, "q", torch.bfloat16, 4)
+    B, Hq, d = _decode_query(q)
     _check(k_cache, "k_cache", torch.bfloat16, 4)
-    _check(v_cache, "v_cache", torch.bfloat16, 4)
-    _check(block_table, "block_table", torch.int32, 2)
-    _check(seq_lens, "seq_lens", torch.int32, 1)
-    B, Hq, one, d = q.shape
-    if one != 1:
-        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
     num_pages, page_size, Hkv, dk = k_cache.shape
-    if v_cache.shape != k_cache.shape or dk != d:
+    if dk != d:
         raise ValueError("k_cache and v_cache must both be [num_pages, page_size, Hkv, d]")
-    if block_table.shape[0] != B or seq_lens.shape[0] != B:
+    _check(v_cache, "v_cache", torch.bfloat16, 4, k_cache.shape)
+    _check(block_table, "block_table", torch.int32, 2)
+    if block_table.shape[0] != B:
         raise ValueError("block_table and seq_lens need one row per sequence")
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    _check(seq_lens, "seq_lens", torch.int32, 1, (B,))
+    _check_out(o, "o", torch.bfloat16, (B, Hq, 1, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq))
+    _check_workspace(workspace, 0)
+    dev = _device(stream, q=q, k_cache=k_cache, v_cache=v_cache, block_table=block_table,
+                  seq_lens=seq_lens, o=o, lse=lse, workspace=workspace)
     max_seq_len = int(max_seq_len)
-    if workspace is None:
-        nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, max_seq_len, d, num_splits)
-        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
-                                 _ptr(block_table), _ptr(seq_lens), B, Hq, Hkv, num_pages,
-                                 page_size, block_table.shape[1], max_seq_len, d, scale,
-                                 int(num_splits), _ptr(workspace), workspace.numel(),
-                                 _stream_ptr(stream))
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        if workspace is None:
+            nbytes = attn_decode_workspace_bytes(B, Hq, Hkv, max_seq_len, d, num_splits)
+            workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_decode_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(o), _ptr(lse),
+                                     _ptr(block_table), _ptr(seq_lens), B, Hq, Hkv, num_pages,
+                                     page_size, block_table.shape[1], max_seq_len, d, scale,
+                                     int(num_splits), _ptr(workspace), workspace.numel(),
+                                     _stream_ptr(stream))
     _raise(rc, "attn_decode_paged")
     return o, lse
 
@@ -354,19 +442,22 @@ def attn_decode_noalloc(q, k, v, o=None, lse=None, scale=None, num_splits=0, ret
     AttnError(ATTN_ERR_WORKSPACE) when the call would need more than that array."""
     import torch
 
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _check(t, n, torch.bfloat16, 4)
-    B, Hq, one, d = q.shape
-    if one != 1:
-        raise ValueError("decode takes one query token per sequence (q.shape[2] == 1)")
+    B, Hq, d = _decode_query(q)
+    _check(k, "k", torch.bfloat16, 4)
     Hkv, Nk = k.shape[1], k.shape[2]
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None and return_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
-    rc = lib().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nk,
-                                   d, scale, int(num_splits), _stream_ptr(stream))
+    _check(k, "k", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check_out(o, "o", torch.bfloat16, (B, Hq, 1, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq))
+    dev = _device(stream, q=q, k=k, v=v, o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv,
+                                       Nk, d, scale, int(num_splits), _stream_ptr(stream))
     _raise(rc, "attn_decode_noalloc")
     return o, lse
 
