@@ -85,10 +85,13 @@ static int check_args(int B, int Hq, int Hkv, int Nq, int Nk, int d, int mask_ki
 
 /*
  * One query row: scores over every key, mask, softmax, P V.
- * s and e are caller-provided scratch of Nk doubles each.
+ * s and vis are caller-provided scratch of Nk entries each.  kblocks, when not NULL, is the
+ * row's entry of a block-sparse layout (one byte per block of block_k keys): a key is visible
+ * only if its block is selected as well.
  */
 static void attend_row(const double *q, const double *K, const double *V, int Nk, int d,
                        int64_t p, int mask_kind, int window, int n_sink, double scale,
+                       const unsigned char *kblocks, int block_k,
                        double *s, unsigned char *vis, double *o, double *lse) {
     int64_t j;
     int t;
@@ -99,7 +102,8 @@ static void attend_row(const double *q, const double *K, const double *V, int Nk
         double acc = 0.0;
         for (t = 0; t < d; ++t) acc += q[t] * K[j * (int64_t)d + t];
         s[j] = scale * acc;
-        vis[j] = (unsigned char)oracle_visible(p, j, mask_kind, window, n_sink);
+        vis[j] = (unsigned char)(oracle_visible(p, j, mask_kind, window, n_sink) &&
+                                 (kblocks == NULL || kblocks[j / block_k] != 0));
         if (vis[j]) {
             if (!any || s[j] > m) m = s[j];
             any = 1;
@@ -151,7 +155,7 @@ int oracle_attn(const double *q, const double *k, const double *v, double *o, do
                 const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
                 double l_out;
                 attend_row(q + r * d, Kb, Vb, Nk, d, i + (int64_t)Nk - Nq, mask_kind, window,
-                           n_sink, scale, s, vis, o + r * d, &l_out);
+                           n_sink, scale, NULL, 1, s, vis, o + r * d, &l_out);
                 if (lse) lse[r] = l_out;
             }
         }
@@ -194,7 +198,62 @@ int oracle_attn_rows(const double *q, const double *k, const double *v, int B, i
                 const double *Kb = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
                 const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
                 attend_row(q + r * d, Kb, Vb, Nk, d, i + (int64_t)Nk - Nq, mask_kind, window,
-                           n_sink, scale, s, vis, o_rows + t * d, &lse_rows[t]);
+                           n_sink, scale, NULL, 1, s, vis, o_rows + t * d, &lse_rows[t]);
+            }
+        }
+        free(s);
+        free(vis);
+    }
+    return failed ? -2 : 0;
+}
+
+/*
+ * Block-sparse forward ("Quadratic Complexity Bottleneck", sparse attention patterns: the
+ * sequence is cut into blocks and attention is computed within and between selected blocks).
+ * The selection is fixed and given by the caller: block_mask[hm][i / block_q][j / block_k]
+ * != 0 selects the block of query rows and keys that holds row i and key j, with
+ * hm = h when mask_heads == Hq (one layout per query head) and hm = 0 when mask_heads == 1 (one
+ * layout for every head); layout [mask_heads][ceil(Nq / block_q)][ceil(Nk / block_k)] bytes,
+ * shared by the batch.  Blocks are cut on row indices i and key indices j.  A key is visible
+ * iff its block is selected and the base mask (mask_kind, window, n_sink) admits it; the rest
+ * is oracle_attn.  Returns 0, or -1 on invalid arguments.
+ */
+int oracle_attn_block_sparse(const double *q, const double *k, const double *v, double *o,
+                             double *lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             int mask_kind, int window, int n_sink, double scale,
+                             const unsigned char *block_mask, int mask_heads, int block_q,
+                             int block_k) {
+    if (check_args(B, Hq, Hkv, Nq, Nk, d, mask_kind, window, n_sink)) return -1;
+    if (block_q < 1 || block_k < 1 || (mask_heads != 1 && mask_heads != Hq)) return -1;
+    if (block_mask == NULL && Nq > 0 && Nk > 0) return -1;
+    const int G = Hq / Hkv;
+    const int64_t nqb = ((int64_t)Nq + block_q - 1) / block_q;
+    const int64_t nkb = ((int64_t)Nk + block_k - 1) / block_k;
+    const int64_t rows = (int64_t)B * Hq * Nq;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        unsigned char *vis = (unsigned char *)malloc((size_t)(Nk > 0 ? Nk : 1));
+        if (!s || !vis) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            int64_t r;
+#pragma omp for schedule(dynamic, 16)
+            for (r = 0; r < rows; ++r) {
+                int64_t i = r % Nq;
+                int64_t bh = r / Nq;
+                int64_t h = bh % Hq, b = bh / Hq;
+                int64_t hk = h / G;
+                int64_t hm = mask_heads == 1 ? 0 : h;
+                const double *Kb = k + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                const double *Vb = v + ((b * Hkv + hk) * (int64_t)Nk) * d;
+                const unsigned char *row_blocks = block_mask + (hm * nqb + i / block_q) * nkb;
+                double l_out;
+                attend_row(q + r * d, Kb, Vb, Nk, d, i + (int64_t)Nk - Nq, mask_kind, window,
+                           n_sink, scale, row_blocks, block_k, s, vis, o + r * d, &l_out);
+                if (lse) lse[r] = l_out;
             }
         }
         free(s);

@@ -49,6 +49,10 @@ def _load():
         lib.oracle_visible.restype = ctypes.c_int
         lib.oracle_attn_bwd.argtypes = [dp] * 7 + [ctypes.c_int] * 9 + [ctypes.c_double]
         lib.oracle_attn_bwd.restype = ctypes.c_int
+        lib.oracle_attn_block_sparse.argtypes = ([dp, dp, dp, dp, dp] + [ctypes.c_int] * 9 +
+                                                 [ctypes.c_double, ctypes.c_void_p] +
+                                                 [ctypes.c_int] * 3)
+        lib.oracle_attn_block_sparse.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -79,6 +83,33 @@ def attention(q, k, v, mask_kind=MASK_FULL, window=0, n_sink=0, scale=None):
                              int(mask_kind), int(window), int(n_sink), float(scale))
     if rc != 0:
         raise ValueError("oracle_attn rejected its arguments (rc=%d)" % rc)
+    return o, lse
+
+
+def attention_block_sparse(q, k, v, block_mask, mask_kind=MASK_FULL, window=0, n_sink=0,
+                           scale=None, block_q=128, block_k=128):
+    """Block-sparse O and LSE: key j is visible to row i of head h iff
+    block_mask[hm, i // block_q, j // block_k] is non-zero (hm = h, or 0 for a layout shared by
+    every head) and the base mask admits it.  block_mask: [1 or Hq, ceil(Nq/block_q),
+    ceil(Nk/block_k)], any integer or bool dtype.  Returns (o fp64, lse fp64) as attention().
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, d = q.shape
+    _, Hkv, Nk, _ = k.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    bm = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+    nqb, nkb = -(-Nq // block_q), -(-Nk // block_k)
+    if bm.ndim != 3 or bm.shape[0] not in (1, Hq) or bm.shape[1:] != (nqb, nkb):
+        raise ValueError("block_mask must be [1 or Hq, %d, %d], got %s" % (nqb, nkb, bm.shape))
+    o = np.zeros((B, Hq, Nq, d), dtype=np.float64)
+    lse = np.zeros((B, Hq, Nq), dtype=np.float64)
+    rc = _load().oracle_attn_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq,
+                                          Hkv, Nq, Nk, d, int(mask_kind), int(window),
+                                          int(n_sink), float(scale), bm.ctypes.data,
+                                          int(bm.shape[0]), int(block_q), int(block_k))
+    if rc != 0:
+        raise ValueError("oracle_attn_block_sparse rejected its arguments (rc=%d)" % rc)
     return o, lse
 
 

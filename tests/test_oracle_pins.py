@@ -150,12 +150,13 @@ def test_causal_first_rows_closed_form():
 # --------------------------------------------------------------------------------------------
 # P6  brute force on tiny inputs: 50-digit Decimal, no max subtraction, mask from set definition
 # --------------------------------------------------------------------------------------------
-def _decimal_attention(q, k, v, Nq, Nk, d, mask, w, s, scale):
+def _decimal_attention(q, k, v, Nq, Nk, d, mask, w, s, scale, keep=None):
+    """keep(i, j), if given, further restricts the visible set (block-sparse layouts)."""
     getcontext().prec = 50
     sc = Decimal(repr(scale))
     out, lses = [], []
     for i in range(Nq):
-        vis = sorted(visible_set(i + Nk - Nq, Nk, mask, w, s))
+        vis = sorted(j for j in visible_set(i + Nk - Nq, Nk, mask, w, s) if keep is None or keep(i, j))
         if not vis:
             out.append([0.0] * d)
             lses.append(-math.inf)
