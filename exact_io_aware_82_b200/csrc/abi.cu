@@ -755,7 +755,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ATTN_DECODE_NOA
 void* g_noalloc_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device, looked up once per device (in
-// host code the array's name is only a host-side stand-in, never a device address).
+// host code the array's name is only a host-side stand-in, never a device address).  The
+// address is kept for the process's life: the header rules out use across a device reset.
 int noalloc_scratch(void** out) {
   int dev = 0;
   int rc = cuda_status(cudaGetDevice(&dev));

@@ -238,6 +238,9 @@ ATTN_API int attn_decode_paged(const void *q, const void *k_cache, const void *v
  *    num_splits lowers the need;
  *  - the first call on each device looks up the array's device address (and may make CUDA load
  *    the library's device code on that device); make that first call before any stream capture;
+ *  - that address is kept for the life of the process: do not use the library across a device
+ *    reset (cudaDeviceReset, or a primary context torn down and made again), after which the
+ *    kept address would no longer name the array;
  *  - all calls on a device share the one array, which keeps the last call's contents; every call
  *    writes the part it reads, so nothing needs clearing, but two calls that overlap on the GPU
  *    (different streams, or different host threads, without ordering between them) race on it.

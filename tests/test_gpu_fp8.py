@@ -5,10 +5,12 @@ Tolerance (derived from the arithmetic; the inputs are exact, so the only roundi
 fp32 accumulation is that of the weights): the kernel rounds 128 * P to E4M3 (3 mantissa bits,
 relative error up to 2^-4) for the P V product and keeps the row sums in fp32.  A numpy model of
 exactly that rounding against the oracle, on causal n = 512 and 2048, full n = 1024 and sliding
-w = 128 + 4 sinks, gives a max error of 0.046 (rows that see few keys: a single rounded weight
+w = 128 + 4 sinks, local + global and Nq != Nk, output rounded to bf16, gives a max error of
+0.054 (rows that see few keys: a single rounded weight
 carries most of the row) and a mean error of at most 0.0027.  The test allows max|dO| <= 0.1,
 mean|dO| <= 6e-3; the log-sum-exp does not see the rounding (fp32 scores and sums) and keeps the
-bf16 bound of 1e-3 relative.
+bf16 bound of 1e-3 relative.  tests/test_tolerance_models.py holds that model (a CPU test) and
+checks the margin.
 """
 
 import math
@@ -22,11 +24,10 @@ from exact_io_aware_82_b200 import attn as A
 from exact_io_aware_82_b200 import build as Bld
 from oracle import oracle as O
 
-from ._parity import assert_close, oracle_rows_one_head, sample_rows, to64
+from ._parity import TOL_FP8, assert_close, oracle_rows_one_head, sample_rows, to64
 
 pytestmark = pytest.mark.gpu
 FULL, CAUSAL, SLIDING, LOCAL = A.MASK_FULL, A.MASK_CAUSAL, A.MASK_SLIDING, A.MASK_LOCAL_GLOBAL
-TOL_FP8 = dict(max_abs=0.1, mean_abs=6e-3, lse_rel=1e-3)
 
 
 @pytest.fixture(scope="module", autouse=True)

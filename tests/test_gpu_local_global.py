@@ -95,6 +95,6 @@ def test_local_global_backward(Nq, Nk, w, g, Hq, Hkv):
 
 def test_local_global_prefill_n32768_w2048_g4():
     w = 2048
-    _full_size_check(9, 1, 32, 8, 32768, LOCAL, w, 4, whole_heads=[], n_random=12,
+    _full_size_check(9, 1, 32, 8, 32768, LOCAL, w, 4, whole_heads=[(0, 31)], n_random=12,
                      structural=(0, 1, 3, 4, 5, w - 1, w, w + 1, w + 4, w + 5, 16384,
                                  32767 - w, 32767))

@@ -175,7 +175,7 @@ def test_gqa_causal_prefill_b2_h32_kv8_n8192():
 
 def test_sliding_window_prefill_n32768_w4096_sinks4():
     w = 4096
-    _full_size_check(4, 1, 32, 8, 32768, SLIDING, w, 4, whole_heads=[], n_random=12,
+    _full_size_check(4, 1, 32, 8, 32768, SLIDING, w, 4, whole_heads=[(0, 31)], n_random=12,
                      structural=(0, 1, 3, 4, 5, w - 1, w, w + 1, w + 2, w + 3, w + 4, 2 * w,
                                  32767))
 
