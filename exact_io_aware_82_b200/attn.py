@@ -78,7 +78,7 @@ def lib():
         L.attn_decode_paged.restype = i
         L.attn_fwd_fp8.argtypes = [vp] * 8 + [i] * 9 + [f, vp]
         L.attn_fwd_fp8.restype = i
-        L.attn_fwd_block_sparse.argtypes = [vp] * 6 + [i] * 11 + [f, vp]
+        L.attn_fwd_block_sparse.argtypes = [vp] * 6 + [i] * 10 + [f, vp]
         L.attn_fwd_block_sparse.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i] * 7
         L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t

@@ -28,6 +28,44 @@ def test_header_declarations_match_binding():
     assert declared_functions() == sorted(A.EXPORTS)
 
 
+def declared_parameters():
+    """Each declared function's parameters as the ctypes class that carries them: pointers
+    (and the stream handle) as c_void_p, then int, float, size_t, long long."""
+    text = re.sub(r"/\*.*?\*/", " ", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(([^)]*)\)", text):
+        params = " ".join(m.group(2).split())
+        kinds = []
+        for prm in ([] if params in ("", "void") else params.split(",")):
+            prm = prm.strip()
+            if "*" in prm or prm.startswith("attn_stream_t"):
+                kinds.append(ctypes.c_void_p)
+            elif prm.startswith("size_t"):
+                kinds.append(ctypes.c_size_t)
+            elif prm.startswith("long long"):
+                kinds.append(ctypes.c_longlong)
+            elif prm.startswith("float"):
+                kinds.append(ctypes.c_float)
+            elif prm.startswith("int"):
+                kinds.append(ctypes.c_int)
+            else:
+                raise AssertionError("unexpected parameter type: " + prm)
+        out[m.group(1)] = kinds
+    return out
+
+
+def test_binding_argtypes_match_header(lib):
+    # a binding that passes one argument too many or too few would shift every argument after
+    # it; each declared parameter must have an argtype of the same kind
+    params = declared_parameters()
+    assert sorted(params) == declared_functions()
+    for name, kinds in params.items():
+        got = list(getattr(lib, name).argtypes)
+        assert len(got) == len(kinds), "%s: %d argtypes, header declares %d" % (name, len(got), len(kinds))
+        for n, (a, b) in enumerate(zip(got, kinds)):
+            assert a is b, "%s parameter %d: binding %s, header %s" % (name, n, a, b)
+
+
 def test_library_exports_every_declared_symbol(lib):
     for name in declared_functions():
         assert hasattr(lib, name), name
