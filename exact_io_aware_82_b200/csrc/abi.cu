@@ -79,6 +79,14 @@ int configure_fwd(DeviceInfo* info) {
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
       if (rc != ATTN_OK) return rc;
     }
+    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+        fwd::fwd_bf16_sparse_sm100_kernel<false>, fwd::fwd_bf16_sparse_sm100_kernel<true>};
+    for (auto* kern : sparse_kernels) {
+      const int rc = cuda_status(cudaFuncSetAttribute(kern,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(fwd::kSmemBytesSparse)));
+      if (rc != ATTN_OK) return rc;
+    }
     info->fwd_configured = true;
   }
   if (g_encode == nullptr) {
@@ -373,7 +381,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
       encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -395,6 +403,58 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
     fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+  return cuda_status(cudaGetLastError());
+}
+
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const uint8_t* block_mask, int mask_heads, int B, int Hq, int Hkv,
+                          int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                          float scale, attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  if (mask_heads != 1 && mask_heads != Hq) return ATTN_ERR_INVALID_ARG;
+  if (B > 0 && Nq > 0 && Nk > 0 && block_mask == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (d != fwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  const int mask_qtiles = (Nq + fwd::kBM - 1) / fwd::kBM, mask_ktiles = (Nk + fwd::kBN - 1) / fwd::kBN;
+  if (mask_ktiles > fwd::kMaxSparseTiles) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Nk == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
+                             static_cast<size_t>(B) * Hq * Nq, d, st);
+  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  fwd::Params p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.c = scale * kLog2e;
+  if (p.c == 0.f) p.c = 1e-30f;
+  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.block_mask = block_mask;
+  p.mask_heads = mask_heads;
+  p.mask_qtiles = mask_qtiles;
+  p.mask_ktiles = mask_ktiles;
+  const dim3 grid(static_cast<unsigned>(units));
+  if (scale < 0.f)
+    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
+  else
+    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -427,7 +487,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
       encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = num_seqs;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -476,7 +536,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
       encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
