@@ -109,7 +109,7 @@ NCU_TRAFFIC = {
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
 # up grids and tensor maps)
 FAMILY_SOURCES = {
-    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh"),
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
     "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
 }

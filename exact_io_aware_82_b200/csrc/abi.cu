@@ -70,7 +70,7 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
         fwd::fwd_bf16_sm100_kernel<false, true>,  fwd::fwd_bf16_sm100_kernel<true, true>,
         fwd::fwd_fp8_sm100_kernel<false>,         fwd::fwd_fp8_sm100_kernel<true>};
@@ -79,7 +79,7 @@ int configure_fwd(DeviceInfo* info) {
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
       if (rc != ATTN_OK) return rc;
     }
-    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sparse_sm100_kernel<false>, fwd::fwd_bf16_sparse_sm100_kernel<true>};
     for (auto* kern : sparse_kernels) {
       const int rc = cuda_status(cudaFuncSetAttribute(kern,
@@ -188,14 +188,15 @@ int launch_fill_empty(T* o, float* lse, size_t rows, int d, cudaStream_t stream)
   return cuda_status(cudaGetLastError());
 }
 
-// 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x 128 rows,
-// 128-byte swizzle (the layout tcgen05.mma descriptors read).  Rows past `rows` read as zero.
-int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
+// 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x box_rows rows,
+// 128-byte swizzle (the layout tcgen05.mma descriptors read).  Rows past `rows` read as zero
+// and are not written.
+int encode_map(CUtensorMap* map, const void* base, int rows, int heads, uint32_t box_rows = 128) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
                                  static_cast<cuuint64_t>(rows) * fwd::kD * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -203,6 +204,9 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+// The output map of the prefill kernels: each warp stores its 32 rows of a tile as a box.
+constexpr uint32_t kOutBoxRows = 32;
 
 // 3-D tiled TMA map over [heads][rows][128] E4M3 codes (one byte each), read as boxes of the full
 // 128-byte row width x 128 rows x 1 head with the 128-byte swizzle.
@@ -222,7 +226,8 @@ int encode_map_e4m3(CUtensorMap* map, const void* base, int rows, int heads) {
 
 // 3-D tiled TMA map over a token-major packed [rows][heads][128] bf16 tensor, read as boxes of
 // 64 columns x 1 head x 128 rows (same shared-memory layout as encode_map).
-int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
+int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads,
+                      uint32_t box_rows = 128) {
   // dimensions (d, rows, heads): rows second, so that a box is a 64 x 128 block of one head as
   // in the dense map (a box that is one element wide in its second dimension copies measurably
   // slower); the row stride (heads * d) exceeds the head stride (d)
@@ -230,7 +235,7 @@ int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(heads) * fwd::kD * 2,
                                  static_cast<cuuint64_t>(fwd::kD) * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -377,9 +382,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -400,9 +406,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.cu_k = nullptr;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -429,9 +435,10 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -452,9 +459,9 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.mask_ktiles = mask_ktiles;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -483,9 +490,10 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                           num_seqs * Hq;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
-      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
+      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK ||
+      encode_map_packed(&to, o, total_q, Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = num_seqs;
@@ -504,9 +512,9 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.cu_k = cu_seqlens_k;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -532,9 +540,10 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -556,9 +565,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.descale_v = descale_v;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "dev/ptx_f8.cuh"
+#include "dev/ptx_store.cuh"
 
 namespace attn {
 namespace fwd {
@@ -130,7 +131,8 @@ __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); 
 // between selected blocks); dense bf16 tensors only.
 template <bool kNeg, bool kVarlen, bool kFp8, bool kSparse>
 __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                          const CUtensorMap& tm_v, const Params& p) {
+                                          const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                          const Params& p) {
   static_assert(!kSparse || (!kVarlen && !kFp8), "block-sparse layouts take dense bf16 tensors");
   constexpr int kHalves = kFp8 ? 1 : 2;                          // TMA boxes per tile
   constexpr uint32_t kTile = kFp8 ? kTileBytes / 2 : kTileBytes;  // bytes of one tile
@@ -235,6 +237,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     dev::tma_prefetch_desc(&tm_q);
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
+    dev::tma_prefetch_desc(&tm_o);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -576,6 +579,14 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + h
                                   : static_cast<size_t>(bh) * p.Nq + grow;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
+      // This warp's 32 rows leave as two 32-row x 64-column TMA boxes staged, 128-byte
+      // swizzled, in the tile's Q buffer, which no MMA reads any more (bar_o[t] covered every
+      // MMA of the tile).  A tile without steps never waited for its Q copy, and a box of
+      // packed sequences must not reach past its sequence: those rows use plain stores (a box
+      // wholly past the last row is not stored at all; a dense box is clipped at Nq).
+      const int wrow0 = r0 + t * kBM + (warp & 3) * 32;  // first row of this warp's box
+      const bool tma_out = cnt > 0 && wrow0 < nq && (!kVarlen || wrow0 + 31 < nq);
+      const uint32_t box0 = dev::smem_u32(sm.q[t]) + (warp & 3) * 4096;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
@@ -591,11 +602,31 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         for (int e = 0; e < 32; e += 2)
           pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
                                         __uint_as_float(o[e + 1]) * inv_l);
-        if (valid) {
+        if (tma_out) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const int c16 = cc * 4 + v4;  // 16-byte chunk of the 256-byte row
+            const uint32_t a = box0 + (c16 >> 3) * kHalfBytes + lane * 128 +
+                               (static_cast<uint32_t>((c16 & 7) ^ (lane & 7)) << 4);
+            dev::st_shared_v4(a, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        } else if (valid) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
+      }
+      if (tma_out) {
+        dev::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int half = 0; half < 2; ++half)
+            dev::tma_store_3d(&tm_o, box0 + half * kHalfBytes, half * 64,
+                              kVarlen ? q_base + wrow0 : wrow0, kVarlen ? h : bh);
+          dev::bulk_commit_group();
+          dev::bulk_wait_group_read0();  // the buffer is free again before the CTA ends
+        }
+        __syncwarp();
       }
       if (valid && p.lse != nullptr) {
         const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
@@ -619,8 +650,9 @@ template <bool kNeg, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, p);
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 // bf16 Q, K, V (dense) under a block-sparse layout
@@ -628,8 +660,9 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sparse_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                  const __grid_constant__ CUtensorMap tm_k,
-                                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, p);
+                                 const __grid_constant__ CUtensorMap tm_v,
+                                 const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 // E4M3 Q, K, V with per-(b, head) descale factors (dense)
@@ -637,8 +670,9 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, p);
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 }  // namespace fwd
