@@ -111,7 +111,7 @@ NCU_TRAFFIC = {
 FAMILY_SOURCES = {
     "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
-    "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
+    "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
 }
 
 

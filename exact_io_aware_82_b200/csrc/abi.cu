@@ -770,6 +770,21 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_UNSUPPORTED;
   }
+  // the same blocks as the dK/dV kernel writes them: boxes of 32 queries x 32 keys, one per row
+  // warp and sub-step, staged with the 64-byte swizzle
+  CUtensorMap tds_out;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(bwd::kT), static_cast<cuuint64_t>(bwd::kT),
+                                static_cast<cuuint64_t>(B) * Hq * (L.pairs > 0 ? L.pairs : 1)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(bwd::kT) * 2,
+                                   static_cast<cuuint64_t>(bwd::kT) * bwd::kT * 2};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    if (g_encode(&tds_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.ds, dims, strides, box, estride,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_UNSUPPORTED;
+  }
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
   bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
                                                bwd::kPrepRowsPerBlock),
@@ -778,7 +793,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       dsum, Nq, p.npad, prow, mask, nkb, p.ds_off);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(units_kv), bwd::kThreads, bwd::kSmemKVBytes, st>>>(
-      tq, tk, tv, tdo, p);
+      tq, tk, tv, tdo, tds_out, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
       tds, tk, p);
