@@ -83,6 +83,8 @@ WORKLOADS = {
                                                     n_sink=0, seed=7, page_size=16),
 }
 PROFILING_ONLY = ("decode_b8_h32_kv8_n32768_d128", "paged_decode_b8_h32_kv8_n32768_p16_d128")
+# fp32 FMA peak of the CUDA cores (TFLOP/s), for the fp32 workload, which uses no tensor core
+FP32_FMA_PEAK_TFLOPS = round(148 * 128 * 2 * 1965e6 / 1e12, 1)
 HEADLINE = "causal_b4_h16_n2048_d128"
 DECODE = "decode_b64_h32_kv8_n32768_d128"
 
@@ -508,13 +510,18 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
             # no FP8 GEMM was measured: the bf16 figure times the nominal ratio 4.5 / 2.25
             peak = round(2.0 * peaks["bf16_tflops"], 1)
         if w["kind"] == "fwd_f32":
-            bound, peak = "fp32-fma", None
+            # fp32 FMA on the CUDA cores: 148 SMs x 128 FMA lanes x 2 FLOP x 1965 MHz (the
+            # maximum SM clock), no tensor core
+            bound, peak = "alu", FP32_FMA_PEAK_TFLOPS
     tr = NCU_TRAFFIC.get(name)
     traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash(family_of(w)) else None
+    source = peak_kind + (" burst" if bound == "tensor" else "") + (
+        " bf16 x 2 (nominal FP8 / BF16 ratio)" if w["kind"] == "fwd_fp8" else "")
+    if bound == "alu":
+        source = "derived: 148 SMs x 128 fp32 FMA/clk x 2 FLOP x 1965 MHz"
     roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic,
-            "peak_source": peak_kind + (" burst" if bound == "tensor" else "")
-            + (" bf16 x 2 (nominal FP8 / BF16 ratio)" if w["kind"] == "fwd_fp8" else "")}
+            "peak_source": source}
 
     # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
     host_in = [t.cpu().pin_memory() for t in wl.inputs]
