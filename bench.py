@@ -70,6 +70,11 @@ WORKLOADS = {
     "paged_decode_b64_h32_kv8_n32768_p16_d128": dict(kind="decode_paged", B=64, Hq=32, Hkv=8,
                                                      N=32768, d=128, mask=FULL, window=0,
                                                      n_sink=0, seed=7, page_size=16),
+    # a fixed block-sparse layout (BigBird style: diagonal band, global first block row and
+    # column, 3 random blocks per row) over a full base mask
+    "block_sparse_b1_h32_kv8_n32768_d128": dict(kind="fwd_block_sparse", B=1, Hq=32, Hkv=8,
+                                                N=32768, d=128, mask=FULL, window=0, n_sink=0,
+                                                seed=11, n_random=3),
     # an eighth of the decode workloads (1 GiB of cache), for ncu captures that must stay small
     "decode_b8_h32_kv8_n32768_d128": dict(kind="decode", B=8, Hq=32, Hkv=8, N=32768, d=128,
                                           mask=FULL, window=0, n_sink=0, seed=5),
@@ -106,9 +111,9 @@ NCU_TRAFFIC = {
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
 # up grids and tensor maps)
 FAMILY_SOURCES = {
-    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh"),
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
-    "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh"),
+    "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
 }
 
 
@@ -165,6 +170,14 @@ def work_of(w):
         fl = sum(acc.attn_flops(1, w["Hq"], n, n, w["d"], w["mask"], w["window"], w["n_sink"])
                  for n in w["lens"])
         return fl, "TFLOP/s", 1e12
+    if w["kind"] == "fwd_block_sparse":
+        import synth
+
+        nt = -(-w["N"] // 128)
+        bm = synth.block_layout_bigbird(w["seed"], nt, nt, w["n_random"])
+        pairs = acc.block_sparse_pairs(bm, w["N"], w["N"], w["mask"], w["window"], w["n_sink"],
+                                       Hq=w["Hq"])
+        return 4 * w["d"] * w["B"] * pairs, "TFLOP/s", 1e12
     if w["kind"] == "bwd":
         return acc.attn_bwd_flops(w["B"], w["Hq"], w["N"], w["N"], w["d"], w["mask"], w["window"],
                                   w["n_sink"]), "TFLOP/s", 1e12
@@ -188,6 +201,9 @@ def config_of(name, w, n_gpus):
         c.update({"window": w["window"], "n_sink": w["n_sink"]})
     if w["mask"] == LOCAL_GLOBAL:
         c.update({"window_each_side": w["window"], "n_global": w["n_sink"]})
+    if w["kind"] == "fwd_block_sparse":
+        c.update({"layout": "128x128 blocks: diagonal band of 3, first block row and column, "
+                            "%d seeded random blocks per row; one layout for all heads" % w["n_random"]})
     c["inputs"] = {"fwd_f32": "fp32", "fwd_fp8": "e4m3 codes, fp32 scale per (b, head)"}.get(
         w["kind"], "bf16")
     c["l2"] = "flushed before every timed step (256 MiB write)"
@@ -319,6 +335,14 @@ class Workload:
             self.inputs = xs + scs
             self.lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
             self.o = torch.empty((B, Hq, N, d), dtype=torch.bfloat16, device="cuda")
+        elif w["kind"] == "fwd_block_sparse":
+            q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, N, d), dt, "cuda")
+            k = synth.normal_torch(seed, synth.K_ID, (B, Hkv, N, d), dt, "cuda")
+            v = synth.normal_torch(seed, synth.V_ID, (B, Hkv, N, d), dt, "cuda")
+            nt = -(-N // 128)
+            bm = torch.from_numpy(synth.block_layout_bigbird(w["seed"], nt, nt, w["n_random"])).cuda()
+            self.inputs = [q, k, v, bm]
+            self.lse = torch.empty((B, Hq, N), dtype=torch.float32, device="cuda")
         elif w["kind"] == "bwd":
             # the forward's outputs for these inputs are inputs of the backward step
             q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, N, d), dt, "cuda")
@@ -369,6 +393,9 @@ class Workload:
         elif w["kind"] == "fwd_varlen":
             A.attn_fwd_varlen(x[0], x[1], x[2], x[3], x[3], self.max_len, o=o, lse=lse,
                               mask_kind=w["mask"], window=w["window"], n_sink=w["n_sink"])
+        elif w["kind"] == "fwd_block_sparse":
+            A.attn_fwd_block_sparse(x[0], x[1], x[2], x[3], o=o, lse=lse, mask_kind=w["mask"],
+                                    window=w["window"], n_sink=w["n_sink"])
         elif w["kind"] == "fwd_f32":
             A.attn_fwd_f32(x[0], x[1], x[2], o=o, lse=lse, mask_kind=w["mask"],
                            window=w["window"], n_sink=w["n_sink"])

@@ -9,5 +9,5 @@ from . import accounting  # noqa: F401
 from .attn import (MASK_CAUSAL, MASK_FULL, MASK_LOCAL_GLOBAL, MASK_SLIDING,  # noqa: F401
                    AttnError, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
                    attn_decode_noalloc, attn_decode_num_splits, attn_decode_paged,
-                   attn_decode_workspace_bytes, attn_fwd, attn_fwd_f32, attn_fwd_fp8,
-                   attn_fwd_varlen, attn_get_device_error)
+                   attn_decode_workspace_bytes, attn_fwd, attn_fwd_block_sparse, attn_fwd_f32,
+                   attn_fwd_fp8, attn_fwd_varlen, attn_get_device_error)

@@ -116,3 +116,53 @@ def _local_global_pairs(Nq: int, Nk: int, w: int, g: int) -> int:
     rows = win + (G - inter)
     rows = np.where((p >= 0) & (p < g), Nk, rows)
     return int(rows.sum())
+
+
+def _visible_in(p, c0: int, c1: int, mask_kind: int, w: int, s: int, Nk: int):
+    """Visible keys in [c0, c1] (inclusive, c1 < Nk) for each query position in the array p."""
+    import numpy as np
+
+    def span(lo, hi):  # size of [max(lo, c0), min(hi, c1)] for array bounds lo, hi
+        return np.maximum(0, np.minimum(hi, c1) - np.maximum(lo, c0) + 1)
+
+    p = np.asarray(p, dtype=np.int64)
+    if mask_kind == MASK_FULL:
+        return np.full(p.shape, c1 - c0 + 1, dtype=np.int64)
+    if mask_kind == MASK_CAUSAL:
+        return span(np.zeros_like(p), p)
+    if mask_kind == MASK_SLIDING:
+        win = span(p - w + 1, p)  # window keys, causal by construction
+        sinks = span(np.zeros_like(p), np.minimum(p, s - 1))  # sinks, causal
+        both = span(np.maximum(p - w + 1, 0), np.minimum(p, s - 1))  # sinks inside the window
+        return win + sinks - both
+    if mask_kind == MASK_LOCAL_GLOBAL:
+        g = min(s, Nk)
+        glob_row = (p >= 0) & (p < s)
+        win = span(p - w, p + w)
+        gk = span(np.zeros_like(p), np.full(p.shape, g - 1))
+        both = span(np.maximum(p - w, 0), np.minimum(p + w, g - 1))
+        return np.where(glob_row, c1 - c0 + 1, win + gk - both)
+    raise ValueError("mask_kind")
+
+
+def block_sparse_pairs(block_mask, Nq: int, Nk: int, mask_kind: int, window: int = 0,
+                       n_sink: int = 0, Hq: int = 1, block: int = 128) -> int:
+    """Visible pairs of one batch row under a block-sparse layout, summed over the Hq query
+    heads: a pair counts when its block is selected (block_mask [1 or Hq][qtiles][ktiles]; a
+    single layout serves every head) and the base mask admits it."""
+    import numpy as np
+
+    bm = np.asarray(block_mask) != 0
+    off = Nk - Nq
+    total = 0
+    for hm in range(bm.shape[0]):
+        heads = Hq if bm.shape[0] == 1 else 1
+        for qt, kt in zip(*np.nonzero(bm[hm])):
+            r0, r1 = qt * block, min(Nq, (qt + 1) * block)
+            c0, c1 = kt * block, min(Nk, (kt + 1) * block) - 1
+            if r0 >= r1 or c0 > c1:
+                continue
+            p = np.arange(r0, r1, dtype=np.int64) + off
+            total += heads * int(_visible_in(p, c0, c1, mask_kind, window, n_sink, Nk).sum())
+    return total
+

@@ -28,7 +28,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libattn.so"
 EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "attn_fwd", "attn_fwd_f32",
            "attn_decode_workspace_bytes", "attn_decode", "attn_decode_num_splits",
            "attn_get_device_error", "attn_debug_timeout_probe", "attn_decode_noalloc",
-           "attn_fwd_varlen", "attn_decode_paged", "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_fp8")
+           "attn_fwd_varlen", "attn_decode_paged", "attn_bwd", "attn_bwd_workspace_bytes", "attn_fwd_fp8",
+           "attn_fwd_block_sparse")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
 DECODE_NOALLOC_MAX_BYTES = 32 << 20
@@ -77,6 +78,8 @@ def lib():
         L.attn_decode_paged.restype = i
         L.attn_fwd_fp8.argtypes = [vp] * 8 + [i] * 9 + [f, vp]
         L.attn_fwd_fp8.restype = i
+        L.attn_fwd_block_sparse.argtypes = [vp] * 6 + [i] * 10 + [f, vp]
+        L.attn_fwd_block_sparse.restype = i
         L.attn_bwd_workspace_bytes.argtypes = [i] * 7
         L.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
         L.attn_bwd.argtypes = [vp] * 9 + [i] * 9 + [f, vp, ctypes.c_size_t, vp]
@@ -182,6 +185,43 @@ def attn_fwd(q, k, v, o=None, lse=None, mask_kind=MASK_FULL, window=0, n_sink=0,
         rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
                             int(mask_kind), int(window), int(n_sink), scale, _stream_ptr(stream))
     _raise(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_block_sparse(q, k, v, block_mask, o=None, lse=None, mask_kind=MASK_FULL, window=0,
+                          n_sink=0, scale=None, return_lse=True, stream=None):
+    """attn_fwd under a fixed block-sparse layout: block_mask uint8 (or bool) [1 or Hq,
+    ceil(Nq/128), ceil(Nk/128)] selects the 128 x 128 blocks each head attends (one layout for
+    every head when its first dimension is 1).  Returns (o, lse) as attn_fwd."""
+    import torch
+
+    _check(q, "q", torch.bfloat16, 4)
+    B, Hq, Nq, d = q.shape
+    _check(k, "k", torch.bfloat16, 4)
+    Hkv, Nk = k.shape[1], k.shape[2]
+    _check(k, "k", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    _check(v, "v", torch.bfloat16, 4, (B, Hkv, Nk, d))
+    if isinstance(block_mask, torch.Tensor) and block_mask.dtype == torch.bool:
+        block_mask = block_mask.view(torch.uint8)
+    _check(block_mask, "block_mask", torch.uint8, 3)
+    shape = (block_mask.shape[0], -(-Nq // 128), -(-Nk // 128))
+    if block_mask.shape[0] not in (1, Hq):
+        raise ValueError("block_mask must have 1 or Hq = %d layouts, got %d" % (Hq, block_mask.shape[0]))
+    _check(block_mask, "block_mask", torch.uint8, 3, shape)
+    _check_out(o, "o", torch.bfloat16, (B, Hq, Nq, d))
+    _check_out(lse, "lse", torch.float32, (B, Hq, Nq))
+    dev = _device(stream, q=q, k=k, v=v, block_mask=block_mask, o=o, lse=lse)
+    with torch.cuda.device(dev):
+        if o is None:
+            o = torch.empty_like(q)
+        if lse is None and return_lse:
+            lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+        rc = lib().attn_fwd_block_sparse(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse),
+                                         _ptr(block_mask), int(block_mask.shape[0]), B, Hq, Hkv,
+                                         Nq, Nk, d, int(mask_kind), int(window), int(n_sink),
+                                         scale, _stream_ptr(stream))
+    _raise(rc, "attn_fwd_block_sparse")
     return o, lse
 
 

@@ -70,13 +70,21 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
         fwd::fwd_bf16_sm100_kernel<false, true>,  fwd::fwd_bf16_sm100_kernel<true, true>,
         fwd::fwd_fp8_sm100_kernel<false>,         fwd::fwd_fp8_sm100_kernel<true>};
     for (auto* kern : kernels) {
       const int rc = cuda_status(cudaFuncSetAttribute(
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
+      if (rc != ATTN_OK) return rc;
+    }
+    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+        fwd::fwd_bf16_sparse_sm100_kernel<false>, fwd::fwd_bf16_sparse_sm100_kernel<true>};
+    for (auto* kern : sparse_kernels) {
+      const int rc = cuda_status(cudaFuncSetAttribute(kern,
+                                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(fwd::kSmemBytesSparse)));
       if (rc != ATTN_OK) return rc;
     }
     info->fwd_configured = true;
@@ -180,14 +188,15 @@ int launch_fill_empty(T* o, float* lse, size_t rows, int d, cudaStream_t stream)
   return cuda_status(cudaGetLastError());
 }
 
-// 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x 128 rows,
-// 128-byte swizzle (the layout tcgen05.mma descriptors read).  Rows past `rows` read as zero.
-int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
+// 3-D tiled TMA map over a [heads][rows][128] bf16 tensor: box of 64 columns x box_rows rows,
+// 128-byte swizzle (the layout tcgen05.mma descriptors read).  Rows past `rows` read as zero
+// and are not written.
+int encode_map(CUtensorMap* map, const void* base, int rows, int heads, uint32_t box_rows = 128) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(fwd::kD) * 2,
                                  static_cast<cuuint64_t>(rows) * fwd::kD * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -195,6 +204,9 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads) {
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
+
+// The output map of the prefill kernels: each warp stores its 32 rows of a tile as a box.
+constexpr uint32_t kOutBoxRows = 32;
 
 // 3-D tiled TMA map over [heads][rows][128] E4M3 codes (one byte each), read as boxes of the full
 // 128-byte row width x 128 rows x 1 head with the 128-byte swizzle.
@@ -214,7 +226,8 @@ int encode_map_e4m3(CUtensorMap* map, const void* base, int rows, int heads) {
 
 // 3-D tiled TMA map over a token-major packed [rows][heads][128] bf16 tensor, read as boxes of
 // 64 columns x 1 head x 128 rows (same shared-memory layout as encode_map).
-int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
+int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads,
+                      uint32_t box_rows = 128) {
   // dimensions (d, rows, heads): rows second, so that a box is a 64 x 128 block of one head as
   // in the dense map (a box that is one element wide in its second dimension copies measurably
   // slower); the row stride (heads * d) exceeds the head stride (d)
@@ -222,7 +235,7 @@ int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads) {
                               static_cast<cuuint64_t>(heads)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(heads) * fwd::kD * 2,
                                  static_cast<cuuint64_t>(fwd::kD) * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, box_rows, 1};
   const cuuint32_t estride[3] = {1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -369,11 +382,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -392,9 +406,62 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.cu_k = nullptr;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+  return cuda_status(cudaGetLastError());
+}
+
+int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                          const uint8_t* block_mask, int mask_heads, int B, int Hq, int Hkv,
+                          int Nq, int Nk, int d, int mask_kind, int window, int n_sink,
+                          float scale, attn_stream_t stream) {
+  int rc = check_fwd_args(q, k, v, o, B, Hq, Hkv, Nq, Nk, mask_kind, window, n_sink, scale);
+  if (rc != ATTN_OK) return rc;
+  if (mask_heads != 1 && mask_heads != Hq) return ATTN_ERR_INVALID_ARG;
+  if (B > 0 && Nq > 0 && Nk > 0 && block_mask == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (d != fwd::kD) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_UNSUPPORTED;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return ATTN_ERR_UNSUPPORTED;
+  const int mask_qtiles = (Nq + fwd::kBM - 1) / fwd::kBM, mask_ktiles = (Nk + fwd::kBN - 1) / fwd::kBN;
+  if (mask_ktiles > fwd::kMaxSparseTiles) return ATTN_ERR_UNSUPPORTED;
+  DeviceInfo* info = nullptr;
+  if ((rc = current_device(&info)) != ATTN_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (B == 0 || Nq == 0) return ATTN_OK;
+  if (Nk == 0)
+    return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
+                             static_cast<size_t>(B) * Hq * Nq, d, st);
+  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
+  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
+  CUtensorMap tq, tk, tv, to;
+  if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
+  fwd::Params p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.mask = make_mask(mask_kind, window, n_sink, Nk);
+  p.c = scale * kLog2e;
+  if (p.c == 0.f) p.c = 1e-30f;
+  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.block_mask = block_mask;
+  p.mask_heads = mask_heads;
+  p.mask_qtiles = mask_qtiles;
+  p.mask_ktiles = mask_ktiles;
+  const dim3 grid(static_cast<unsigned>(units));
+  if (scale < 0.f)
+    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
+  else
+    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -423,11 +490,12 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                           num_seqs * Hq;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
-      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
+      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK ||
+      encode_map_packed(&to, o, total_q, Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = num_seqs;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -444,9 +512,9 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.cu_k = cu_seqlens_k;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -472,11 +540,12 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
   if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK ||
+      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
-  fwd::Params p;
+  fwd::Params p{};
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
@@ -496,9 +565,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.descale_v = descale_v;
   const dim3 grid(static_cast<unsigned>(units));
   if (scale < 0.f)
-    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -701,6 +770,21 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_UNSUPPORTED;
   }
+  // the same blocks as the dK/dV kernel writes them: boxes of 32 queries x 32 keys, one per row
+  // warp and sub-step, staged with the 64-byte swizzle
+  CUtensorMap tds_out;
+  {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(bwd::kT), static_cast<cuuint64_t>(bwd::kT),
+                                static_cast<cuuint64_t>(B) * Hq * (L.pairs > 0 ? L.pairs : 1)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(bwd::kT) * 2,
+                                   static_cast<cuuint64_t>(bwd::kT) * bwd::kT * 2};
+    const cuuint32_t box[3] = {32, 32, 1};
+    const cuuint32_t estride[3] = {1, 1, 1};
+    if (g_encode(&tds_out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, p.ds, dims, strides, box, estride,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_UNSUPPORTED;
+  }
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
   bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
                                                bwd::kPrepRowsPerBlock),
@@ -709,7 +793,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       dsum, Nq, p.npad, prow, mask, nkb, p.ds_off);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(units_kv), bwd::kThreads, bwd::kSmemKVBytes, st>>>(
-      tq, tk, tv, tdo, p);
+      tq, tk, tv, tdo, tds_out, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
       tds, tk, p);

@@ -39,6 +39,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "dev/ptx_store.cuh"
 
 namespace attn {
 namespace bwd {
@@ -277,11 +278,16 @@ constexpr uint32_t kSubBytes = kSub * 128;       // rows of a sub-step inside on
 // ------------------------------------------------------------------------------------------
 // 2. dK, dV: one CTA per (b, kv head, key block)
 // ------------------------------------------------------------------------------------------
+// dS^T of one sub-step leaves through shared memory: each row warp stages its 32 keys x 32
+// queries (64-byte rows, 64-byte swizzle) and stores them with one TMA box.
+constexpr uint32_t kDsBoxBytes = 32 * 32 * 2;
+
 struct __align__(1024) SmemKV {
   uint8_t k[kTileBytes];
   uint8_t v[kTileBytes];
   uint8_t q[2][kTileBytes];
   uint8_t dout[2][kTileBytes];
+  uint8_t ds_stage[kRowThreads / 32][kDsBoxBytes];  // one box per row warp
   float lse2[2][kT];  // per stage: the query tile's LSE * log2(e) and D, copied with Q and dO
   float dsum[2][kT];
   uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_free[2], bar_done;
@@ -290,12 +296,14 @@ struct __align__(1024) SmemKV {
   int abort;
 };
 constexpr size_t kSmemKVBytes = sizeof(SmemKV) + 1024;
+static_assert(kSmemKVBytes <= 227 * 1024, "shared memory of the dK/dV kernel");
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
-                    const __grid_constant__ CUtensorMap tm_do, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_ds, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                           ~uintptr_t(1023));
@@ -333,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
     dev::tma_prefetch_desc(&tm_do);
+    dev::tma_prefetch_desc(&tm_ds);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -522,18 +531,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::tmem_st16(t_dpt, dk16);
       {
         // the same bf16 dS^T values into this (key block, query tile) block for the dQ kernel:
-        // row r (key), columns 64h + 32ch .. +31 (queries)
+        // rows 32 (warp & 3) .. +31 (keys), columns 64h + 32ch .. +31 (queries), staged in this
+        // warp's box (64-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
+        // once the box's previous store has read it, then one TMA store
         const int hq = hk * p.G + n / nqt;
         const long long slot = static_cast<long long>(b * p.Hq + hq) * p.ds_pairs + ds_base + n % nqt;
-        uint4* dst = reinterpret_cast<uint4*>(p.ds + slot * (kT * kT) + r * kT + h * kSub + ch * 32);
+        const uint32_t box = dev::smem_u32(sm.ds_stage[warp]);
+        if (m > 0) {
+          if (lane == 0) dev::bulk_wait_group_read0();
+          __syncwarp();
+        }
 #pragma unroll
         for (int v4 = 0; v4 < 4; ++v4)
-          dst[v4] = make_uint4(dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
+          dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
+                            dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
+        dev::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          dev::tma_store_3d(&tm_ds, box, h * kSub + ch * 32, (warp & 3) * 32, static_cast<int>(slot));
+          dev::bulk_commit_group();
+        }
       }
       dev::tmem_wait_st();
       dev::tc_fence_before();
       dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
     }
+
+    // every staged box has been read by its store before the CTA can end
+    if (lane == 0) dev::bulk_wait_group_read0();
+    __syncwarp();
 
     // ---- epilogue: dV and scale * dK rows of this CTA's keys, bf16, a column half per warp ----
     const bool valid = j < p.Nk;

@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "dev/ptx_f8.cuh"
+#include "dev/ptx_store.cuh"
 
 namespace attn {
 namespace fwd {
@@ -77,6 +78,11 @@ struct Params {
   const float* descale_q;  // [B][Hq]
   const float* descale_k;  // [B][Hkv]
   const float* descale_v;  // [B][Hkv]
+  // block-sparse layout (dense tensors only): block_mask[hm][query tile][key tile] != 0
+  // selects that 128 x 128 block, hm = h when mask_heads == Hq and 0 when mask_heads == 1
+  const uint8_t* block_mask;
+  int mask_heads;
+  int mask_qtiles, mask_ktiles;  // ceil(Nq / 128), ceil(Nk / 128)
 };
 
 struct __align__(1024) Smem {
@@ -91,6 +97,18 @@ struct __align__(1024) Smem {
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base to 1024 B
+
+// Block-sparse CTAs list the key tiles they visit (selected for one of their two query tiles
+// and admitted by the base mask) right after Smem: tile index and, per entry, which query tiles
+// (bit t) take part.
+constexpr int kMaxSparseTiles = 4096;  // key tiles per row of the layout (Nk <= 524288)
+struct SparseList {
+  uint16_t tile[kMaxSparseTiles];
+  uint8_t bits[kMaxSparseTiles];
+  int count;
+};
+constexpr size_t kSmemBytesSparse = sizeof(Smem) + sizeof(SparseList) + 1024;
+static_assert(kSmemBytesSparse <= 227 * 1024, "shared memory of a block-sparse CTA");
 
 // Is every (row, key) of the 128x128 block of query tile rows [P0, P0+127] x keys of tile kt
 // visible?  Conservative (uses all 128 rows even past Nq).
@@ -108,9 +126,14 @@ __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); 
 // sequence is masked on its own (p_i = i + Nk_s - Nq_s).  Otherwise the dense [B][H][N][d] form.
 // kFp8: Q, K, V hold E4M3 codes (a 128 x 128 tile is 16 KB, one 128-byte-wide TMA box) and both
 // products run as kind::f8f6f4 MMAs, P being rounded to E4M3 (times kPScaleF8) in TMEM.
-template <bool kNeg, bool kVarlen, bool kFp8>
+// kSparse: a block-sparse layout (Params::block_mask) further restricts the key tiles of each
+// query tile ("Quadratic Complexity Bottleneck", sparse attention patterns: attention within and
+// between selected blocks); dense bf16 tensors only.
+template <bool kNeg, bool kVarlen, bool kFp8, bool kSparse>
 __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                          const CUtensorMap& tm_v, const Params& p) {
+                                          const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                          const Params& p) {
+  static_assert(!kSparse || (!kVarlen && !kFp8), "block-sparse layouts take dense bf16 tensors");
   constexpr int kHalves = kFp8 ? 1 : 2;                          // TMA boxes per tile
   constexpr uint32_t kTile = kFp8 ? kTileBytes / 2 : kTileBytes;  // bytes of one tile
   constexpr float kThreshold = kFp8 ? kRescaleThresholdF8 : kRescaleThreshold;
@@ -145,7 +168,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   const int last_row = min(r0 + kRowsPerCta, nq) - 1;
   // key tiles of the whole CTA (what the producer loads, in this order) ...
   const TileRange tr = key_tiles(mask, r0 + off, last_row + off, kBN);
-  const int nk = tr.count();
+  const int nk_range = tr.count();
   // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
   TileRange trt[2];
   for (int t = 0; t < 2; ++t) {
@@ -157,6 +180,41 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   auto in_range = [&](const TileRange& r, int j) {
     const int u = tr.tile(j);
     return u < r.ns || (u >= r.lo && u <= r.hi);
+  };
+  SparseList& sp = *reinterpret_cast<SparseList*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(Smem));
+  if (kSparse && warp == 0) {
+    // the steps of a block-sparse CTA: the range's key tiles selected for query tile 0 or 1,
+    // compacted in range order by one warp (ballot + prefix count)
+    const int hm = p.mask_heads == 1 ? 0 : h;
+    const uint8_t* row0 =
+        p.block_mask + (static_cast<size_t>(hm) * p.mask_qtiles + 2 * qb) * p.mask_ktiles;
+    const uint8_t* row1 = row0 + p.mask_ktiles;  // read only if query tile 1 has rows
+    int base = 0;
+    for (int j0 = 0; j0 < nk_range; j0 += 32) {
+      const int j = j0 + lane;
+      uint32_t bits = 0u;
+      int kt = 0;
+      if (j < nk_range) {
+        kt = tr.tile(j);
+        const bool t0 = in_range(trt[0], j) && __ldg(row0 + kt) != 0;
+        const bool t1 = in_range(trt[1], j) && __ldg(row1 + kt) != 0;
+        bits = (t0 ? 1u : 0u) | (t1 ? 2u : 0u);
+      }
+      const uint32_t sel = __ballot_sync(0xffffffffu, bits != 0u);
+      if (bits != 0u) {
+        const int pos = base + __popc(sel & ((1u << lane) - 1u));
+        sp.tile[pos] = static_cast<uint16_t>(kt);
+        sp.bits[pos] = static_cast<uint8_t>(bits);
+      }
+      base += __popc(sel);
+    }
+    if (lane == 0) sp.count = base;
+  }
+  // key tile of step j, and whether query tile t takes part in it
+  auto step_tile = [&](int j) { return kSparse ? static_cast<int>(sp.tile[j]) : tr.tile(j); };
+  auto takes_part = [&](int t, int j) {
+    if (kSparse) return ((sp.bits[j] >> t) & 1u) != 0u;
+    return in_range(t ? trt[1] : trt[0], j);
   };
 
   // ---- set-up ----
@@ -179,6 +237,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     dev::tma_prefetch_desc(&tm_q);
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
+    dev::tma_prefetch_desc(&tm_o);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -189,6 +248,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   dev::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  const int nk = kSparse ? sp.count : nk_range;  // steps of the CTA
   if (warp >= 8) {
     // ========== third warpgroup: TMA producer, MMA issuer, two idle warps ==========
     dev::regs_decrease<kRegsOther>();
@@ -210,7 +270,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
                                r0 + t * kBM, bh);
         q_issued = true;
         for (int j = 0; j < nk; ++j) {
-          const int kt = tr.tile(j);
+          const int kt = step_tile(j);
           const int s = j & 1;
           const uint32_t ph = ((j >> 1) & 1) ^ 1;
           if (!wait_bounded(dev::smem_u32(&sm.bar_kempty[s]), ph, abort)) break;
@@ -312,14 +372,14 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       auto wait_v = [&](int j) {
         return wait_bounded(dev::smem_u32(&sm.bar_vfull[j & 1]), (j >> 1) & 1, abort);
       };
-      auto next_step = [&](const TileRange& r, int j) {
+      auto next_step = [&](int t, int j) {
         int q = j + 1;
-        while (q < nk && !in_range(r, q)) ++q;
+        while (q < nk && !takes_part(t, q)) ++q;
         return q;
       };
       // per tile: cur = the step whose S has been issued and whose P V is next; cnt = steps
       // whose P V has been issued (the tile's barrier phases count only its own steps)
-      int cur0 = next_step(trt[0], -1), cur1 = next_step(trt[1], -1);
+      int cur0 = next_step(0, -1), cur1 = next_step(1, -1);
       int cnt0 = 0, cnt1 = 0;
       auto first_s = [&](int t, int cur) {
         if (cur >= nk) return true;
@@ -336,7 +396,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         dev::tc_fence_after();
         issue_pv(t, j & 1, cnt > 0);
         ++cnt;
-        const int nxt = next_step(trt[t], j);
+        const int nxt = next_step(t, j);
         if (nxt < nk) {
           if (!wait_k(nxt)) return false;
           dev::tc_fence_after();
@@ -389,14 +449,13 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
     bool ok = true;
 
-    const TileRange mine = t ? trt[1] : trt[0];
     int cnt = 0;  // steps this tile has processed
     for (int j = 0; j < nk; ++j) {
-      if (!in_range(mine, j)) continue;
+      if (!takes_part(t, j)) continue;
       ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), cnt & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
       dev::tc_fence_after();
-      const int kt = tr.tile(j);
+      const int kt = step_tile(j);
       const int key0 = kt * kBN;
 
       // the whole 128-column score row of this thread, one wait
@@ -520,6 +579,14 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + h
                                   : static_cast<size_t>(bh) * p.Nq + grow;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
+      // This warp's 32 rows leave as two 32-row x 64-column TMA boxes staged, 128-byte
+      // swizzled, in the tile's Q buffer, which no MMA reads any more (bar_o[t] covered every
+      // MMA of the tile).  A tile without steps never waited for its Q copy, and a box of
+      // packed sequences must not reach past its sequence: those rows use plain stores (a box
+      // wholly past the last row is not stored at all; a dense box is clipped at Nq).
+      const int wrow0 = r0 + t * kBM + (warp & 3) * 32;  // first row of this warp's box
+      const bool tma_out = cnt > 0 && wrow0 < nq && (!kVarlen || wrow0 + 31 < nq);
+      const uint32_t box0 = dev::smem_u32(sm.q[t]) + (warp & 3) * 4096;
 #pragma unroll 1
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t o[32];
@@ -535,11 +602,31 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         for (int e = 0; e < 32; e += 2)
           pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
                                         __uint_as_float(o[e + 1]) * inv_l);
-        if (valid) {
+        if (tma_out) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4) {
+            const int c16 = cc * 4 + v4;  // 16-byte chunk of the 256-byte row
+            const uint32_t a = box0 + (c16 >> 3) * kHalfBytes + lane * 128 +
+                               (static_cast<uint32_t>((c16 & 7) ^ (lane & 7)) << 4);
+            dev::st_shared_v4(a, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        } else if (valid) {
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
+      }
+      if (tma_out) {
+        dev::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          for (int half = 0; half < 2; ++half)
+            dev::tma_store_3d(&tm_o, box0 + half * kHalfBytes, half * 64,
+                              kVarlen ? q_base + wrow0 : wrow0, kVarlen ? h : bh);
+          dev::bulk_commit_group();
+          dev::bulk_wait_group_read0();  // the buffer is free again before the CTA ends
+        }
+        __syncwarp();
       }
       if (valid && p.lse != nullptr) {
         const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
@@ -563,8 +650,19 @@ template <bool kNeg, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, kVarlen, false>(tm_q, tm_k, tm_v, p);
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, tm_o, p);
+}
+
+// bf16 Q, K, V (dense) under a block-sparse layout
+template <bool kNeg>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_bf16_sparse_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                 const __grid_constant__ CUtensorMap tm_k,
+                                 const __grid_constant__ CUtensorMap tm_v,
+                                 const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 // E4M3 Q, K, V with per-(b, head) descale factors (dense)
@@ -572,8 +670,9 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, false, true>(tm_q, tm_k, tm_v, p);
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 }  // namespace fwd

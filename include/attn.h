@@ -106,6 +106,25 @@ ATTN_API int attn_fwd(const void *q, const void *k, const void *v, void *o, floa
              attn_stream_t stream);
 
 /*
+ * attn_fwd_block_sparse - attn_fwd under a fixed block-sparse layout ("Quadratic Complexity
+ * Bottleneck", sparse attention patterns: the sequence cut into blocks, attention computed
+ * within and between selected blocks; the selection is the caller's).
+ *   block_mask  DEVICE uint8 [mask_heads][ceil(Nq / 128)][ceil(Nk / 128)]: entry (hm, qt, kt)
+ *               != 0 selects query rows [128 qt, 128 qt + 128) against keys [128 kt, 128 kt + 128)
+ *               of head h, hm = h when mask_heads == Hq, hm = 0 when mask_heads == 1 (one
+ *               layout for every head); shared by the batch.  Read only, not kept.
+ *   A key is visible to a query row iff its block is selected and the mask (mask_kind, window,
+ *   n_sink) admits it; a row with no visible key gets O = 0 and LSE = -inf.
+ *   mask_heads == 1 or Hq (else ATTN_ERR_INVALID_ARG); block_mask may be NULL only when there
+ *   is nothing to compute; ceil(Nk / 128) <= 4096 (else ATTN_ERR_UNSUPPORTED).
+ *   Other arguments, layouts and rules as attn_fwd.
+ */
+ATTN_API int attn_fwd_block_sparse(const void *q, const void *k, const void *v, void *o,
+                                   float *lse, const uint8_t *block_mask, int mask_heads, int B,
+                                   int Hq, int Hkv, int Nq, int Nk, int d, int mask_kind,
+                                   int window, int n_sink, float scale, attn_stream_t stream);
+
+/*
  * attn_fwd_varlen - attn_fwd on packed variable-length sequences ("What Lost, and Why", the note
  * on sequence packing: several sequences concatenated in one batch row, attention masked block
  * diagonally so that it resets at every boundary given by cu_seqlens).

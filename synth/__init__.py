@@ -137,6 +137,20 @@ def normal_e4m3(seed: int, tensor_id: int, shape, head_axes: int = 2):
 # directly on the GPU; equality with the numpy stream is checked on the CPU by the tests).
 # --------------------------------------------------------------------------------------------
 
+def block_layout_bigbird(seed: int, n_qtiles: int, n_ktiles: int, n_random: int = 3) -> np.ndarray:
+    """A fixed block-sparse layout [1][n_qtiles][n_ktiles] (uint8) in the BigBird style: the
+    three blocks around the diagonal, the first block row and column (global), and n_random
+    further key blocks per block row, drawn without replacement from the seeded generator."""
+    bm = np.zeros((1, n_qtiles, n_ktiles), np.uint8)
+    r = np.random.default_rng(seed)
+    for qt in range(n_qtiles):
+        bm[0, qt, max(0, qt - 1):min(n_ktiles, qt + 2)] = 1
+        bm[0, qt, r.choice(n_ktiles, size=min(n_random, n_ktiles), replace=False)] = 1
+    bm[0, 0, :] = 1
+    bm[0, :, 0] = 1
+    return bm
+
+
 def _s64(c: int) -> int:
     c &= _MASK64
     return c - (1 << 64) if c >= (1 << 63) else c

@@ -115,3 +115,15 @@ def test_tensors_on_two_devices_are_refused():
     raises(ValueError, "one device", A.attn_fwd, q, k, v, o=t(2, 8, 5, 128, device="meta"))
     raises(ValueError, "one device", A.attn_decode, t(3, 8, 1, 128), t(3, 2, 100, 128),
            t(3, 2, 100, 128), workspace=t(16, dtype=u8, device="meta"))
+
+
+def test_block_sparse_layout_checks():
+    q, k, v = t(2, 8, 300, 128), t(2, 2, 450, 128), t(2, 2, 450, 128)
+    raises(ValueError, "CUDA tensors", A.attn_fwd_block_sparse, q, k, v, t(1, 3, 4, dtype=u8))
+    raises(ValueError, "CUDA tensors", A.attn_fwd_block_sparse, q, k, v, t(8, 3, 4, dtype=torch.bool))
+    raises(ValueError, "block_mask must have shape", A.attn_fwd_block_sparse, q, k, v, t(1, 3, 3, dtype=u8))
+    raises(ValueError, "block_mask must have shape", A.attn_fwd_block_sparse, q, k, v, t(1, 2, 4, dtype=u8))
+    raises(ValueError, "1 or Hq", A.attn_fwd_block_sparse, q, k, v, t(2, 3, 4, dtype=u8))
+    raises(TypeError, "block_mask must be", A.attn_fwd_block_sparse, q, k, v, t(1, 3, 4, dtype=i32))
+    raises(ValueError, "v must have shape", A.attn_fwd_block_sparse, q, k, t(2, 2, 449, 128),
+           t(1, 3, 4, dtype=u8))
