@@ -381,13 +381,27 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       // whose P V has been issued (the tile's barrier phases count only its own steps)
       int cur0 = next_step(0, -1), cur1 = next_step(1, -1);
       int cnt0 = 0, cnt1 = 0;
-      auto first_s = [&](int t, int cur) {
-        if (cur >= nk) return true;
-        if (!wait_k(cur)) return false;
+      // K_j can be waited for at any time up to step j + 2: K_(j+2) reuses the slot of K_j,
+      // which is released at the end of step j - 1.  A block-sparse tile may skip many steps
+      // (the other tile takes them); the S of a step more than two ahead is then deferred
+      // (pend) and issued during the step before it, ahead of that K slot's release.  Dense
+      // masks never skip that far: a tile's steps are contiguous after its first, which is
+      // step 0 or 1.
+      int pend0 = -1, pend1 = -1;
+      auto issue_s_at = [&](int t, int j) {
+        if (!wait_k(j)) return false;
         dev::tc_fence_after();
-        issue_s(t, cur & 1);
+        issue_s(t, j & 1);
         dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
         return true;
+      };
+      auto first_s = [&](int t, int cur) {
+        if (cur >= nk) return true;
+        if (kSparse && cur > 1) {
+          (t ? pend1 : pend0) = cur;
+          return true;
+        }
+        return issue_s_at(t, cur);
       };
       // one step of tile t at step j: P V, then the S of its next step (or the final commit)
       auto step = [&](int t, int j, int& cur, int& cnt) {
@@ -398,10 +412,11 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         ++cnt;
         const int nxt = next_step(t, j);
         if (nxt < nk) {
-          if (!wait_k(nxt)) return false;
-          dev::tc_fence_after();
-          issue_s(t, nxt & 1);
-          dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
+          if (kSparse && nxt > j + 2) {
+            (t ? pend1 : pend0) = nxt;
+          } else if (!issue_s_at(t, nxt)) {
+            return false;
+          }
         } else {
           dev::umma_commit(dev::smem_u32(&sm.bar_o[t]));
         }
@@ -420,6 +435,17 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       for (int j = 0; ok && j < nk; ++j) {
         if (!(ok = wait_v(j))) break;
         if (!(ok = step(0, j, cur0, cnt0) && step(1, j, cur1, cnt1))) break;
+        if constexpr (kSparse) {
+          // deferred S of step j + 1 (K_(j+1) is released below)
+          if (pend0 == j + 1) {
+            if (!(ok = issue_s_at(0, j + 1))) break;
+            pend0 = -1;
+          }
+          if (pend1 == j + 1) {
+            if (!(ok = issue_s_at(1, j + 1))) break;
+            pend1 = -1;
+          }
+        }
         // every P V reading V_j and every S reading K_(j+1) is issued by now
         dev::umma_commit(dev::smem_u32(&sm.bar_vempty[j & 1]));
         if (j + 1 < nk) {
