@@ -5,13 +5,20 @@
 
 A step is one call of the library on one batch of synthetic input (iid N(0,1), seeded,
 counter-based generator in ``synth``), with the inputs resident in HBM.  The headline workload
-is causal self-attention prefill, B=4, Hq=Hkv=16, n=2048, d=128, bf16 (fp32 accumulate); the
-same line carries the split-K decode workload (64 sequences x 1 token, Hq=32, Hkv=8, 32768
-cached keys) under "decode", because the metric names both.
+is the largest single-GPU prefill: causal sliding-window attention, B=1, Hq=32, Hkv=8 (GQA),
+n=32768, d=128, a 4096-key window plus 4 always-visible sink tokens, bf16 (fp32 accumulate).
+The same line carries, each with its own timing, roofline, end-to-end figure, clocks and CPU
+baseline, the GQA causal prefill (B=2, Hq=32, Hkv=8, n=8192) under "gqa_causal", the causal
+prefill (B=4, Hq=Hkv=16, n=2048) under "causal", and the split-K decode workload (64 sequences x
+1 token, Hq=32, Hkv=8, 32768 cached keys) under "decode", because the metric names both prefill
+and decode.
 
 Timing: W warm-up steps, then K timed steps; before every timed step a 256 MiB buffer is
 written (more than the 126 MB L2) and the step itself is bracketed by CUDA events on the
-launching stream; ``ms_per_step`` is the mean of the K event intervals.  With N > 1 (torchrun,
+launching stream; ``ms_per_step`` is the mean of the K event intervals.  The headline and the
+decode entry time exactly K steps; the two other prefill entries time at least K steps and as
+many more as give about 0.2 s of device time, so that the clock sampler (NVML, every 1 ms) sees
+the GPU under load; their own ``steps`` says how many.  With N > 1 (torchrun,
 one process per GPU) every rank runs its own replica of the workload on its own GPU (weak
 scaling: independent batches, no data-path collective), the ranks meet at a barrier before and
 after the timed loop, and the slowest rank's time sets the whole-job throughput.
@@ -85,8 +92,16 @@ WORKLOADS = {
 PROFILING_ONLY = ("decode_b8_h32_kv8_n32768_d128", "paged_decode_b8_h32_kv8_n32768_p16_d128")
 # fp32 FMA peak of the CUDA cores (TFLOP/s), for the fp32 workload, which uses no tensor core
 FP32_FMA_PEAK_TFLOPS = round(148 * 128 * 2 * 1965e6 / 1e12, 1)
-HEADLINE = "causal_b4_h16_n2048_d128"
+HEADLINE = "sliding_b1_h32_kv8_n32768_w4096_s4_d128"
 DECODE = "decode_b64_h32_kv8_n32768_d128"
+# entries of the default line besides the headline: (key, workload, fixed step count?)
+EXTRAS = (("gqa_causal", "gqa_causal_b2_h32_kv8_n8192_d128", False),
+          ("causal", "causal_b4_h16_n2048_d128", False),
+          ("decode", DECODE, True))
+# nominal datasheet denominators, quoted beside the measured ones: dense bf16 tensor peak of a
+# B200, and the HBM bandwidth the decode target is stated against
+NOMINAL = {"tensor": 2250.0, "hbm": 8000.0}
+MIN_TIMED_MS = 200.0
 
 # DRAM traffic per launch of each workload's dominant kernel, from one ncu capture
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the sources of that
@@ -111,7 +126,8 @@ NCU_TRAFFIC = {
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
 # up grids and tensor maps)
 FAMILY_SOURCES = {
-    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh",
+                "dev/exp2_poly.cuh"),
     "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
     "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
 }
@@ -221,7 +237,7 @@ _REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_po
 
 
 class ClockSampler:
-    def __init__(self, device_index, interval_s=0.005):
+    def __init__(self, device_index, interval_s=0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.interval = interval_s
         self.ok = False
@@ -483,13 +499,20 @@ def whole_job_value(work_per_step, steps, total_ms_max, world, scale):
     return world * work_per_step * steps / (total_ms_max * 1e-3) / scale
 
 
-def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_kind):
+def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_kind,
+                 min_timed_ms=0.0):
+    """Time one workload.  With min_timed_ms > 0 the step count grows past ``steps`` until the
+    timed steps add up to about that much device time (the same count on every rank)."""
     import torch
 
     wl = Workload(name, rank)
     w = wl.w
     work, unit, scale = work_of(w)
     A = wl.A
+    if min_timed_ms > 0:
+        probe = timed_loop(wl.run, 3, warmup, flush, dist_on)
+        est = max_over_ranks(min(probe), dist_on)
+        steps = max(steps, int(math.ceil(min_timed_ms / max(est, 1e-3))))
     sampler = ClockSampler(torch.cuda.current_device())
     times = timed_loop(wl.run, steps, warmup, flush, dist_on, sampler)
     err = A.attn_get_device_error()
@@ -522,30 +545,93 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
     roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,
             "frac": round(achieved / peak, 4) if peak else None, "traffic": traffic,
             "peak_source": source}
+    if bound in NOMINAL and w["kind"] != "fwd_fp8":
+        roof["peak_nominal"] = NOMINAL[bound]
+        roof["frac_nominal"] = round(achieved / NOMINAL[bound], 4)
 
     # end to end through the public API with host buffers: H2D of inputs, call, D2H of results
-    host_in = [t.cpu().pin_memory() for t in wl.inputs]
-    dev_in = [torch.empty_like(t) for t in wl.inputs]
-    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.outputs]
+    e2e = end_to_end(wl, work, scale, unit, max(3, min(steps, 20)), flush, world, dist_on)
+    return dict(wl=wl, work=work, unit=unit, value=value, ms_per_step=ms_per_step,
+                roofline=roof, e2e=e2e, clocks=sampler.report(),
+                launches=wl.launches_per_step * steps, steps=steps)
 
-    def e2e_step():
-        for dst, src in zip(dev_in, host_in):
+
+def end_to_end(wl, work, scale, unit, steps, flush, world, dist_on):
+    """The metric through the public API from pinned host buffers: every step copies its inputs
+    host -> device, runs the call and copies its results device -> host.
+
+    Pipelined (the reported value): the copies run on their own streams, two device copies of
+    the inputs alternate, so the upload of step i + 1 overlaps the call and the download of step
+    i; a call waits for its inputs and for the download of the previous results (the outputs
+    are single-buffered).  The serial figure (each step's upload, call and download one after
+    the other on one stream) is reported beside it.  An L2 flush precedes every call."""
+    import torch
+
+    host_in = [t.cpu().pin_memory() for t in wl.inputs]
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in wl.outputs]
+    dev_in = [[torch.empty_like(t) for t in wl.inputs] for _ in range(2)]
+    h2d_bytes = sum(t.numel() * t.element_size() for t in host_in)
+    d2h_bytes = sum(t.numel() * t.element_size() for t in host_out)
+
+    def serial_step():
+        for dst, src in zip(dev_in[0], host_in):
             dst.copy_(src, non_blocking=True)
-        wl.run(dev_in)
+        wl.run(dev_in[0])
         for dst, src in zip(host_out, wl.outputs):
             dst.copy_(src, non_blocking=True)
 
-    e2e_times = timed_loop(e2e_step, max(3, min(steps, 20)), 2, flush, dist_on)
-    e2e_ms = max_over_ranks(sum(e2e_times), dist_on) / len(e2e_times)
-    h2d = sum(t.numel() * t.element_size() for t in host_in)
-    d2h = sum(t.numel() * t.element_size() for t in host_out)
-    e2e = {"value": round(world * work / (e2e_ms * 1e-3) / scale, 3), "unit": unit,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-           "ms_per_step": round(e2e_ms, 4)}
-    del host_in, dev_in
-    return dict(wl=wl, work=work, unit=unit, value=value, ms_per_step=ms_per_step,
-                roofline=roof, e2e=e2e, clocks=sampler.report(),
-                launches=wl.launches_per_step * steps)
+    serial = timed_loop(serial_step, steps, 2, flush, dist_on)
+    serial_ms = max_over_ranks(sum(serial), dist_on) / len(serial)
+
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def pipelined(n):
+        ev_comp = [torch.cuda.Event() for _ in range(n)]
+        ev_up = [torch.cuda.Event() for _ in range(n)]
+        ev_down = [torch.cuda.Event() for _ in range(n)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        up.wait_stream(comp)
+        start.record(up)
+        for i in range(n):
+            buf = dev_in[i & 1]
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(ev_comp[i - 2])  # the call two steps back read this buffer
+                for dst, src in zip(buf, host_in):
+                    dst.copy_(src, non_blocking=True)
+                ev_up[i].record(up)
+            comp.wait_event(ev_up[i])
+            if i >= 1:
+                comp.wait_event(ev_down[i - 1])  # the previous results have left
+            flush.zero_()
+            wl.run(buf)
+            ev_comp[i].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(ev_comp[i])
+                for dst, src in zip(host_out, wl.outputs):
+                    dst.copy_(src, non_blocking=True)
+                ev_down[i].record(down)
+        end.record(down)
+        comp.wait_stream(down)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end)
+
+    pipelined(2)  # warm-up
+    if dist_on:
+        import torch.distributed as dist
+
+        dist.barrier()
+    total = max_over_ranks(pipelined(steps), dist_on)
+    if dist_on:
+        dist.barrier()
+    ms = total / steps
+    return {"value": round(world * work / (ms * 1e-3) / scale, 3), "unit": unit,
+            "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
+            "ms_per_step": round(ms, 4), "steps": steps,
+            "pipelined": "upload of step i+1 overlaps the call and download of step i",
+            "serial_ms_per_step": round(serial_ms, 4),
+            "serial_value": round(world * work / (serial_ms * 1e-3) / scale, 3)}
 
 
 # ----------------------------------------------------------------------------------------------
@@ -652,6 +738,45 @@ def oracle_sample(name, budget_s, seed=0, host=None):
             seqs += 1
         return done, secs, cores, "%d of %d sequences (all %d heads, %d cached keys in %d-key pages)" % (
             seqs, B, Hq, N, ps)
+
+    if w["kind"] in ("fwd", "fwd_block_sparse"):
+        # one (b, query head) slice at a time (its Q slice and its kv head's K, V slices are
+        # drawn alone, not timed), a growing batch of its rows
+        bm = None
+        if w["kind"] == "fwd_block_sparse":
+            assert w["mask"] == FULL, "the block-sparse sample cuts query blocks of a full mask"
+            nt = -(-N // 128)
+            bm = synth.block_layout_bigbird(w["seed"], nt, nt, w["n_random"])
+        done_rows, secs, work, batch = 0, 0.0, 0, 64
+        while secs < budget_s and done_rows < B * Hq * N:
+            b, h = int(rng.integers(0, B)), int(rng.integers(0, Hq))
+            qq = _draw_slice(w, synth.Q_ID, b * Hq + h, N * d).reshape(1, 1, N, d)
+            kk = _draw_slice(w, synth.K_ID, b * Hkv + h // G, N * d).reshape(1, 1, N, d)
+            vv = _draw_slice(w, synth.V_ID, b * Hkv + h // G, N * d).reshape(1, 1, N, d)
+            if bm is None:
+                rows = rng.integers(0, N, size=batch)
+                t0 = time.perf_counter()
+                O.attention_rows(qq, kk, vv, rows, w["mask"], w["window"], w["n_sink"], scale)
+                secs += time.perf_counter() - t0
+                work += sum(4 * d * acc.visible_pairs(1, int(r) + 1, w["mask"], w["window"],
+                                                      w["n_sink"]) if w["mask"] != FULL
+                            else 4 * d * N for r in rows)
+                done_rows += batch
+            else:
+                # whole 128-row query blocks: the layout row of block qt applies to all of them
+                for qt in rng.integers(0, bm.shape[1], size=max(1, batch // 128)):
+                    lo, hi = int(qt) * 128, min(N, int(qt) * 128 + 128)
+                    t0 = time.perf_counter()
+                    O.attention_block_sparse(qq[:, :, lo:hi], kk, vv, bm[:, qt:qt + 1], FULL,
+                                             scale=scale)
+                    secs += time.perf_counter() - t0
+                    keys = sum(min(128, N - 128 * j) for j in range(bm.shape[2]) if bm[0, qt, j])
+                    work += 4 * d * (hi - lo) * keys
+                    done_rows += hi - lo
+            batch = min(batch * 2, 4096)
+        return work, secs, cores, "%d output rows of random (b, head) slices, drawn at random " \
+            "(with replacement)%s" % (done_rows, " in whole 128-row blocks" if bm is not None
+                                      else "")
 
     q = draw(synth.Q_ID, (B, Hq, N, d)) if host is None else host[0]
     k = draw(synth.K_ID, (B, Hkv, N, d)) if host is None else host[1]
@@ -793,16 +918,20 @@ def main():
                 "config": config_of(name, w, world), "roofline": r["roofline"], "e2e": r["e2e"],
                 "gpu_launches": r["launches"], "clocks": r["clocks"]}
         del r["wl"]
+        cpu_on = rank == 0 and world == 1 and not args.no_cpu_baseline
         if args.workload is None and name == HEADLINE:
-            d = measure_ours(DECODE, max(5, args.steps // 5), args.warmup, rank, world, dist_on,
-                             flush, peaks, peak_kind)
-            del d["wl"]
-            line["decode"] = {"workload": DECODE, "value": round(d["value"], 2), "unit": d["unit"],
-                              "ms_per_step": round(d["ms_per_step"], 4),
-                              "roofline": d["roofline"], "e2e": d["e2e"], "clocks": d["clocks"],
-                              "gpu_launches": d["launches"]}
-            line["gpu_launches"] += d["launches"]
-        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            for key, xname, fixed in EXTRAS:
+                x = measure_ours(xname, args.steps, args.warmup, rank, world, dist_on, flush,
+                                 peaks, peak_kind, 0.0 if fixed else MIN_TIMED_MS)
+                del x["wl"]
+                sub = {"workload": xname, "config": config_of(xname, WORKLOADS[xname], world),
+                       "value": round(x["value"], 3), "unit": x["unit"], "steps": x["steps"],
+                       "ms_per_step": round(x["ms_per_step"], 5), "roofline": x["roofline"],
+                       "e2e": x["e2e"], "clocks": x["clocks"], "gpu_launches": x["launches"]}
+                if cpu_on:
+                    sub["cpu_baseline"] = cpu_baseline(xname, budget_s=8.0)
+                line[key] = sub
+        if cpu_on:
             line["cpu_baseline"] = cpu_baseline(name)
         if rank == 0:
             print(json.dumps(line), flush=True)

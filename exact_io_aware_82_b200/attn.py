@@ -32,7 +32,7 @@ EXPORTS = ("attn_abi_version", "attn_status_string", "attn_last_error_detail", "
            "attn_fwd_block_sparse")
 
 # size of the library-owned scratch array behind attn_decode_noalloc (include/attn.h)
-DECODE_NOALLOC_MAX_BYTES = 32 << 20
+DECODE_NOALLOC_MAX_BYTES = 64 << 20
 
 _lib = None
 

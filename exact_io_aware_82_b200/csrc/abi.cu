@@ -14,6 +14,7 @@
 #include "bwd_sm100.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_tc.cuh"
 #include "fwd_f32.cuh"
 #include "fwd_sm100.cuh"
 
@@ -29,6 +30,7 @@ struct DeviceInfo {
   int num_sms = 0;
   bool fwd_configured = false;
   bool bwd_configured = false;
+  bool dtc_configured = false;
 };
 
 std::mutex g_mutex;
@@ -102,6 +104,26 @@ int configure_fwd(DeviceInfo* info) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Raises the dynamic shared memory limit of the tensor-core decode kernels on first use (and
+// looks up the tensor-map encoder, as configure_fwd does).
+int configure_decode_tc(DeviceInfo* info) {
+  int rc = configure_fwd(info);
+  if (rc != ATTN_OK) return rc;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!info->dtc_configured) {
+    void (*kernels[4])(CUtensorMap, CUtensorMap, CUtensorMap, float*, float*, int, int, int, int,
+                       int, float) = {dtc::decode_tc_kernel<1>, dtc::decode_tc_kernel<2>,
+                                      dtc::decode_tc_kernel<4>, dtc::decode_tc_kernel<8>};
+    for (auto* kern : kernels) {
+      rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(dtc::kSmemBytes)));
+      if (rc != ATTN_OK) return rc;
+    }
+    info->dtc_configured = true;
+  }
+  return ATTN_OK;
+}
 
 // Raises the dynamic shared memory limit of the backward kernels on first use.
 int configure_bwd(DeviceInfo* info) {
@@ -257,11 +279,14 @@ int decode_splits(int B, int Hkv, int Nk, int G, int requested, int num_sms) {
   const int min_splits = Nk > 0 ? (Nk + max_chunk - 1) / max_chunk : 1;
   int s = requested;
   if (s <= 0) {
-    // enough CTAs for several waves of 2 resident CTAs per SM, chunks of at most max_chunk
-    const int groups = B * Hkv > 0 ? B * Hkv : 1;
-    const int want = (4 * 2 * num_sms + groups - 1) / groups;
-    const int by_len = Nk > 0 ? (Nk + 255) / 256 : 1;  // at least 256 keys per split
-    s = want < by_len ? want : by_len;
+    // chunks of whole 128-key tiles, at most the tensor-core kernel's dtc::kMaxChunk keys, and
+    // small enough for about 4 CTAs per SM (2 are resident at a time)
+    const long long groups = B * Hkv > 0 ? static_cast<long long>(B) * Hkv : 1;
+    const long long want = (4LL * num_sms + groups - 1) / groups;
+    long long chunk = Nk > 0 ? (Nk + want - 1) / want : 1;
+    chunk = (chunk + dtc::kTile - 1) / dtc::kTile * dtc::kTile;
+    if (chunk > dtc::kMaxChunk) chunk = dtc::kMaxChunk;
+    s = Nk > 0 ? static_cast<int>((Nk + chunk - 1) / chunk) : 1;
   }
   if (s < min_splits) s = min_splits;
   if (s < 1) s = 1;
@@ -311,6 +336,26 @@ int decode_run(const void* q, const void* k, const void* v, void* o, float* lse,
   float* ws_lse = ws_o + static_cast<size_t>(B) * Hq * splits * dec::kD;
   const float c = scale * kLog2e;
   const dim3 grid(splits, Hkv, B);
+  if (pg == nullptr && chunk <= dtc::kMaxChunk) {
+    // contiguous cache, chunks of at most kMaxChunk keys: the tensor-core split kernel
+    int rc = configure_decode_tc(const_cast<DeviceInfo*>(info));
+    if (rc != ATTN_OK) return rc;
+    CUtensorMap tq, tk, tv;
+    if (encode_map(&tq, q, B * Hq, 1, dtc::kN) != ATTN_OK ||
+        encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK || encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      return ATTN_ERR_UNSUPPORTED;
+    switch (G) {
+      case 1: dtc::decode_tc_kernel<1><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
+      case 2: dtc::decode_tc_kernel<2><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
+      case 4: dtc::decode_tc_kernel<4><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
+      default: dtc::decode_tc_kernel<8><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
+    }
+    rc = cuda_status(cudaGetLastError());
+    if (rc != ATTN_OK) return rc;
+    dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(
+        ws_o, ws_lse, static_cast<__nv_bfloat16*>(o), lse, splits);
+    return cuda_status(cudaGetLastError());
+  }
   const auto* qb = static_cast<const __nv_bfloat16*>(q);
   const auto* kb = static_cast<const __nv_bfloat16*>(k);
   const auto* vb = static_cast<const __nv_bfloat16*>(v);
@@ -400,6 +445,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = nullptr;
@@ -451,6 +497,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.front_heavy = (mask_kind == ATTN_MASK_FULL || mask_kind == ATTN_MASK_LOCAL_GLOBAL) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.block_mask = block_mask;
@@ -506,6 +553,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = (max_seqlen_q + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = cu_seqlens_q;
@@ -556,6 +604,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = nullptr;

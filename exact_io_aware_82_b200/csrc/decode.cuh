@@ -76,6 +76,35 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// The G scores of one key in the shared score buffer ([chunk][G] floats, 16-byte aligned).
+template <int G>
+__device__ __forceinline__ void load_scores(const float* p, float (&sc)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + i);
+      sc[i] = x.x, sc[i + 1] = x.y, sc[i + 2] = x.z, sc[i + 3] = x.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    sc[0] = x.x, sc[1] = x.y;
+  } else {
+    sc[0] = p[0];
+  }
+}
+template <int G>
+__device__ __forceinline__ void store_scores(float* p, const float (&sc)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4)
+      *reinterpret_cast<float4*>(p + i) = make_float4(sc[i], sc[i + 1], sc[i + 2], sc[i + 3]);
+  } else if constexpr (G == 2) {
+    *reinterpret_cast<float2*>(p) = make_float2(sc[0], sc[1]);
+  } else {
+    p[0] = sc[0];
+  }
+}
+
 // kPage: 0 = contiguous cache; 1 = paged, any page size; 2 = paged, pages of at least 2U keys
 // (one page lookup per warp iteration).
 template <int G, int kPage>
@@ -88,7 +117,8 @@ __device__ __forceinline__ void decode_split(const __nv_bfloat16* __restrict__ q
   constexpr int U = unroll<G>();
   constexpr int NV = U * G;        // partial dot products per thread per iteration
   constexpr int PER_LANE = NV / 16;  // fully reduced scores each lane ends with
-  extern __shared__ float smem[];   // scores/probabilities [chunk][G], later the P V partials
+  extern __shared__ __align__(16) float smem[];  // scores/probabilities [chunk][G], later the
+                                                 // P V partials
   __shared__ float red_m[kWarps][G];
   __shared__ float stat[2][G];     // max (log2 units) and sum per head
 
@@ -197,23 +227,37 @@ __device__ __forceinline__ void decode_split(const __nv_bfloat16* __restrict__ q
         part[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
       }
     }
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i) {
-      const int idx = sl * PER_LANE + i;  // = u * G + g
+    if constexpr (PER_LANE == 2 && G >= 2) {
+      // the lane's two scores are heads g, g + 1 of one key: one 8-byte store (a warp's
+      // stores then fill 256 consecutive bytes)
+      const int idx = sl * 2;  // = u * G + g
       const int u = idx / G, g = idx % G;
       const int key = kw + 2 * u + half;
-      if (key < n) smem[key * G + g] = part[i];
+      if (key < n) *reinterpret_cast<float2*>(smem + key * G + g) = make_float2(part[0], part[1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < PER_LANE; ++i) {
+        const int idx = sl * PER_LANE + i;  // = u * G + g
+        const int u = idx / G, g = idx % G;
+        const int key = kw + 2 * u + half;
+        if (key < n) smem[key * G + g] = part[i];
+      }
     }
   }
   __syncthreads();
 
   // ---------------- softmax statistics per head ----------------
+  // a key's G scores are read and written as one unit (16-byte words for G >= 4), so that the
+  // lanes of a warp touch consecutive words instead of every G-th one (bank conflicts)
   float mx[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) mx[g] = -INFINITY;
-  for (int key = tid; key < n; key += kThreads)
+  for (int key = tid; key < n; key += kThreads) {
+    float sc[G];
+    load_scores<G>(smem + key * G, sc);
 #pragma unroll
-    for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], smem[key * G + g]);
+    for (int g = 0; g < G; ++g) mx[g] = fmaxf(mx[g], sc[g]);
+  }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -233,13 +277,16 @@ __device__ __forceinline__ void decode_split(const __nv_bfloat16* __restrict__ q
     mx[g] = stat[0][g];
     sum[g] = 0.f;
   }
-  for (int key = tid; key < n; key += kThreads)
+  for (int key = tid; key < n; key += kThreads) {
+    float sc[G];
+    load_scores<G>(smem + key * G, sc);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float pr = exp2f(smem[key * G + g] - mx[g]);
-      smem[key * G + g] = pr;
-      sum[g] += pr;
+      sc[g] = exp2f(sc[g] - mx[g]);
+      sum[g] += sc[g];
     }
+    store_scores<G>(smem + key * G, sc);
+  }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
 #pragma unroll
@@ -289,9 +336,11 @@ __device__ __forceinline__ void decode_split(const __nv_bfloat16* __restrict__ q
   __syncthreads();  // all probabilities consumed; the score buffer becomes the partial buffer
   if (half == 0)
 #pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) smem[(warp * G + g) * kD + 8 * sl + e] = acc[g][e];
+    for (int g = 0; g < G; ++g) {
+      float4* dst = reinterpret_cast<float4*>(smem + (warp * G + g) * kD + 8 * sl);
+      dst[0] = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
+      dst[1] = make_float4(acc[g][4], acc[g][5], acc[g][6], acc[g][7]);
+    }
   __syncthreads();
   for (int idx = tid; idx < G * kD; idx += kThreads) {
     const int g = idx / kD, dcol = idx % kD;

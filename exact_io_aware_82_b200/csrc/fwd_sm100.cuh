@@ -36,8 +36,11 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "dev/ptx_f8.cuh"
+#include "dev/exp2_poly.cuh"
 #include "dev/ptx_store.cuh"
 
 namespace attn {
@@ -58,6 +61,14 @@ static_assert(kThreads * kRegsLaunch <= 65536, "launch register budget");
 constexpr uint32_t kTileBytes = kBM * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column half
 constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
+// bf16 weights: of every 8 pairs of scores in a tile without masked entries, this many take
+// their exponentials on the FMA pipe (dev/exp2_poly.cuh) instead of the multi-function unit
+#ifndef ATTN_EMU_PAIRS
+#define ATTN_EMU_PAIRS 0
+#endif
+
+constexpr int kEmuPairs = ATTN_EMU_PAIRS;
+static_assert(kEmuPairs >= 0 && kEmuPairs <= 8, "pairs out of 8");
 // E4M3 operands (kFp8): P is scaled by kPScaleF8 before it is rounded to E4M3 and the running
 // maximum is refreshed whenever it grows by more than 1 (log2 units), so scaled P stays below
 // 2 * 128 = 256 <= 448 (the largest E4M3 value) while small weights keep 128x more range.
@@ -72,6 +83,10 @@ struct Params {
   const int* cu_k;            // [cu_q[s], cu_q[s+1]) and key rows [cu_k[s], cu_k[s+1])
   float c;  // scale * log2(e): scores are handled in log2 units (never 0, see the host code)
   int num_qblocks;
+  // query blocks are taken in ascending order (the heaviest come first when the rows that see
+  // the most keys are at the front: global query rows, or a block layout's global block row);
+  // otherwise descending (causal and sliding masks: later rows see more keys)
+  int front_heavy;
   __nv_bfloat16* o;
   float* lse;
   // E4M3 operands only: per (b, head) factors that turn the codes into values
@@ -144,10 +159,10 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work unit: heaviest query blocks first (causal), the G heads of a kv head adjacent ----
+  // ---- work unit: heaviest query blocks first, the G heads of a kv head adjacent ----
   const int nbh = p.B * p.Hq;
   const int unit = blockIdx.x;
-  const int qb = p.num_qblocks - 1 - unit / nbh;
+  const int qb = p.front_heavy ? unit / nbh : p.num_qblocks - 1 - unit / nbh;
   const int bh = unit % nbh;
   const int b = bh / p.Hq, h = bh % p.Hq;
   const int bkv = b * p.Hkv + h / p.G;
@@ -490,7 +505,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       for (int cc = 0; cc < 4; ++cc) dev::tmem_ld32(t_s + cc * 32, r + cc * 32);
       dev::tmem_wait_ld_regs(r);
 
-      if (!tile_is_full(mask, P0, kt)) {
+      const bool full = tile_is_full(mask, P0, kt);
+      if (!full) {
         // visible columns of this row inside the tile: (lo <= col <= hi) or col < sk,
         // as a 128-bit set built with shifts, then one bit test and select per column (no
         // per-column branches, whatever the compiler knows about hi, lo and sk)
@@ -570,15 +586,32 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           }
           dev::tmem_st16(t_s + half * 16, pk);
         } else {
+          // s * c - m_use two at a time; then 2^x on the multi-function unit, or, for
+          // kEmuPairs of every 8 pairs of a tile no mask touches, on the FMA pipe
+          // (exp2_poly2: a masked score must give exactly 0, which only ex2 does)
+          const uint64_t c2 = dev::pack2(c, c), nm2 = dev::pack2(-m_use, -m_use);
           uint32_t pk[32];
+          auto weights = [&](auto emulate) {
 #pragma unroll
-          for (int e = 0; e < 64; e += 2) {
-            const int col = half * 64 + e;
-            const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
-            const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
-            acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
-            pk[e >> 1] = dev::pack_bf16x2(p0, p1);
-          }
+            for (int e = 0; e < 64; e += 2) {
+              const int col = half * 64 + e;
+              const uint64_t x = dev::fma2(dev::pack2(__uint_as_float(r[col]),
+                                                      __uint_as_float(r[col + 1])), c2, nm2);
+              float2 pr;
+              if (decltype(emulate)::value && ((col >> 1) * kEmuPairs) % 8 < kEmuPairs) {
+                pr = dev::exp2_poly2(x);
+              } else {
+                const float2 xx = dev::unpack2(x);
+                pr = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+              }
+              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr);
+              pk[e >> 1] = dev::pack_bf16x2(pr.x, pr.y);
+            }
+          };
+          if (kEmuPairs > 0 && full)
+            weights(std::true_type{});
+          else
+            weights(std::false_type{});
           dev::tmem_st32(t_s + half * 32, pk);
         }
       }

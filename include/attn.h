@@ -265,7 +265,7 @@ ATTN_API int attn_decode_paged(const void *q, const void *k_cache, const void *v
  *    (different streams, or different host threads, without ordering between them) race on it.
  * The pages describe no counterpart of this entry point; it exists for callers only.
  */
-#define ATTN_DECODE_NOALLOC_MAX_BYTES (32u << 20)
+#define ATTN_DECODE_NOALLOC_MAX_BYTES (64u << 20)
 
 ATTN_API int attn_decode_noalloc(const void *q, const void *k, const void *v, void *o, float *lse,
                                  int B, int Hq, int Hkv, int Nk, int d, float scale,

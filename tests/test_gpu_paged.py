@@ -113,15 +113,11 @@ def test_paged_decode_all_lengths_zero():
     run_case(54, [0, 0], 8, 2, 16)
 
 
-def test_paged_equals_contiguous_decode_bitwise():
-    # pages laid out in order (page p = keys [p*ps, (p+1)*ps) of one (b, all heads) slab) give
-    # the same keys in the same order; with a split count whose chunk is already a multiple of
-    # 32 keys (the paged chunk granularity: 6000 / 47 -> 128) both calls use the same chunks,
-    # so the results are identical
-    B, Hq, Hkv, N, d, ps, splits = 4, 32, 8, 6000, 128, 16, 47
-    q = synth.normal_torch(55, synth.Q_ID, (B, Hq, 1, d), device="cuda")
-    k = synth.normal_torch(55, synth.K_ID, (B, Hkv, N, d), device="cuda")
-    v = synth.normal_torch(55, synth.V_ID, (B, Hkv, N, d), device="cuda")
+def _paged_vs_contiguous(seed, B, Hq, Hkv, N, ps, splits):
+    d = 128
+    q = synth.normal_torch(seed, synth.Q_ID, (B, Hq, 1, d), device="cuda")
+    k = synth.normal_torch(seed, synth.K_ID, (B, Hkv, N, d), device="cuda")
+    v = synth.normal_torch(seed, synth.V_ID, (B, Hkv, N, d), device="cuda")
     oc, lc = A.attn_decode(q, k, v, num_splits=splits)
     npg = N // ps + 1
     to_pages = lambda t: torch.nn.functional.pad(  # noqa: E731
@@ -130,7 +126,23 @@ def test_paged_equals_contiguous_decode_bitwise():
     sl = torch.full((B,), N, dtype=torch.int32, device="cuda")
     op, lp = A.attn_decode_paged(q, to_pages(k), to_pages(v), table, sl, N, num_splits=splits)
     torch.cuda.synchronize()
+    return (oc, lc), (op, lp)
+
+
+def test_paged_equals_contiguous_decode_bitwise():
+    # pages laid out in order (page p = keys [p*ps, (p+1)*ps) of one (b, all heads) slab) give
+    # the same keys in the same order; with chunks of more than 1024 keys (6144 / 4 = 1536, a
+    # multiple of the paged path's 32-key granularity) both calls run the CUDA-core split
+    # kernel on the same chunks, so the results are identical
+    (oc, lc), (op, lp) = _paged_vs_contiguous(55, 4, 32, 8, 6144, 16, 4)
     assert torch.equal(op, oc) and torch.equal(lp, lc)
+
+
+def test_paged_matches_tensor_core_contiguous_decode():
+    # chunks of at most 1024 keys: the contiguous cache goes through the tensor-core split
+    # kernel, the paged one through the CUDA-core kernel; the two agree within the bf16 limits
+    (oc, lc), (op, lp) = _paged_vs_contiguous(57, 4, 32, 8, 6000, 16, 47)
+    assert_close(to64(op), to64(lp), to64(oc), to64(lc), TOL_BF16, "paged vs contiguous")
 
 
 def test_page_number_outside_cache_is_flagged_not_followed():
