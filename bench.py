@@ -126,9 +126,8 @@ NCU_TRAFFIC = {
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
 # up grids and tensor maps)
 FAMILY_SOURCES = {
-    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh",
-                "dev/exp2_poly.cuh"),
-    "decode": ("decode.cuh", "common.cuh", "dev/ptx.cuh"),
+    "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
+    "decode": ("decode.cuh", "decode_tc.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
     "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
 }
 
@@ -159,6 +158,34 @@ def kernel_sources_hash(family: str) -> str:
         with open(os.path.join(csrc, f)) as fh:
             h.update((f + "\0" + code_tokens(fh.read())).encode())
     return h.hexdigest()[:16]
+
+
+def fp8_gemm_peak():
+    """Measured dense E4M3 tensor throughput of this GPU (TFLOP/s): torch._scaled_mm (cuBLASLt)
+    on 8192^3 E4M3 x E4M3 -> bf16 with per-tensor scales, best of 10 after 3 warm-ups (the
+    method the bf16 figure of MEASURED_PEAKS.json uses, with the FP8 GEMM).  None if the call is
+    unavailable."""
+    import torch
+
+    n = 8192
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()  # column-major
+        one = torch.ones((), device="cuda")
+        for _ in range(3):
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        return round(2 * n ** 3 / (best * 1e-3) / 1e12, 1)
+    except (RuntimeError, AttributeError, TypeError):
+        return None
 
 
 def load_peaks():
@@ -529,17 +556,22 @@ def measure_ours(name, steps, warmup, rank, world, dist_on, flush, peaks, peak_k
         bound, peak, punit = "hbm", peaks["hbm_gbs"], "GB/s"
     else:
         bound, peak, punit = "tensor", peaks["bf16_tflops"], "TFLOP/s"
+        fp8_peak = None
         if w["kind"] == "fwd_fp8":
-            # no FP8 GEMM was measured: the bf16 figure times the nominal ratio 4.5 / 2.25
-            peak = round(2.0 * peaks["bf16_tflops"], 1)
+            fp8_peak = fp8_gemm_peak()
+            # measured here; if the FP8 GEMM cannot run, the bf16 figure times the nominal
+            # ratio 4.5 / 2.25
+            peak = fp8_peak if fp8_peak else round(2.0 * peaks["bf16_tflops"], 1)
         if w["kind"] == "fwd_f32":
             # fp32 FMA on the CUDA cores: 148 SMs x 128 FMA lanes x 2 FLOP x 1965 MHz (the
             # maximum SM clock), no tensor core
             bound, peak = "alu", FP32_FMA_PEAK_TFLOPS
     tr = NCU_TRAFFIC.get(name)
     traffic = tr["bytes"] if tr and tr["src"] == kernel_sources_hash(family_of(w)) else None
-    source = peak_kind + (" burst" if bound == "tensor" else "") + (
-        " bf16 x 2 (nominal FP8 / BF16 ratio)" if w["kind"] == "fwd_fp8" else "")
+    source = peak_kind + (" burst" if bound == "tensor" else "")
+    if w["kind"] == "fwd_fp8":
+        source = ("measured in this run: torch._scaled_mm E4M3 8192^3, best of 10" if fp8_peak
+                  else peak_kind + " burst bf16 x 2 (nominal FP8 / BF16 ratio)")
     if bound == "alu":
         source = "derived: 148 SMs x 128 fp32 FMA/clk x 2 FLOP x 1965 MHz"
     roof = {"bound": bound, "achieved": round(achieved, 2), "peak": peak, "unit": punit,

@@ -112,9 +112,12 @@ int configure_decode_tc(DeviceInfo* info) {
   if (rc != ATTN_OK) return rc;
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->dtc_configured) {
-    void (*kernels[4])(CUtensorMap, CUtensorMap, CUtensorMap, float*, float*, int, int, int, int,
-                       int, float) = {dtc::decode_tc_kernel<1>, dtc::decode_tc_kernel<2>,
-                                      dtc::decode_tc_kernel<4>, dtc::decode_tc_kernel<8>};
+    void (*kernels[8])(CUtensorMap, CUtensorMap, CUtensorMap, float*, float*, int, int, int, int,
+                       int, float, dec::Paged) = {
+        dtc::decode_tc_kernel<1, false>, dtc::decode_tc_kernel<2, false>,
+        dtc::decode_tc_kernel<4, false>, dtc::decode_tc_kernel<8, false>,
+        dtc::decode_tc_kernel<1, true>,  dtc::decode_tc_kernel<2, true>,
+        dtc::decode_tc_kernel<4, true>,  dtc::decode_tc_kernel<8, true>};
     for (auto* kern : kernels) {
       rc = cuda_status(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                             static_cast<int>(dtc::kSmemBytes)));
@@ -336,20 +339,41 @@ int decode_run(const void* q, const void* k, const void* v, void* o, float* lse,
   float* ws_lse = ws_o + static_cast<size_t>(B) * Hq * splits * dec::kD;
   const float c = scale * kLog2e;
   const dim3 grid(splits, Hkv, B);
-  if (pg == nullptr && chunk <= dtc::kMaxChunk) {
-    // contiguous cache, chunks of at most kMaxChunk keys: the tensor-core split kernel
+  if (chunk <= dtc::kMaxChunk && (pg == nullptr || pg->page_shift >= dtc::kMinTcPageShift)) {
+    // chunks of at most kMaxChunk keys, contiguous or in pages of at least 64 keys: the
+    // tensor-core split kernel
     int rc = configure_decode_tc(const_cast<DeviceInfo*>(info));
     if (rc != ATTN_OK) return rc;
     CUtensorMap tq, tk, tv;
-    if (encode_map(&tq, q, B * Hq, 1, dtc::kN) != ATTN_OK ||
-        encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK || encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
-      return ATTN_ERR_UNSUPPORTED;
-    switch (G) {
-      case 1: dtc::decode_tc_kernel<1><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
-      case 2: dtc::decode_tc_kernel<2><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
-      case 4: dtc::decode_tc_kernel<4><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
-      default: dtc::decode_tc_kernel<8><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c); break;
+    if (encode_map(&tq, q, B * Hq, 1, dtc::kN) != ATTN_OK) return ATTN_ERR_UNSUPPORTED;
+    if (pg == nullptr) {
+      if (encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK || encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+        return ATTN_ERR_UNSUPPORTED;
+    } else {
+      const long long rows = static_cast<long long>(pg->num_pages) << pg->page_shift;
+      const uint32_t piece = (1u << pg->page_shift) < 32u ? (1u << pg->page_shift) : 32u;
+      if (rows > 0x7fffffffLL || encode_map_packed(&tk, k, static_cast<int>(rows), Hkv, piece) != ATTN_OK ||
+          encode_map_packed(&tv, v, static_cast<int>(rows), Hkv, piece) != ATTN_OK)
+        return ATTN_ERR_UNSUPPORTED;
     }
+    const dec::Paged pgv = pg != nullptr ? *pg : dec::Paged{};
+    const bool paged = pg != nullptr;
+#define ATTN_LAUNCH_DTC(GG)                                                                      \
+  do {                                                                                           \
+    if (paged)                                                                                   \
+      dtc::decode_tc_kernel<GG, true><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(             \
+          tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, pgv);                         \
+    else                                                                                         \
+      dtc::decode_tc_kernel<GG, false><<<grid, dtc::kThreads, dtc::kSmemBytes, st>>>(            \
+          tq, tk, tv, ws_o, ws_lse, Hq, Hkv, Nk, chunk, splits, c, pgv);                         \
+  } while (0)
+    switch (G) {
+      case 1: ATTN_LAUNCH_DTC(1); break;
+      case 2: ATTN_LAUNCH_DTC(2); break;
+      case 4: ATTN_LAUNCH_DTC(4); break;
+      default: ATTN_LAUNCH_DTC(8); break;
+    }
+#undef ATTN_LAUNCH_DTC
     rc = cuda_status(cudaGetLastError());
     if (rc != ATTN_OK) return rc;
     dec::decode_combine_kernel<<<B * Hq, dec::kD, 0, st>>>(
@@ -642,6 +666,26 @@ int attn_fwd_f32(const float* q, const float* k, const float* v, float* o, float
   p.G = Hq / Hkv;
   p.mask = make_mask(mask_kind, window, n_sink, Nk);
   p.c = scale * kLog2e;
+  // the kv head's whole K and V in shared memory (at most 512 keys, about 200 KB): one warp per
+  // query row; otherwise the tiled kernel
+  const size_t small_bytes = d == 64 ? f32::small_smem_bytes<64>(Nk) : f32::small_smem_bytes<128>(Nk);
+  if (Nk <= 32 * f32::kSmallMaxChunks && small_bytes <= 200 * 1024) {
+    const dim3 grid((Nq + f32::kSmallWarps - 1) / f32::kSmallWarps, Hq, B);
+    if (d == 64) {
+      rc = cuda_status(cudaFuncSetAttribute(f32::fwd_f32_small_kernel<64>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(small_bytes)));
+      if (rc != ATTN_OK) return rc;
+      f32::fwd_f32_small_kernel<64><<<grid, f32::kSmallWarps * 32, small_bytes, st>>>(q, k, v, o, lse, p);
+    } else {
+      rc = cuda_status(cudaFuncSetAttribute(f32::fwd_f32_small_kernel<128>,
+                                            cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                            static_cast<int>(small_bytes)));
+      if (rc != ATTN_OK) return rc;
+      f32::fwd_f32_small_kernel<128><<<grid, f32::kSmallWarps * 32, small_bytes, st>>>(q, k, v, o, lse, p);
+    }
+    return cuda_status(cudaGetLastError());
+  }
   if (d == 64) {
     dim3 grid((Nq + f32::rows_per_cta<64>() - 1) / f32::rows_per_cta<64>(), Hq, B);
     f32::fwd_f32_kernel<64><<<grid, f32::kWarps * 32, 0, st>>>(q, k, v, o, lse, p);

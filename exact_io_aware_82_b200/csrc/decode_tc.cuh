@@ -1,4 +1,4 @@
-// Split-K decode on the tensor cores, contiguous KV cache.
+// Split-K decode on the tensor cores, contiguous or paged KV cache.
 //
 // The method is that of decode.cuh ("Attention Research" (learning-materials), section 1: a
 // decode step reads the whole KV cache, so it is bound by HBM bandwidth; section 2:
@@ -27,6 +27,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "dev/ptx_store.cuh"
 
 namespace attn {
@@ -49,6 +50,10 @@ constexpr uint32_t kPBlockBytes = kN * 64 * 2;       // P^T rows of 64 keys: 16 
 constexpr uint32_t kPTileBytes = 2 * kPBlockBytes;   // 4 KB per tile of 128 keys
 constexpr uint32_t kTmemCols = 256;                  // S^T: kMaxTiles x 16 columns; O^T: 16
 constexpr uint32_t kOCol = kMaxTiles * kN;
+// Paged caches take this kernel from 64-key pages up: with 16-key pages the 16 boxes per tile
+// streamed slower than the CUDA-core kernel's loads (4.7 vs 5.5 TB/s); with 64- and 256-key
+// pages faster (6.2-6.3 vs 5.1-5.4 TB/s).
+constexpr int kMinTcPageShift = 6;
 
 struct __align__(1024) Smem {
   uint8_t ring[kStages][kTileBytes];
@@ -67,15 +72,20 @@ __device__ __forceinline__ void softmax_bar_sync() {
   asm volatile("bar.sync 1, %0;" ::"n"(kSoftThreads) : "memory");
 }
 
-// Q: [B * Hq][d] (one token per sequence); K, V: [B][Hkv][Nk][d]; partials as decode.cuh:
-// ws_o [B][Hq][splits][d] (O_s / l_s), ws_lse [B][Hq][splits] (natural log).
-template <int G>
+// Q: [B * Hq][d] (one token per sequence); partials as decode.cuh: ws_o [B][Hq][splits][d]
+// (O_s / l_s), ws_lse [B][Hq][splits] (natural log).
+// kPaged = false: K, V [B][Hkv][Nk][d], maps (d, Nk, B * Hkv) read as 128-key boxes.
+// kPaged = true: the paged cache of decode.cuh, K, V [num_pages][page_size][Hkv][d], maps
+// (d, num_pages * page_size, Hkv) read as boxes of min(page_size, 32) keys (chunks are whole
+// multiples of 32 keys, so a box never crosses a page); a page number outside the cache is not
+// followed (the box is taken past the last row, which reads as zero) and is flagged.
+template <int G, bool kPaged>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, float* __restrict__ ws_o,
                      float* __restrict__ ws_lse, int Hq, int Hkv, int Nk, int chunk, int splits,
-                     float c) {
+                     float c, dec::Paged pg) {
   static_assert(G == 1 || G == 2 || G == 4 || G == 8, "query heads per kv head");
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -83,7 +93,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int s = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int j0 = s * chunk;
-  const int n = max(0, min(Nk - j0, chunk));  // keys of this split
+  // keys of this sequence: Nk (contiguous cache) or its own length (paged cache)
+  const int len = kPaged ? max(0, min(__ldg(pg.seq_lens + b), Nk)) : Nk;
+  const int n = max(0, min(len - j0, chunk));  // keys of this split
   const int T = (n + kTile - 1) / kTile;
   auto out_row = [&](int g) { return (static_cast<size_t>(b) * Hq + hk * G + g) * splits + s; };
 
@@ -145,9 +157,31 @@ __global__ void __launch_bounds__(kThreads, 2)
         dev::mbar_arrive_expect_tx(bf, kTileBytes);
         const CUtensorMap* map = u < T ? &tm_k : &tm_v;
         const int row = j0 + (u < T ? u : u - T) * kTile;  // rows past Nk read as zero
-        for (int half = 0; half < 2; ++half)
-          dev::tma_load_3d(dev::smem_u32(sm.ring[st]) + half * kHalfBytes, map, bf, half * 64,
-                           row, b * Hkv + hk);
+        if constexpr (!kPaged) {
+          for (int half = 0; half < 2; ++half)
+            dev::tma_load_3d(dev::smem_u32(sm.ring[st]) + half * kHalfBytes, map, bf, half * 64,
+                             row, b * Hkv + hk);
+        } else {
+          // pieces of min(page_size, 32) keys, each inside one page
+          const int psize = 1 << pg.page_shift;
+          const int piece = psize < 32 ? psize : 32;
+          const long long rows_total = static_cast<long long>(pg.num_pages) << pg.page_shift;
+          for (int r = 0; r < kTile; r += piece) {
+            const int key = row + r;  // logical key of the piece's first row
+            int tok = static_cast<int>(rows_total);  // past the last row: reads as zero
+            if (key < len) {
+              const int lp = key >> pg.page_shift;
+              const int phys = lp < pg.max_pages ? __ldg(pg.block_table + static_cast<size_t>(b) * pg.max_pages + lp) : -1;
+              if (phys >= 0 && phys < pg.num_pages)
+                tok = (phys << pg.page_shift) + (key & (psize - 1));
+              else
+                atomicExch(&g_device_error, ATTN_ERR_INVALID_ARG);
+            }
+            for (int half = 0; half < 2; ++half)
+              dev::tma_load_3d(dev::smem_u32(sm.ring[st]) + half * kHalfBytes + r * 128, map, bf,
+                               half * 64, tok, hk);
+          }
+        }
         ++issued;
       }
       // ---- drain: every copy this thread started has landed before the CTA ends ----

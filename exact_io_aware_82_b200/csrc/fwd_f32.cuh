@@ -126,5 +126,113 @@ __global__ void __launch_bounds__(kWarps * 32)
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Small problems (the K and V rows of one kv head fit in shared memory, e.g. n = 256, d = 64):
+// the tiled kernel above then runs a handful of CTAs through a long dependent chain of key
+// tiles.  Here every CTA copies the kv head's whole K and V into shared memory at once and each
+// warp computes one query row: all scores of the row (lane = key within a 32-key chunk, four
+// independent partial sums per dot product), the exact row max and sum by warp shuffles, then
+// P V (lane = output columns, each weight broadcast from its lane).  Same definition and
+// results as the tiled kernel; no online rescaling is needed since the whole row is at hand.
+// ------------------------------------------------------------------------------------------
+constexpr int kSmallWarps = 8;     // query rows per CTA
+constexpr int kSmallMaxChunks = 16;  // keys per row: at most 16 x 32 = 512
+template <int D>
+__host__ __device__ constexpr int small_stride() { return D + 4; }  // padded row (floats)
+template <int D>
+__host__ __device__ constexpr size_t small_smem_bytes(int Nk) {
+  return static_cast<size_t>(Nk) * small_stride<D>() * 2 * sizeof(float);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kSmallWarps * 32)
+    fwd_f32_small_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                         const float* __restrict__ v, float* __restrict__ o,
+                         float* __restrict__ lse, const Params p) {
+  constexpr int S = small_stride<D>();
+  constexpr int kCols = D / 32;
+  extern __shared__ float4 smem_f4[];
+  float* ks = reinterpret_cast<float*>(smem_f4);
+  float* vs = ks + static_cast<size_t>(p.Nk) * S;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const size_t bh = static_cast<size_t>(b) * p.Hq + h;
+  const size_t bkv = static_cast<size_t>(b) * p.Hkv + h / p.G;
+  const float4* kb = reinterpret_cast<const float4*>(k + bkv * p.Nk * D);
+  const float4* vb = reinterpret_cast<const float4*>(v + bkv * p.Nk * D);
+  for (int e = tid; e < p.Nk * (D / 4); e += kSmallWarps * 32) {
+    const int r = e / (D / 4), c4 = e % (D / 4);
+    *reinterpret_cast<float4*>(ks + r * S + 4 * c4) = __ldg(kb + e);
+    *reinterpret_cast<float4*>(vs + r * S + 4 * c4) = __ldg(vb + e);
+  }
+  __syncthreads();
+
+  const int row = blockIdx.x * kSmallWarps + warp;
+  if (row >= p.Nq) return;
+  const int prow = row + p.Nk - p.Nq;
+  const float4* qr = reinterpret_cast<const float4*>(q + (bh * p.Nq + row) * D);
+  float qv[D];
+#pragma unroll
+  for (int c4 = 0; c4 < D / 4; ++c4) {
+    const float4 x = __ldg(qr + c4);
+    qv[4 * c4] = x.x, qv[4 * c4 + 1] = x.y, qv[4 * c4 + 2] = x.z, qv[4 * c4 + 3] = x.w;
+  }
+  const int nchunks = (p.Nk + 31) / 32;
+  float sc[kSmallMaxChunks];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int cix = 0; cix < kSmallMaxChunks; ++cix) {
+    sc[cix] = -INFINITY;
+    if (cix >= nchunks) continue;
+    const int key = cix * 32 + lane;
+    if (key < p.Nk && key_visible(p.mask, prow, key)) {
+      const float* kr = ks + key * S;
+      float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+      for (int t = 0; t < D; t += 4) {
+        const float4 kk = *reinterpret_cast<const float4*>(kr + t);
+        a0 = fmaf(qv[t], kk.x, a0);
+        a1 = fmaf(qv[t + 1], kk.y, a1);
+        a2 = fmaf(qv[t + 2], kk.z, a2);
+        a3 = fmaf(qv[t + 3], kk.w, a3);
+      }
+      sc[cix] = ((a0 + a1) + (a2 + a3)) * p.c;  // log2 units
+      mx = fmaxf(mx, sc[cix]);
+    }
+  }
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, sh));
+  float l = 0.f;
+  const float m_use = mx == -INFINITY ? 0.f : mx;
+#pragma unroll
+  for (int cix = 0; cix < kSmallMaxChunks; ++cix) {
+    sc[cix] = cix < nchunks ? exp2f(sc[cix] - m_use) : 0.f;  // 0 for masked keys
+    l += sc[cix];
+  }
+#pragma unroll
+  for (int sh = 16; sh > 0; sh >>= 1) l += __shfl_xor_sync(0xffffffffu, l, sh);
+  float acc[kCols];
+#pragma unroll
+  for (int cc = 0; cc < kCols; ++cc) acc[cc] = 0.f;
+#pragma unroll
+  for (int cix = 0; cix < kSmallMaxChunks; ++cix) {
+    if (cix >= nchunks) break;
+    const int keys = min(32, p.Nk - cix * 32);
+#pragma unroll 4
+    for (int jj = 0; jj < keys; ++jj) {
+      const float pj = __shfl_sync(0xffffffffu, sc[cix], jj);
+      const float* vr = vs + (cix * 32 + jj) * S;
+#pragma unroll
+      for (int cc = 0; cc < kCols; ++cc) acc[cc] = fmaf(pj, vr[lane + 32 * cc], acc[cc]);
+    }
+  }
+  const float inv = l > 0.f ? 1.f / l : 0.f;
+  float* orow = o + (bh * p.Nq + row) * D;
+#pragma unroll
+  for (int cc = 0; cc < kCols; ++cc) orow[lane + 32 * cc] = acc[cc] * inv;
+  if (lane == 0 && lse != nullptr)
+    lse[bh * p.Nq + row] = l > 0.f ? (mx + log2f(l)) * 0.69314718055994531f : -INFINITY;
+}
+
 }  // namespace f32
 }  // namespace attn

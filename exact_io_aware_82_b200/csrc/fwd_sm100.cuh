@@ -36,11 +36,9 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
-#include <type_traits>
 
 #include "common.cuh"
 #include "dev/ptx_f8.cuh"
-#include "dev/exp2_poly.cuh"
 #include "dev/ptx_store.cuh"
 
 namespace attn {
@@ -61,18 +59,14 @@ static_assert(kThreads * kRegsLaunch <= 65536, "launch register budget");
 constexpr uint32_t kTileBytes = kBM * kD * 2;  // 32 KB, bf16
 constexpr uint32_t kHalfBytes = kBM * 64 * 2;  // one 128-byte-swizzled column half
 constexpr float kRescaleThreshold = 8.0f;      // log2 units: rescale O only if the max grows by >8
-// bf16 weights: of every 8 pairs of scores in a tile without masked entries, this many take
-// their exponentials on the FMA pipe (dev/exp2_poly.cuh) instead of the multi-function unit
-#ifndef ATTN_EMU_PAIRS
-#define ATTN_EMU_PAIRS 0
-#endif
 
-constexpr int kEmuPairs = ATTN_EMU_PAIRS;
-static_assert(kEmuPairs >= 0 && kEmuPairs <= 8, "pairs out of 8");
+
 // E4M3 operands (kFp8): P is scaled by kPScaleF8 before it is rounded to E4M3 and the running
 // maximum is refreshed whenever it grows by more than 1 (log2 units), so scaled P stays below
 // 2 * 128 = 256 <= 448 (the largest E4M3 value) while small weights keep 128x more range.
 constexpr float kPScaleF8 = 128.0f;
+constexpr float kLog2PScaleF8 = 7.0f;
+
 constexpr float kRescaleThresholdF8 = 1.0f;
 
 struct Params {
@@ -489,6 +483,19 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
     bool ok = true;
+    // O_t *= alpha (per row), in tensor memory; O_t is complete here (the commit for S_t(j)
+    // covered PV_t(j-1)) and the next P V has not been issued
+    auto rescale_o = [&](float alpha) {
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t o[32];
+        dev::tmem_ld32(t_o + cc * 32, o);
+        dev::tmem_wait_ld_regs(o);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        dev::tmem_st32(t_o + cc * 32, o);
+      }
+    };
 
     int cnt = 0;  // steps this tile has processed
     for (int j = 0; j < nk; ++j) {
@@ -522,8 +529,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       }
 
       // row max of the raw scores (min when the scale is negative): 3-input max tree
-      float mx;
-      {
+      auto row_max = [&]() {
         float a[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r[i]);
@@ -538,10 +544,63 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
 #pragma unroll
         for (int i = 0; i < 8; ++i)
           a[i] = kNeg ? fminf(a[i], __uint_as_float(r[120 + i])) : fmaxf(a[i], __uint_as_float(r[120 + i]));
-        mx = kNeg ? dev::min3(dev::min3(a[0], a[1], a[2]), dev::min3(a[3], a[4], a[5]), fminf(a[6], a[7]))
-                  : dev::max3(dev::max3(a[0], a[1], a[2]), dev::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-      }
-      const float tmax = (mx == masked) ? neg_inf() : mx * c;
+        const float mx =
+            kNeg ? dev::min3(dev::min3(a[0], a[1], a[2]), dev::min3(a[3], a[4], a[5]), fminf(a[6], a[7]))
+                 : dev::max3(dev::max3(a[0], a[1], a[2]), dev::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+        return (mx == masked) ? neg_inf() : mx * c;  // in log2 units
+      };
+
+      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t (E4M3: four
+      // codes of kPScaleF8 * P per column over the first 32); the row sum accumulates in 8
+      // independent packed pairs
+      float2 acc[4];
+      auto weights = [&](float m_ref_now) {
+        const float m_use = (m_ref_now == neg_inf()) ? 0.f : m_ref_now;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if constexpr (kFp8) {
+            // the exponent carries log2(kPScaleF8), so the weights come out already scaled
+            // for the E4M3 product (the row sum takes the factor back out below)
+            const uint64_t c2 = dev::pack2(c, c);
+            const uint64_t nm2 = dev::pack2(kLog2PScaleF8 - m_use, kLog2PScaleF8 - m_use);
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 64; e += 4) {
+              const int col = half * 64 + e;
+              float2 pr[2];
+#pragma unroll
+              for (int h2 = 0; h2 < 2; ++h2) {
+                const int cc2 = col + 2 * h2;
+                const float2 xx = dev::unpack2(dev::fma2(
+                    dev::pack2(__uint_as_float(r[cc2]), __uint_as_float(r[cc2 + 1])), c2, nm2));
+                pr[h2] = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+              }
+              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr[0]);
+              acc[((e >> 1) + 1) & 3] = dev::add2(acc[((e >> 1) + 1) & 3], pr[1]);
+              pk[e >> 2] = dev::pack_e4m3x4(pr[0].x, pr[0].y, pr[1].x, pr[1].y);
+            }
+            dev::tmem_st16(t_s + half * 16, pk);
+          } else {
+            // s * c - m_use two at a time (packed fp32 FMA), 2^x on the multi-function unit
+            const uint64_t c2 = dev::pack2(c, c), nm2 = dev::pack2(-m_use, -m_use);
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const int col = half * 64 + e;
+              const float2 xx = dev::unpack2(dev::fma2(
+                  dev::pack2(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), c2, nm2));
+              const float2 pr = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr);
+              pk[e >> 1] = dev::pack_bf16x2(pr.x, pr.y);
+            }
+            dev::tmem_st32(t_s + half * 32, pk);
+          }
+        }
+      };
+
+      const float tmax = row_max();
       const float m_new = fmaxf(m_ref, tmax);
       float alpha = 1.f;
       if (m_new > m_ref + kThreshold) {
@@ -549,76 +608,12 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         m_ref = m_new;
       }
       l *= alpha;
-      const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
-
-      // rescale the running output O_t (complete: the commit for S_t(j) covered PV_t(j-1))
-      if (cnt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          dev::tmem_ld32(t_o + cc * 32, o);
-          dev::tmem_wait_ld_regs(o);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          dev::tmem_st32(t_o + cc * 32, o);
-        }
-      }
-
-      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t (E4M3: four
-      // codes of kPScaleF8 * P per column over the first 32); the row sum accumulates in 8
-      // independent packed pairs
-      float2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        if constexpr (kFp8) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 64; e += 4) {
-            const int col = half * 64 + e;
-            const float p0 = dev::ex2_approx(fmaf(__uint_as_float(r[col]), c, -m_use));
-            const float p1 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 1]), c, -m_use));
-            const float p2 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 2]), c, -m_use));
-            const float p3 = dev::ex2_approx(fmaf(__uint_as_float(r[col + 3]), c, -m_use));
-            acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], make_float2(p0, p1));
-            acc[((e >> 1) + 1) & 3] = dev::add2(acc[((e >> 1) + 1) & 3], make_float2(p2, p3));
-            pk[e >> 2] = dev::pack_e4m3x4(p0 * kPScaleF8, p1 * kPScaleF8, p2 * kPScaleF8,
-                                          p3 * kPScaleF8);
-          }
-          dev::tmem_st16(t_s + half * 16, pk);
-        } else {
-          // s * c - m_use two at a time; then 2^x on the multi-function unit, or, for
-          // kEmuPairs of every 8 pairs of a tile no mask touches, on the FMA pipe
-          // (exp2_poly2: a masked score must give exactly 0, which only ex2 does)
-          const uint64_t c2 = dev::pack2(c, c), nm2 = dev::pack2(-m_use, -m_use);
-          uint32_t pk[32];
-          auto weights = [&](auto emulate) {
-#pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-              const int col = half * 64 + e;
-              const uint64_t x = dev::fma2(dev::pack2(__uint_as_float(r[col]),
-                                                      __uint_as_float(r[col + 1])), c2, nm2);
-              float2 pr;
-              if (decltype(emulate)::value && ((col >> 1) * kEmuPairs) % 8 < kEmuPairs) {
-                pr = dev::exp2_poly2(x);
-              } else {
-                const float2 xx = dev::unpack2(x);
-                pr = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
-              }
-              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr);
-              pk[e >> 1] = dev::pack_bf16x2(pr.x, pr.y);
-            }
-          };
-          if (kEmuPairs > 0 && full)
-            weights(std::true_type{});
-          else
-            weights(std::false_type{});
-          dev::tmem_st32(t_s + half * 32, pk);
-        }
-      }
+      if (cnt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o(alpha);
+      weights(m_ref);
       acc[0] = dev::add2(acc[0], acc[1]);
       acc[2] = dev::add2(acc[2], acc[3]);
       acc[0] = dev::add2(acc[0], acc[2]);
-      l += acc[0].x + acc[0].y;
+      l += kFp8 ? (acc[0].x + acc[0].y) * (1.f / kPScaleF8) : acc[0].x + acc[0].y;
       dev::tmem_wait_st();
       dev::tc_fence_before();
       dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));

@@ -138,23 +138,38 @@ def test_paged_equals_contiguous_decode_bitwise():
     assert torch.equal(op, oc) and torch.equal(lp, lc)
 
 
-def test_paged_matches_tensor_core_contiguous_decode():
-    # chunks of at most 1024 keys: the contiguous cache goes through the tensor-core split
-    # kernel, the paged one through the CUDA-core kernel; the two agree within the bf16 limits
-    (oc, lc), (op, lp) = _paged_vs_contiguous(57, 4, 32, 8, 6000, 16, 47)
-    assert_close(to64(op), to64(lp), to64(oc), to64(lc), TOL_BF16, "paged vs contiguous")
+def test_paged_equals_contiguous_tensor_core_decode_bitwise():
+    # chunks of at most 1024 keys (6000 / 47 -> 128, already a multiple of 32) and pages of 64
+    # keys: both caches go through the tensor-core split kernel, with the same keys in the same
+    # tiles, so the results are identical too
+    (oc, lc), (op, lp) = _paged_vs_contiguous(57, 4, 32, 8, 6000, 64, 47)
+    assert torch.equal(op, oc) and torch.equal(lp, lc)
 
 
-def test_page_number_outside_cache_is_flagged_not_followed():
-    d, ps = 128, 16
+def test_tensor_core_and_cuda_core_decode_agree():
+    # the same problem through both split kernels (chunks of 128 keys vs 1536 keys)
+    B, Hq, Hkv, N, d = 2, 16, 4, 6144, 128
+    q = synth.normal_torch(58, synth.Q_ID, (B, Hq, 1, d), device="cuda")
+    k = synth.normal_torch(58, synth.K_ID, (B, Hkv, N, d), device="cuda")
+    v = synth.normal_torch(58, synth.V_ID, (B, Hkv, N, d), device="cuda")
+    ot, lt = A.attn_decode(q, k, v, num_splits=48)
+    oc, lc = A.attn_decode(q, k, v, num_splits=4)
+    torch.cuda.synchronize()
+    assert_close(to64(ot), to64(lt), to64(oc), to64(lc), TOL_BF16, "tensor-core vs CUDA-core")
+
+
+@pytest.mark.parametrize("ps", [16, 64])  # the CUDA-core and the tensor-core split kernels
+def test_page_number_outside_cache_is_flagged_not_followed(ps):
+    d = 128
     lens = [100, 200]
+    npg = (200 + ps - 1) // ps
     q = synth.normal_torch(56, synth.Q_ID, (2, 8, 1, d), device="cuda")
-    kc = synth.normal_torch(56, synth.K_ID, (40, ps, 2, d), device="cuda")
-    vc = synth.normal_torch(56, synth.V_ID, (40, ps, 2, d), device="cuda")
-    table = torch.arange(2 * 13, dtype=torch.int32, device="cuda").reshape(2, 13)
-    table[1, 3] = 1 << 30  # far outside the 40 pages
+    kc = synth.normal_torch(56, synth.K_ID, (2 * npg + 14, ps, 2, d), device="cuda")
+    vc = synth.normal_torch(56, synth.V_ID, (2 * npg + 14, ps, 2, d), device="cuda")
+    table = torch.arange(2 * npg, dtype=torch.int32, device="cuda").reshape(2, npg)
+    table[1, 1] = 1 << 30  # far outside the pool
     good = table.clone()
-    good[1, 3] = 39
+    good[1, 1] = 2 * npg + 13
     sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
     o_bad, _ = A.attn_decode_paged(q, kc, vc, table, sl, 200)
     assert A.attn_get_device_error() == A.ATTN_ERR_INVALID_ARG

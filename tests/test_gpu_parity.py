@@ -45,7 +45,9 @@ def test_fp32_single_head_full_workload():
 @pytest.mark.parametrize("Nq,Nk,mask,w,s,Hq,Hkv", [
     (1, 1, FULL, 0, 0, 1, 1), (33, 33, CAUSAL, 0, 0, 2, 1), (70, 150, CAUSAL, 0, 0, 4, 2),
     (150, 70, CAUSAL, 0, 0, 2, 2), (129, 129, SLIDING, 17, 3, 4, 1), (100, 100, SLIDING, 1, 0, 1, 1),
-    (65, 200, FULL, 0, 0, 8, 2)])
+    (65, 200, FULL, 0, 0, 8, 2),
+    # more than 512 keys: the tiled fp32 kernel (up to 512, the one with K/V in shared memory)
+    (40, 700, SLIDING, 100, 2, 2, 1), (30, 600, FULL, 0, 0, 2, 2)])
 def test_fp32_masks(d, Nq, Nk, mask, w, s, Hq, Hkv):
     (q, k, v), (q64, k64, v64) = f32_inputs(5, 2, Hq, Hkv, Nq, Nk, d)
     o, lse = A.attn_fwd_f32(q, k, v, mask_kind=mask, window=w, n_sink=s)
