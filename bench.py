@@ -107,20 +107,22 @@ MIN_TIMED_MS = 200.0
 # (dram__bytes_read.sum + dram__bytes_write.sum), keyed by the hash of the sources of that
 # kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
-    "causal_b4_h16_n2048_d128": {"bytes": 145144064, "src": "3b03bfebcd8b4903"},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 471887360, "src": "3b03bfebcd8b4903"},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 686198016, "src": "3b03bfebcd8b4903"},
-    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293224960, "src": "3b03bfebcd8b4903"},
-    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 828471040, "src": "3b03bfebcd8b4903"},
-    "fp8_causal_b4_h16_n2048_d128": {"bytes": 53103360, "src": "3b03bfebcd8b4903"},
+    "full_b1_h1_n256_d64_f32": {"bytes": 260608, "src": "02e210e28044d0c4"},
+    "causal_b4_h16_n2048_d128": {"bytes": 136256000, "src": "db22c40767b52c14"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 479916032, "src": "db22c40767b52c14"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 698571520, "src": "db22c40767b52c14"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1303387888, "src": "db22c40767b52c14"},
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 771768064, "src": "db22c40767b52c14"},
+    "fp8_causal_b4_h16_n2048_d128": {"bytes": 54390528, "src": "db22c40767b52c14"},
+    "block_sparse_b1_h32_kv8_n32768_d128": {"bytes": 1000239104, "src": "db22c40767b52c14"},
     # the backward step's three kernels together (prep + dK/dV + dQ)
-    "bwd_causal_b4_h16_n2048_d128": {"bytes": 1018073344, "src": "1309a00e4521aaf1"},
-    # captured on the 8-sequence cases; the cache is read once per sequence, so the
-    # 64-sequence launch moves 8x that
-    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1080556288, "src": "f0c69ebeb5d90fd1"},
-    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1080556288, "src": "f0c69ebeb5d90fd1"},
-    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1078285568, "src": "f0c69ebeb5d90fd1"},
-    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1078285568, "src": "f0c69ebeb5d90fd1"},
+    "bwd_causal_b4_h16_n2048_d128": {"bytes": 1037843968, "src": "0ea6bc652cc64f22"},
+    # a decode step's two kernels together (split + combine), captured on the 8-sequence
+    # cases; the cache is read once per sequence, so the 64-sequence step moves 8x that
+    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1084994200, "src": "08a4fbcfc6e70524"},
+    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1084994200, "src": "08a4fbcfc6e70524"},
+    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1085063864, "src": "08a4fbcfc6e70524"},
+    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1085063864, "src": "08a4fbcfc6e70524"},
 }
 
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
@@ -129,12 +131,15 @@ FAMILY_SOURCES = {
     "prefill": ("fwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_f8.cuh", "dev/ptx_store.cuh"),
     "decode": ("decode.cuh", "decode_tc.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
     "bwd": ("bwd_sm100.cuh", "common.cuh", "dev/ptx.cuh", "dev/ptx_store.cuh"),
+    "f32": ("fwd_f32.cuh", "common.cuh"),
 }
 
 
 def family_of(w):
     if w["kind"] in ("decode", "decode_paged"):
         return "decode"
+    if w["kind"] == "fwd_f32":
+        return "f32"
     return "bwd" if w["kind"] == "bwd" else "prefill"
 
 
