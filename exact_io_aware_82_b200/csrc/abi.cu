@@ -409,6 +409,23 @@ __global__ void timeout_probe_kernel(long long limit) {
   __syncthreads();
 }
 
+// The CTAs of a prefill launch.  With an even group size a CTA takes the same 128 rows of two
+// query heads that read one kv head, so its two query tiles see the same keys and every key
+// tile feeds both; otherwise a CTA takes 256 consecutive rows of one head.
+struct FwdSchedule {
+  int head_pair, num_qblocks;
+  long long units;
+};
+
+FwdSchedule fwd_schedule(int batch, int Hq, int Hkv, int rows) {
+  FwdSchedule sc;
+  sc.head_pair = (Hq / Hkv) % 2 == 0 ? 1 : 0;
+  const int per_cta = sc.head_pair ? fwd::kBM : fwd::kRowsPerCta;
+  sc.num_qblocks = (rows + per_cta - 1) / per_cta;
+  sc.units = static_cast<long long>(sc.num_qblocks) * batch * (sc.head_pair ? Hq / 2 : Hq);
+  return sc;
+}
+
 }  // namespace
 }  // namespace attn
 
@@ -447,8 +464,8 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (Nk == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
                              static_cast<size_t>(B) * Hq * Nq, d, st);
-  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
+  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
 
   CUtensorMap tq, tk, tv, to;
@@ -468,13 +485,14 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   // exp2 argument rounds to 0) while masked scores (-inf) still map to weight 0
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
-  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.num_qblocks = sc.num_qblocks;
+  p.head_pair = sc.head_pair;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = nullptr;
   p.cu_k = nullptr;
-  const dim3 grid(static_cast<unsigned>(units));
+  const dim3 grid(static_cast<unsigned>(sc.units));
   if (scale < 0.f)
     fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
@@ -502,8 +520,8 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   if (Nk == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
                              static_cast<size_t>(B) * Hq * Nq, d, st);
-  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
+  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
@@ -520,7 +538,8 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.mask = make_mask(mask_kind, window, n_sink, Nk);
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
-  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.num_qblocks = sc.num_qblocks;
+  p.head_pair = sc.head_pair;
   p.front_heavy = (mask_kind == ATTN_MASK_FULL || mask_kind == ATTN_MASK_LOCAL_GLOBAL) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -528,7 +547,7 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.mask_heads = mask_heads;
   p.mask_qtiles = mask_qtiles;
   p.mask_ktiles = mask_ktiles;
-  const dim3 grid(static_cast<unsigned>(units));
+  const dim3 grid(static_cast<unsigned>(sc.units));
   if (scale < 0.f)
     fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   else
@@ -557,9 +576,8 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   if (num_seqs == 0 || total_q == 0 || max_seqlen_q == 0) return ATTN_OK;
   if (total_k == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(total_q) * Hq, d, st);
-  const long long units = static_cast<long long>((max_seqlen_q + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) *
-                          num_seqs * Hq;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  const FwdSchedule sc = fwd_schedule(num_seqs, Hq, Hkv, max_seqlen_q);
+  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv, to;
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
@@ -576,13 +594,14 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.mask = make_mask(mask_kind, window, n_sink, total_k);
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
-  p.num_qblocks = (max_seqlen_q + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.num_qblocks = sc.num_qblocks;
+  p.head_pair = sc.head_pair;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = cu_seqlens_q;
   p.cu_k = cu_seqlens_k;
-  const dim3 grid(static_cast<unsigned>(units));
+  const dim3 grid(static_cast<unsigned>(sc.units));
   if (scale < 0.f)
     fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
@@ -609,8 +628,8 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   if (q_empty) return ATTN_OK;
   if (Nk == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq * Nq, d, st);
-  const long long units = static_cast<long long>((Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta) * B * Hq;
-  if (units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
+  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
   CUtensorMap tq, tk, tv, to;
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
@@ -627,7 +646,8 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.mask = make_mask(mask_kind, window, n_sink, Nk);
   p.c = scale * kLog2e;
   if (p.c == 0.f) p.c = 1e-30f;
-  p.num_qblocks = (Nq + fwd::kRowsPerCta - 1) / fwd::kRowsPerCta;
+  p.num_qblocks = sc.num_qblocks;
+  p.head_pair = sc.head_pair;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -636,7 +656,7 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.descale_q = descale_q;
   p.descale_k = descale_k;
   p.descale_v = descale_v;
-  const dim3 grid(static_cast<unsigned>(units));
+  const dim3 grid(static_cast<unsigned>(sc.units));
   if (scale < 0.f)
     fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else

@@ -10,8 +10,10 @@
 // Research" (learning-materials), section 2 (TMA and warp specialisation as in
 // FlashAttention-3, here re-expressed with tcgen05 and tensor memory).
 //
-// One CTA computes 256 query rows of one (batch, query head) as two 128-row tiles Q0, Q1 that
-// share every K/V tile.  Warp roles (12 warps = 3 warpgroups, 384 threads):
+// One CTA computes two 128-row query tiles Q0, Q1 that share every K/V tile: the same 128 rows
+// of two query heads of one kv head when the group size is even (both tiles then see exactly the
+// same keys, so every step feeds both), otherwise 256 consecutive rows of one query head.
+// Warp roles (12 warps = 3 warpgroups, 384 threads):
 //   warps 0-3   softmax + epilogue for Q0 (thread t owns row t, TMEM lanes 0-127)
 //   warps 4-7   softmax + epilogue for Q1
 //   warp 8      TMEM allocation and the single-thread tcgen05.mma issuer
@@ -81,6 +83,9 @@ struct Params {
   // the most keys are at the front: global query rows, or a block layout's global block row);
   // otherwise descending (causal and sliding masks: later rows see more keys)
   int front_heavy;
+  // 1: a CTA takes rows [128 qb, 128 qb + 128) of query heads 2i and 2i + 1 (G even, so both
+  // read kv head 2i / G); 0: rows [256 qb, 256 qb + 256) of one query head
+  int head_pair;
   __nv_bfloat16* o;
   float* lse;
   // E4M3 operands only: per (b, head) factors that turn the codes into values
@@ -154,13 +159,19 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   const int lane = tid & 31;
 
   // ---- work unit: heaviest query blocks first, the G heads of a kv head adjacent ----
-  const int nbh = p.B * p.Hq;
+  const bool pair = p.head_pair != 0;
+  const int heads_cta = pair ? 2 : 1;            // query heads of one CTA
+  const int rows_cta = pair ? kBM : kRowsPerCta;  // query rows of one CTA (per head)
+  const int nbh = p.B * (p.Hq / heads_cta);
   const int unit = blockIdx.x;
   const int qb = p.front_heavy ? unit / nbh : p.num_qblocks - 1 - unit / nbh;
-  const int bh = unit % nbh;
-  const int b = bh / p.Hq, h = bh % p.Hq;
+  const int b = (unit % nbh) / (p.Hq / heads_cta);
+  const int h = (unit % nbh) % (p.Hq / heads_cta) * heads_cta;  // (first) query head
   const int bkv = b * p.Hkv + h / p.G;
-  const int r0 = qb * kRowsPerCta;
+  const int r0 = qb * rows_cta;
+  // query tile t: its first row and its query head
+  auto tile_row0 = [&](int t) { return pair ? r0 : r0 + t * kBM; };
+  auto tile_head = [&](int t) { return pair ? h + t : h; };
   // rows of this (sequence, head): q_base / k_base = first packed row, nq / nkeys = lengths
   int q_base = 0, k_base = 0, nq = p.Nq, nkeys = p.Nk;
   MaskSpec mask = p.mask;
@@ -174,14 +185,14 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     if (r0 >= nq) return;  // the whole CTA leaves together: this sequence is shorter
   }
   const int off = nkeys - nq;
-  const int last_row = min(r0 + kRowsPerCta, nq) - 1;
+  const int last_row = min(r0 + rows_cta, nq) - 1;
   // key tiles of the whole CTA (what the producer loads, in this order) ...
   const TileRange tr = key_tiles(mask, r0 + off, last_row + off, kBN);
   const int nk_range = tr.count();
   // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
   TileRange trt[2];
   for (int t = 0; t < 2; ++t) {
-    const int lo_row = r0 + t * kBM, hi_row = min(lo_row + kBM, nq) - 1;
+    const int lo_row = tile_row0(t), hi_row = min(lo_row + kBM, nq) - 1;
     trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
                              : key_tiles(mask, lo_row + off, hi_row + off, kBN);
   }
@@ -194,10 +205,14 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   if (kSparse && warp == 0) {
     // the steps of a block-sparse CTA: the range's key tiles selected for query tile 0 or 1,
     // compacted in range order by one warp (ballot + prefix count)
-    const int hm = p.mask_heads == 1 ? 0 : h;
-    const uint8_t* row0 =
-        p.block_mask + (static_cast<size_t>(hm) * p.mask_qtiles + 2 * qb) * p.mask_ktiles;
-    const uint8_t* row1 = row0 + p.mask_ktiles;  // read only if query tile 1 has rows
+    // layout row of query tile t (read only if the tile has rows)
+    auto layout_row = [&](int t) {
+      const int hm = p.mask_heads == 1 ? 0 : tile_head(t);
+      return p.block_mask +
+             (static_cast<size_t>(hm) * p.mask_qtiles + tile_row0(t) / kBM) * p.mask_ktiles;
+    };
+    const uint8_t* row0 = layout_row(0);
+    const uint8_t* row1 = layout_row(1);
     int base = 0;
     for (int j0 = 0; j0 < nk_range; j0 += 32) {
       const int j = j0 + lane;
@@ -273,10 +288,10 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                               q_base + r0 + t * kBM, h);
+                               q_base + tile_row0(t), tile_head(t));
             else
               dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                               r0 + t * kBM, bh);
+                               tile_row0(t), b * p.Hq + tile_head(t));
         q_issued = true;
         for (int j = 0; j < nk; ++j) {
           const int kt = step_tile(j);
@@ -475,10 +490,12 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_off + t * 128;
     const uint32_t t_o = tmem + lane_off + 256 + t * 128;
-    const int P0 = r0 + t * kBM + off;  // key position of the tile's first row
+    const int hq = tile_head(t);        // query head of this tile
+    const int P0 = tile_row0(t) + off;  // key position of the tile's first row
     const int prow = P0 + row;          // key position of this thread's row
     // scores in log2 units: c = scale * log2(e), times the Q and K descale factors for E4M3
-    const float c = kFp8 ? p.c * __ldg(p.descale_q + bh) * __ldg(p.descale_k + bkv) : p.c;
+    const float c =
+        kFp8 ? p.c * __ldg(p.descale_q + b * p.Hq + hq) * __ldg(p.descale_k + bkv) : p.c;
     const float masked = kNeg ? pos_inf() : neg_inf();
     float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
     float l = 0.f;            // running sum of exp2(s*c - m_ref)
@@ -625,20 +642,20 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     ok = __all_sync(0xffffffffu, ok);
     if (ok) {
       dev::tc_fence_after();
-      const int grow = r0 + t * kBM + row;
+      const int grow = tile_row0(t) + row;
       const bool valid = grow < nq;
       // E4M3: undo the scale of P and apply the V descale factor
       const float o_mul = kFp8 ? __ldg(p.descale_v + bkv) / kPScaleF8 : 1.f;
       const float inv_l = l > 0.f ? o_mul / l : 0.f;
-      const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + h
-                                  : static_cast<size_t>(bh) * p.Nq + grow;
+      const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + hq
+                                  : static_cast<size_t>(b * p.Hq + hq) * p.Nq + grow;
       uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
       // This warp's 32 rows leave as two 32-row x 64-column TMA boxes staged, 128-byte
       // swizzled, in the tile's Q buffer, which no MMA reads any more (bar_o[t] covered every
       // MMA of the tile).  A tile without steps never waited for its Q copy, and a box of
       // packed sequences must not reach past its sequence: those rows use plain stores (a box
       // wholly past the last row is not stored at all; a dense box is clipped at Nq).
-      const int wrow0 = r0 + t * kBM + (warp & 3) * 32;  // first row of this warp's box
+      const int wrow0 = tile_row0(t) + (warp & 3) * 32;  // first row of this warp's box
       const bool tma_out = cnt > 0 && wrow0 < nq && (!kVarlen || wrow0 + 31 < nq);
       const uint32_t box0 = dev::smem_u32(sm.q[t]) + (warp & 3) * 4096;
 #pragma unroll 1
@@ -676,7 +693,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         if (lane == 0) {
           for (int half = 0; half < 2; ++half)
             dev::tma_store_3d(&tm_o, box0 + half * kHalfBytes, half * 64,
-                              kVarlen ? q_base + wrow0 : wrow0, kVarlen ? h : bh);
+                              kVarlen ? q_base + wrow0 : wrow0, kVarlen ? hq : b * p.Hq + hq);
           dev::bulk_commit_group();
           dev::bulk_wait_group_read0();  // the buffer is free again before the CTA ends
         }
