@@ -7,6 +7,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -46,6 +47,53 @@ int cuda_status(cudaError_t e) {
 }
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// Work-unit counters of the persistent prefill kernels, one per stream that launches them: calls
+// on one stream run one after another and can share a counter, calls on different streams may
+// overlap and must not.  A counter is zero between launches (the last CTA of a launch to take
+// from it sets it back).  Past kCounterSlots streams on one device, a stream shares the counter
+// of an earlier one.
+constexpr int kCounterSlots = 1024;
+static __device__ unsigned int g_unit_counters[kCounterSlots];
+
+struct CounterTable {
+  unsigned int* base = nullptr;
+  cudaStream_t stream[kCounterSlots] = {};
+  int used = 0;
+};
+CounterTable g_counter_tables[kMaxDevices];
+
+// The counter of `st` on the current device.
+int unit_counter(cudaStream_t st, unsigned int** out) {
+  int dev = 0;
+  int rc = cuda_status(cudaGetDevice(&dev));
+  if (rc != ATTN_OK) return rc;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  CounterTable& tab = g_counter_tables[dev];
+  if (tab.base == nullptr) {
+    void* p = nullptr;
+    rc = cuda_status(cudaGetSymbolAddress(&p, g_unit_counters));
+    if (rc != ATTN_OK) return rc;
+    tab.base = static_cast<unsigned int*>(p);
+  }
+  int slot = -1;
+  for (int i = 0; i < tab.used; ++i)
+    if (tab.stream[i] == st) {
+      slot = i;
+      break;
+    }
+  if (slot < 0) {
+    if (tab.used < kCounterSlots) {
+      slot = tab.used++;
+      tab.stream[slot] = st;
+    } else {
+      slot = static_cast<int>(reinterpret_cast<uintptr_t>(st) % kCounterSlots);
+    }
+  }
+  *out = tab.base + slot;
+  return ATTN_OK;
+}
+
 // Looks up the current device once: compute capability 10.x and the SM count; raises the
 // dynamic shared memory limit of the tensor-core kernel on first use.
 int current_device(DeviceInfo** out) {
@@ -72,7 +120,7 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
         fwd::fwd_bf16_sm100_kernel<false, true>,  fwd::fwd_bf16_sm100_kernel<true, true>,
         fwd::fwd_fp8_sm100_kernel<false>,         fwd::fwd_fp8_sm100_kernel<true>};
@@ -81,7 +129,7 @@ int configure_fwd(DeviceInfo* info) {
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
       if (rc != ATTN_OK) return rc;
     }
-    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sparse_sm100_kernel<false>, fwd::fwd_bf16_sparse_sm100_kernel<true>};
     for (auto* kern : sparse_kernels) {
       const int rc = cuda_status(cudaFuncSetAttribute(kern,
@@ -229,9 +277,6 @@ int encode_map(CUtensorMap* map, const void* base, int rows, int heads, uint32_t
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
-
-// The output map of the prefill kernels: each warp stores its 32 rows of a tile as a box.
-constexpr uint32_t kOutBoxRows = 32;
 
 // 3-D tiled TMA map over [heads][rows][128] E4M3 codes (one byte each), read as boxes of the full
 // 128-byte row width x 128 rows x 1 head with the 128-byte swizzle.
@@ -465,13 +510,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
                              static_cast<size_t>(B) * Hq * Nq, d, st);
   const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
-  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
 
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -487,16 +531,18 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = sc.num_qblocks;
   p.head_pair = sc.head_pair;
+  p.units = static_cast<int>(sc.units);
+  if ((rc = unit_counter(st, &p.unit_counter)) != ATTN_OK) return rc;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = nullptr;
   p.cu_k = nullptr;
-  const dim3 grid(static_cast<unsigned>(sc.units));
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -521,12 +567,11 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse,
                              static_cast<size_t>(B) * Hq * Nq, d, st);
   const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
-  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -540,6 +585,8 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = sc.num_qblocks;
   p.head_pair = sc.head_pair;
+  p.units = static_cast<int>(sc.units);
+  if ((rc = unit_counter(st, &p.unit_counter)) != ATTN_OK) return rc;
   p.front_heavy = (mask_kind == ATTN_MASK_FULL || mask_kind == ATTN_MASK_LOCAL_GLOBAL) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -547,11 +594,11 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.mask_heads = mask_heads;
   p.mask_qtiles = mask_qtiles;
   p.mask_ktiles = mask_ktiles;
-  const dim3 grid(static_cast<unsigned>(sc.units));
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
   else
-    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -577,12 +624,11 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   if (total_k == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(total_q) * Hq, d, st);
   const FwdSchedule sc = fwd_schedule(num_seqs, Hq, Hkv, max_seqlen_q);
-  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
-      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK ||
-      encode_map_packed(&to, o, total_q, Hq, kOutBoxRows) != ATTN_OK)
+      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = num_seqs;
@@ -596,16 +642,18 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = sc.num_qblocks;
   p.head_pair = sc.head_pair;
+  p.units = static_cast<int>(sc.units);
+  if ((rc = unit_counter(st, &p.unit_counter)) != ATTN_OK) return rc;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.cu_q = cu_seqlens_q;
   p.cu_k = cu_seqlens_k;
-  const dim3 grid(static_cast<unsigned>(sc.units));
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -629,12 +677,11 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   if (Nk == 0)
     return launch_fill_empty(static_cast<__nv_bfloat16*>(o), lse, static_cast<size_t>(B) * Hq * Nq, d, st);
   const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
-  if (sc.units > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&to, o, Nq, B * Hq, kOutBoxRows) != ATTN_OK)
+      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -648,6 +695,8 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   if (p.c == 0.f) p.c = 1e-30f;
   p.num_qblocks = sc.num_qblocks;
   p.head_pair = sc.head_pair;
+  p.units = static_cast<int>(sc.units);
+  if ((rc = unit_counter(st, &p.unit_counter)) != ATTN_OK) return rc;
   p.front_heavy = (mask_kind == ATTN_MASK_LOCAL_GLOBAL && n_sink > 0) ? 1 : 0;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -656,11 +705,11 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.descale_q = descale_q;
   p.descale_k = descale_k;
   p.descale_v = descale_v;
-  const dim3 grid(static_cast<unsigned>(sc.units));
+  const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   else
-    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
+    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -10,14 +10,16 @@
 // Research" (learning-materials), section 2 (TMA and warp specialisation as in
 // FlashAttention-3, here re-expressed with tcgen05 and tensor memory).
 //
-// One CTA computes two 128-row query tiles Q0, Q1 that share every K/V tile: the same 128 rows
-// of two query heads of one kv head when the group size is even (both tiles then see exactly the
-// same keys, so every step feeds both), otherwise 256 consecutive rows of one query head.
+// A work unit is two 128-row query tiles Q0, Q1 that share every K/V tile: the same 128 rows of
+// two query heads of one kv head when the group size is even (both tiles then see exactly the
+// same keys, so every step feeds both), otherwise 256 consecutive rows of one query head.  The
+// grid is persistent (one CTA per SM, each walking units in order from a shared counter).
 // Warp roles (12 warps = 3 warpgroups, 384 threads):
 //   warps 0-3   softmax + epilogue for Q0 (thread t owns row t, TMEM lanes 0-127)
 //   warps 4-7   softmax + epilogue for Q1
 //   warp 8      TMEM allocation and the single-thread tcgen05.mma issuer
-//   warp 9      TMA producer (Q once, then K_j and V_j through two 2-stage rings)
+//   warp 9      unit fetch and decode (block-sparse: the unit's step list), TMA producer (Q once
+//               per unit, then K_j and V_j through two 2-stage rings)
 //   warps 10-11 idle (they complete the third warpgroup)
 // Registers: launched at kRegsLaunch per thread; the two softmax warpgroups then raise their
 // limit to kRegsSoftmax (a whole 128-column score row lives in registers) and the third
@@ -86,6 +88,9 @@ struct Params {
   // 1: a CTA takes rows [128 qb, 128 qb + 128) of query heads 2i and 2i + 1 (G even, so both
   // read kv head 2i / G); 0: rows [256 qb, 256 qb + 256) of one query head
   int head_pair;
+  int units;                  // work units (query blocks x head groups x batch rows)
+  unsigned int* unit_counter; // zero at launch; the CTAs take units from it in order and the
+                              // last taker sets it back to zero
   __nv_bfloat16* o;
   float* lse;
   // E4M3 operands only: per (b, head) factors that turn the codes into values
@@ -99,30 +104,51 @@ struct Params {
   int mask_qtiles, mask_ktiles;  // ceil(Nq / 128), ceil(Nk / 128)
 };
 
+// One work unit: the two query tiles of a CTA-sized block and the key tiles they visit.
+// Decoded once by the producer warp and handed to the other roles through shared memory.
+struct Unit {
+  int valid;             // 0: the work is exhausted and the reader leaves
+  int b, h;              // batch row (sequence in variable-length mode), first query head
+  int bkv;               // row block of K/V in the dense [B * Hkv] layout
+  int r0;                // first query row of the block (inside its sequence)
+  int q_base, k_base;    // first packed row of the sequence (variable-length mode)
+  int nq;                // query rows of the sequence
+  int off;               // keys - queries of the sequence (key position of row i = i + off)
+  int nk;                // steps: key tiles the unit visits
+  int s_total;           // S products of the unit (steps summed over the query tiles)
+  MaskSpec mask;         // mask.Nk is the sequence's key count in variable-length mode
+  TileRange tr, trt[2];  // key tiles of the unit and of each query tile
+};
+
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
   uint8_t k[2][kTileBytes];
   uint8_t v[2][kTileBytes];
-  uint64_t bar_q;
+  uint64_t bar_q, bar_qempty;
   uint64_t bar_kfull[2], bar_kempty[2], bar_vfull[2], bar_vempty[2];
   uint64_t bar_s[2], bar_p[2], bar_o[2], bar_drain;
+  uint64_t bar_unit_full[2], bar_unit_empty[2];
+  Unit unit[2];
   uint32_t tmem_base;
   int abort;
 };
 
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base to 1024 B
 
-// Block-sparse CTAs list the key tiles they visit (selected for one of their two query tiles
-// and admitted by the base mask) right after Smem: tile index and, per entry, which query tiles
-// (bit t) take part.
+// Block-sparse units list the key tiles they visit (selected for one of their two query tiles
+// and admitted by the base mask) right after Smem, one list per unit slot: tile index and, per
+// entry, which query tiles (bit t) take part.
 constexpr int kMaxSparseTiles = 4096;  // key tiles per row of the layout (Nk <= 524288)
 struct SparseList {
   uint16_t tile[kMaxSparseTiles];
   uint8_t bits[kMaxSparseTiles];
   int count;
 };
-constexpr size_t kSmemBytesSparse = sizeof(Smem) + sizeof(SparseList) + 1024;
+constexpr size_t kSmemBytesSparse = sizeof(Smem) + 2 * sizeof(SparseList) + 1024;
 static_assert(kSmemBytesSparse <= 227 * 1024, "shared memory of a block-sparse CTA");
+
+// The readers of a unit slot: the 8 softmax warps and the MMA thread.
+constexpr uint32_t kUnitReaders = 9;
 
 // Is every (row, key) of the 128x128 block of query tile rows [P0, P0+127] x keys of tile kt
 // visible?  Conservative (uses all 128 rows even past Nq).
@@ -132,6 +158,53 @@ __device__ __forceinline__ bool tile_is_full(const MaskSpec& m, int P0, int kt) 
 
 __device__ __forceinline__ float neg_inf() { return __int_as_float(0xff800000); }
 __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); }
+
+// Work unit `unit` (0 <= unit < units): heaviest query blocks first, the G heads of a kv head
+// adjacent.  Returns false for a block wholly past its sequence (variable-length mode).
+template <bool kVarlen>
+__device__ __forceinline__ bool decode_unit(const Params& p, int unit, Unit& u) {
+  const bool pair = p.head_pair != 0;
+  const int heads_cta = pair ? 2 : 1;            // query heads of one unit
+  const int rows_cta = pair ? kBM : kRowsPerCta;  // query rows of one unit (per head)
+  const int groups = p.Hq / heads_cta;           // units of one query block per batch row
+  const int nbh = p.B * groups;
+  const int qb = p.front_heavy ? unit / nbh : p.num_qblocks - 1 - unit / nbh;
+  u.b = (unit % nbh) / groups;
+  u.h = (unit % nbh) % groups * heads_cta;
+  u.bkv = u.b * p.Hkv + u.h / p.G;
+  u.r0 = qb * rows_cta;
+  u.q_base = 0;
+  u.k_base = 0;
+  u.nq = p.Nq;
+  int nkeys = p.Nk;
+  u.mask = p.mask;
+  if (kVarlen) {
+    u.q_base = __ldg(p.cu_q + u.b);
+    u.k_base = __ldg(p.cu_k + u.b);
+    // rows are clamped to the packed tensors, so inconsistent offsets cannot reach past them
+    u.nq = u.q_base < 0 ? 0 : max(0, min(__ldg(p.cu_q + u.b + 1), p.Nq) - u.q_base);
+    nkeys = u.k_base < 0 ? 0 : max(0, min(__ldg(p.cu_k + u.b + 1), p.Nk) - u.k_base);
+    u.mask.Nk = nkeys;
+    if (u.r0 >= u.nq) return false;  // this sequence is shorter
+  }
+  u.off = nkeys - u.nq;
+  const int last_row = min(u.r0 + rows_cta, u.nq) - 1;
+  // key tiles of the whole unit (what the producer loads, in this order) ...
+  u.tr = key_tiles(u.mask, u.r0 + u.off, last_row + u.off, kBN);
+  // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
+  for (int t = 0; t < 2; ++t) {
+    const int lo_row = pair ? u.r0 : u.r0 + t * kBM, hi_row = min(lo_row + kBM, u.nq) - 1;
+    u.trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
+                               : key_tiles(u.mask, lo_row + u.off, hi_row + u.off, kBN);
+  }
+  u.nk = u.tr.count();
+  return true;
+}
+
+// does a query tile with key-tile range r take part in the step whose key tile is u?
+__device__ __forceinline__ bool in_range(const TileRange& r, int u) {
+  return u < r.ns || (u >= r.lo && u <= r.hi);
+}
 
 // kNeg: the scale is negative, so the largest scaled score comes from the smallest raw score.
 // kVarlen: packed variable-length sequences ("What Lost, and Why", the sequence-packing note:
@@ -143,10 +216,18 @@ __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); 
 // kSparse: a block-sparse layout (Params::block_mask) further restricts the key tiles of each
 // query tile ("Quadratic Complexity Bottleneck", sparse attention patterns: attention within and
 // between selected blocks); dense bf16 tensors only.
+//
+// The grid is persistent: each CTA takes units from p.unit_counter in unit order (heaviest
+// first) until they run out.  Every role walks the same unit sequence; the barrier phases, the
+// K/V ring position and the per-tile step counts run on across units, so a step is the same
+// whether it opens a unit or not.  The producer publishes each unit in one of two slots
+// (bar_unit_full) and reuses a slot once its readers released it (bar_unit_empty); it loads the
+// next unit's Q as soon as the MMA thread has issued the current unit's last S (bar_qempty), so
+// the next unit's first S products follow the current unit's last P V while the softmax warps
+// write the current unit's output.
 template <bool kNeg, bool kVarlen, bool kFp8, bool kSparse>
 __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                          const CUtensorMap& tm_v, const CUtensorMap& tm_o,
-                                          const Params& p) {
+                                          const CUtensorMap& tm_v, const Params& p) {
   static_assert(!kSparse || (!kVarlen && !kFp8), "block-sparse layouts take dense bf16 tensors");
   constexpr int kHalves = kFp8 ? 1 : 2;                          // TMA boxes per tile
   constexpr uint32_t kTile = kFp8 ? kTileBytes / 2 : kTileBytes;  // bytes of one tile
@@ -154,96 +235,23 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
+  SparseList* lists = reinterpret_cast<SparseList*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(Smem));
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-
-  // ---- work unit: heaviest query blocks first, the G heads of a kv head adjacent ----
   const bool pair = p.head_pair != 0;
-  const int heads_cta = pair ? 2 : 1;            // query heads of one CTA
-  const int rows_cta = pair ? kBM : kRowsPerCta;  // query rows of one CTA (per head)
-  const int nbh = p.B * (p.Hq / heads_cta);
-  const int unit = blockIdx.x;
-  const int qb = p.front_heavy ? unit / nbh : p.num_qblocks - 1 - unit / nbh;
-  const int b = (unit % nbh) / (p.Hq / heads_cta);
-  const int h = (unit % nbh) % (p.Hq / heads_cta) * heads_cta;  // (first) query head
-  const int bkv = b * p.Hkv + h / p.G;
-  const int r0 = qb * rows_cta;
-  // query tile t: its first row and its query head
-  auto tile_row0 = [&](int t) { return pair ? r0 : r0 + t * kBM; };
-  auto tile_head = [&](int t) { return pair ? h + t : h; };
-  // rows of this (sequence, head): q_base / k_base = first packed row, nq / nkeys = lengths
-  int q_base = 0, k_base = 0, nq = p.Nq, nkeys = p.Nk;
-  MaskSpec mask = p.mask;
-  if (kVarlen) {
-    q_base = __ldg(p.cu_q + b);
-    k_base = __ldg(p.cu_k + b);
-    // rows are clamped to the packed tensors, so inconsistent offsets cannot reach past them
-    nq = q_base < 0 ? 0 : max(0, min(__ldg(p.cu_q + b + 1), p.Nq) - q_base);
-    nkeys = k_base < 0 ? 0 : max(0, min(__ldg(p.cu_k + b + 1), p.Nk) - k_base);
-    mask.Nk = nkeys;
-    if (r0 >= nq) return;  // the whole CTA leaves together: this sequence is shorter
-  }
-  const int off = nkeys - nq;
-  const int last_row = min(r0 + rows_cta, nq) - 1;
-  // key tiles of the whole CTA (what the producer loads, in this order) ...
-  const TileRange tr = key_tiles(mask, r0 + off, last_row + off, kBN);
-  const int nk_range = tr.count();
-  // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
-  TileRange trt[2];
-  for (int t = 0; t < 2; ++t) {
-    const int lo_row = tile_row0(t), hi_row = min(lo_row + kBM, nq) - 1;
-    trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
-                             : key_tiles(mask, lo_row + off, hi_row + off, kBN);
-  }
-  // does a query tile with key-tile range r take part in step j (key tile tr.tile(j))?
-  auto in_range = [&](const TileRange& r, int j) {
-    const int u = tr.tile(j);
-    return u < r.ns || (u >= r.lo && u <= r.hi);
-  };
-  SparseList& sp = *reinterpret_cast<SparseList*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(Smem));
-  if (kSparse && warp == 0) {
-    // the steps of a block-sparse CTA: the range's key tiles selected for query tile 0 or 1,
-    // compacted in range order by one warp (ballot + prefix count)
-    // layout row of query tile t (read only if the tile has rows)
-    auto layout_row = [&](int t) {
-      const int hm = p.mask_heads == 1 ? 0 : tile_head(t);
-      return p.block_mask +
-             (static_cast<size_t>(hm) * p.mask_qtiles + tile_row0(t) / kBM) * p.mask_ktiles;
-    };
-    const uint8_t* row0 = layout_row(0);
-    const uint8_t* row1 = layout_row(1);
-    int base = 0;
-    for (int j0 = 0; j0 < nk_range; j0 += 32) {
-      const int j = j0 + lane;
-      uint32_t bits = 0u;
-      int kt = 0;
-      if (j < nk_range) {
-        kt = tr.tile(j);
-        const bool t0 = in_range(trt[0], j) && __ldg(row0 + kt) != 0;
-        const bool t1 = in_range(trt[1], j) && __ldg(row1 + kt) != 0;
-        bits = (t0 ? 1u : 0u) | (t1 ? 2u : 0u);
-      }
-      const uint32_t sel = __ballot_sync(0xffffffffu, bits != 0u);
-      if (bits != 0u) {
-        const int pos = base + __popc(sel & ((1u << lane) - 1u));
-        sp.tile[pos] = static_cast<uint16_t>(kt);
-        sp.bits[pos] = static_cast<uint8_t>(bits);
-      }
-      base += __popc(sel);
-    }
-    if (lane == 0) sp.count = base;
-  }
+  // query tile t of unit u: its first row and its query head
+  auto tile_row0 = [&](const Unit& u, int t) { return pair ? u.r0 : u.r0 + t * kBM; };
+  auto tile_head = [&](const Unit& u, int t) { return pair ? u.h + t : u.h; };
   // key tile of step j, and whether query tile t takes part in it
-  auto step_tile = [&](int j) { return kSparse ? static_cast<int>(sp.tile[j]) : tr.tile(j); };
-  auto takes_part = [&](int t, int j) {
-    if (kSparse) return ((sp.bits[j] >> t) & 1u) != 0u;
-    return in_range(t ? trt[1] : trt[0], j);
+  auto step_tile = [&](const Unit& u, const SparseList& sl, int j) {
+    return kSparse ? static_cast<int>(sl.tile[j]) : u.tr.tile(j);
   };
 
   // ---- set-up ----
   if (tid == 0) {
     dev::mbar_init(dev::smem_u32(&sm.bar_q), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_qempty), 1);
     for (int s = 0; s < 2; ++s) {
       dev::mbar_init(dev::smem_u32(&sm.bar_kfull[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_kempty[s]), 1);
@@ -252,6 +260,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       dev::mbar_init(dev::smem_u32(&sm.bar_s[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kBM);
       dev::mbar_init(dev::smem_u32(&sm.bar_o[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_full[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_empty[s]), kUnitReaders);
     }
     dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
@@ -261,7 +271,6 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     dev::tma_prefetch_desc(&tm_q);
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
-    dev::tma_prefetch_desc(&tm_o);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -272,57 +281,153 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   dev::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
-  const int nk = kSparse ? sp.count : nk_range;  // steps of the CTA
   if (warp >= 8) {
     // ========== third warpgroup: TMA producer, MMA issuer, two idle warps ==========
     dev::regs_decrease<kRegsOther>();
   if (warp == kLoadWarp) {
-    // =============================== TMA producer ===============================
-    if (lane == 0) {
-      int k_issued = 0, v_issued = 0;
-      bool q_issued = false;
-      if (nk > 0) {
-        const uint32_t bq = dev::smem_u32(&sm.bar_q);
-        dev::mbar_arrive_expect_tx(bq, 2 * kTile);
-        for (int t = 0; t < 2; ++t)
-          for (int half = 0; half < kHalves; ++half)
-            if (kVarlen)
-              dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                               q_base + tile_row0(t), tile_head(t));
-            else
-              dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
-                               tile_row0(t), b * p.Hq + tile_head(t));
-        q_issued = true;
-        for (int j = 0; j < nk; ++j) {
-          const int kt = step_tile(j);
-          const int s = j & 1;
-          const uint32_t ph = ((j >> 1) & 1) ^ 1;
-          if (!wait_bounded(dev::smem_u32(&sm.bar_kempty[s]), ph, abort)) break;
+    // ============================ unit fetch + TMA producer ============================
+    int published = 0;            // units handed to the other roles
+    int q_loads = 0;              // Q copies started (one per unit with steps)
+    int k_issued = 0, v_issued = 0;  // K / V copies started (the ring position runs on)
+    bool ok = true, exhausted = false;
+    while (ok) {
+      const int slot = published & 1;
+      // the slot's previous unit (two back) has been released by all its readers
+      if (published >= 2 &&
+          !wait_bounded(dev::smem_u32(&sm.bar_unit_empty[slot]), ((published - 2) >> 1) & 1, abort)) {
+        ok = false;
+        break;
+      }
+      // take units until one has rows; the last taker of the counter resets it for the next launch
+      Unit u;
+      u.valid = 0;
+      while (true) {
+        int f = 0;
+        if (lane == 0) f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+        f = __shfl_sync(0xffffffffu, f, 0);
+        if (f >= p.units) {
+          if (lane == 0 && f == p.units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+          exhausted = true;
+          break;
+        }
+        if (decode_unit<kVarlen>(p, f, u)) {
+          u.valid = 1;
+          break;
+        }
+      }
+      if (u.valid) {
+        if (kSparse) {
+          // the unit's steps: the range's key tiles selected for query tile 0 or 1, compacted in
+          // range order by the warp (ballot + prefix count)
+          SparseList& sl = lists[slot];
+          const uint8_t* row[2];
+          for (int t = 0; t < 2; ++t) {
+            const int hm = p.mask_heads == 1 ? 0 : tile_head(u, t);
+            row[t] = p.block_mask +
+                     (static_cast<size_t>(hm) * p.mask_qtiles + tile_row0(u, t) / kBM) * p.mask_ktiles;
+          }
+          int base = 0, parts = 0;
+          for (int j0 = 0; j0 < u.nk; j0 += 32) {
+            const int j = j0 + lane;
+            uint32_t bits = 0u;
+            int kt = 0;
+            if (j < u.nk) {
+              kt = u.tr.tile(j);
+              // a layout row is read only if its query tile has rows
+              const bool t0 = in_range(u.trt[0], kt) && __ldg(row[0] + kt) != 0;
+              const bool t1 = in_range(u.trt[1], kt) && __ldg(row[1] + kt) != 0;
+              bits = (t0 ? 1u : 0u) | (t1 ? 2u : 0u);
+            }
+            const uint32_t sel = __ballot_sync(0xffffffffu, bits != 0u);
+            if (bits != 0u) {
+              const int pos = base + __popc(sel & ((1u << lane) - 1u));
+              sl.tile[pos] = static_cast<uint16_t>(kt);
+              sl.bits[pos] = static_cast<uint8_t>(bits);
+            }
+            base += __popc(sel);
+            parts += __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(bits)));
+          }
+          u.nk = base;
+          u.s_total = parts;
+          if (lane == 0) sl.count = base;
+        } else {
+          int parts = 0;
+          for (int j = lane; j < u.nk; j += 32) {
+            const int kt = u.tr.tile(j);
+            parts += (in_range(u.trt[0], kt) ? 1 : 0) + (in_range(u.trt[1], kt) ? 1 : 0);
+          }
+          u.s_total = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(parts)));
+        }
+      }
+      if (lane == 0) sm.unit[slot] = u;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_full[slot]));
+      if (!u.valid) break;
+      ++published;
+      if (lane == 0 && u.nk > 0) {
+        const SparseList& sl = lists[slot];
+        // Q of this unit once the previous unit's last S products have read the Q buffers
+        if (q_loads > 0 && !wait_bounded(dev::smem_u32(&sm.bar_qempty), (q_loads - 1) & 1, abort)) {
+          ok = false;
+        } else {
+          const uint32_t bq = dev::smem_u32(&sm.bar_q);
+          dev::mbar_arrive_expect_tx(bq, 2 * kTile);
+          for (int t = 0; t < 2; ++t)
+            for (int half = 0; half < kHalves; ++half)
+              if (kVarlen)
+                dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
+                                 u.q_base + tile_row0(u, t), tile_head(u, t));
+              else
+                dev::tma_load_3d(dev::smem_u32(sm.q[t]) + half * kHalfBytes, &tm_q, bq, half * 64,
+                                 tile_row0(u, t), u.b * p.Hq + tile_head(u, t));
+          ++q_loads;
+        }
+        for (int j = 0; ok && j < u.nk; ++j) {
+          const int kt = step_tile(u, sl, j);
+          const int g = k_issued;  // ring position of this step
+          const int s = g & 1;
+          const uint32_t ph = ((g >> 1) & 1) ^ 1;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_kempty[s]), ph, abort)) { ok = false; break; }
           const uint32_t bk = dev::smem_u32(&sm.bar_kfull[s]);
           dev::mbar_arrive_expect_tx(bk, kTile);
           for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
-                               k_base + kt * kBN, h / p.G);
+                               u.k_base + kt * kBN, u.h / p.G);
             else
               dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bk, half * 64,
-                               kt * kBN, bkv);
+                               kt * kBN, u.bkv);
           ++k_issued;
-          if (!wait_bounded(dev::smem_u32(&sm.bar_vempty[s]), ph, abort)) break;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_vempty[s]), ph, abort)) { ok = false; break; }
           const uint32_t bv = dev::smem_u32(&sm.bar_vfull[s]);
           dev::mbar_arrive_expect_tx(bv, kTile);
           for (int half = 0; half < kHalves; ++half)
             if (kVarlen)
               dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
-                               k_base + kt * kBN, h / p.G);
+                               u.k_base + kt * kBN, u.h / p.G);
             else
               dev::tma_load_3d(dev::smem_u32(sm.v[s]) + half * kHalfBytes, &tm_v, bv, half * 64,
-                               kt * kBN, bkv);
+                               kt * kBN, u.bkv);
           ++v_issued;
         }
       }
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0) {
+      // a producer that gave up still takes its share of the counter, so that the last taker
+      // resets it
+      if (!exhausted) {
+        while (true) {
+          const int f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+          if (f >= p.units) {
+            if (f == p.units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+            break;
+          }
+        }
+      }
       // ---- drain: wait until every copy this thread started has landed ----
-      if (q_issued) wait_drain(dev::smem_u32(&sm.bar_q), 0);
+      if (q_loads > 0) wait_drain(dev::smem_u32(&sm.bar_q), (q_loads - 1) & 1);
       for (int s = 0; s < 2; ++s) {
         // the last load into stage s among loads 0..n-1 is u = largest u < n with u % 2 == s;
         // it completed phase (u / 2) of that stage's full barrier
@@ -334,30 +439,24 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     }
   } else if (warp == kMmaWarp) {
     // ============================ tcgen05.mma issuer =============================
-    if (lane == 0 && nk > 0) {
+    if (lane == 0) {
       // Q, K both K-major; P (TMEM), V MN-major
       constexpr uint32_t idesc_s = kFp8 ? dev::idesc_e4m3_f32(kBM, kBN, 0, 0)
                                         : dev::idesc_bf16_f32(kBM, kBN, 0, 0);
       constexpr uint32_t idesc_o = kFp8 ? dev::idesc_e4m3_f32(kBM, kD, 0, 1)
                                         : dev::idesc_bf16_f32(kBM, kD, 0, 1);
-      const uint32_t q_base[2] = {dev::smem_u32(sm.q[0]), dev::smem_u32(sm.q[1])};
-      const uint32_t tm_s[2] = {tmem + 0, tmem + 128};
-      const uint32_t tm_o[2] = {tmem + 256, tmem + 384};
-
-      // Descriptors are built once per buffer; a K-step only moves the start address, which is
-      // the low field of the descriptor (addresses stay far below its 256 KB range, so adding
-      // the offset >> 4 never carries out of the field).
-      const uint64_t dq[2] = {dev::smem_desc(q_base[0], 16, 1024, dev::kSwizzle128B),
-                              dev::smem_desc(q_base[1], 16, 1024, dev::kSwizzle128B)};
-      const uint64_t dk[2] = {dev::smem_desc(dev::smem_u32(sm.k[0]), 16, 1024, dev::kSwizzle128B),
-                              dev::smem_desc(dev::smem_u32(sm.k[1]), 16, 1024, dev::kSwizzle128B)};
-      const uint64_t dv[2] = {
-          dev::smem_desc(dev::smem_u32(sm.v[0]), kHalfBytes, 1024, dev::kSwizzle128B),
-          dev::smem_desc(dev::smem_u32(sm.v[1]), kHalfBytes, 1024, dev::kSwizzle128B)};
+      // Descriptors are built once; the second buffer of a pair and a K-step only move the start
+      // address, which is the low field of the descriptor (addresses stay far below its 256 KB
+      // range, so adding the offset >> 4 never carries out of the field).
+      constexpr uint32_t kBufStep = kTileBytes >> 4;  // q[1] - q[0], k[1] - k[0], v[1] - v[0]
+      const uint64_t dq0 = dev::smem_desc(dev::smem_u32(sm.q[0]), 16, 1024, dev::kSwizzle128B);
+      const uint64_t dk0 = dev::smem_desc(dev::smem_u32(sm.k[0]), 16, 1024, dev::kSwizzle128B);
+      const uint64_t dv0 =
+          dev::smem_desc(dev::smem_u32(sm.v[0]), kHalfBytes, 1024, dev::kSwizzle128B);
       auto issue_s = [&](int t, int s) {
-        const uint64_t a0 = t ? dq[1] : dq[0];
-        const uint64_t b0 = s ? dk[1] : dk[0];
-        const uint32_t d = t ? tm_s[1] : tm_s[0];
+        const uint64_t a0 = dq0 + static_cast<uint64_t>(t * kBufStep);
+        const uint64_t b0 = dk0 + static_cast<uint64_t>(s * kBufStep);
+        const uint32_t d = tmem + t * 128;
         if constexpr (kFp8) {
           // K = 32 one-byte elements (32 bytes) per MMA, all inside one 128-byte swizzle row
 #pragma unroll
@@ -372,9 +471,9 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         }
       };
       auto issue_pv = [&](int t, int s, bool acc) {
-        const uint64_t b0 = s ? dv[1] : dv[0];
-        const uint32_t d = t ? tm_o[1] : tm_o[0];
-        const uint32_t a = t ? tm_s[1] : tm_s[0];
+        const uint64_t b0 = dv0 + static_cast<uint64_t>(s * kBufStep);
+        const uint32_t d = tmem + 256 + t * 128;
+        const uint32_t a = tmem + t * 128;
         if constexpr (kFp8) {
           // 32 keys per MMA: 8 TMEM columns of packed E4M3 P, 32 rows (4 KB) of V
 #pragma unroll
@@ -389,93 +488,129 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         }
       };
 
-      // K_j lives in k[j & 1] (phase (j >> 1) & 1 of its barriers), V_j likewise in v[j & 1]
-      auto wait_k = [&](int j) {
-        return wait_bounded(dev::smem_u32(&sm.bar_kfull[j & 1]), (j >> 1) & 1, abort);
-      };
-      auto wait_v = [&](int j) {
-        return wait_bounded(dev::smem_u32(&sm.bar_vfull[j & 1]), (j >> 1) & 1, abort);
-      };
-      auto next_step = [&](int t, int j) {
-        int q = j + 1;
-        while (q < nk && !takes_part(t, q)) ++q;
-        return q;
-      };
-      // per tile: cur = the step whose S has been issued and whose P V is next; cnt = steps
-      // whose P V has been issued (the tile's barrier phases count only its own steps)
-      int cur0 = next_step(0, -1), cur1 = next_step(1, -1);
-      int cnt0 = 0, cnt1 = 0;
-      // K_j can be waited for at any time up to step j + 2: K_(j+2) reuses the slot of K_j,
-      // which is released at the end of step j - 1.  A block-sparse tile may skip many steps
-      // (the other tile takes them); the S of a step more than two ahead is then deferred
-      // (pend) and issued during the step before it, ahead of that K slot's release.  Dense
-      // masks never skip that far: a tile's steps are contiguous after its first, which is
-      // step 0 or 1.
-      int pend0 = -1, pend1 = -1;
-      auto issue_s_at = [&](int t, int j) {
-        if (!wait_k(j)) return false;
-        dev::tc_fence_after();
-        issue_s(t, j & 1);
-        dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
-        return true;
-      };
-      auto first_s = [&](int t, int cur) {
-        if (cur >= nk) return true;
-        if (kSparse && cur > 1) {
-          (t ? pend1 : pend0) = cur;
+      bool ok = true;
+      int taken = 0;        // units read from the slots
+      int q_waits = 0;      // Q copies consumed (units with steps)
+      int gbase = 0;        // ring position of the unit's first step
+      int ptot[2] = {0, 0}; // P barrier phases completed per tile, over all units
+      while (ok) {
+        const int slot = taken & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort))) break;
+        const Unit& us = sm.unit[slot];
+        const SparseList& sl = lists[slot];
+        ++taken;
+        if (!us.valid) break;
+        const int nk = us.nk, s_total = us.s_total;
+        const int ns = us.tr.ns, lo = us.tr.lo;  // step j -> key tile (dense)
+        const int ns0 = us.trt[0].ns, lo0 = us.trt[0].lo, hi0 = us.trt[0].hi;
+        const int ns1 = us.trt[1].ns, lo1 = us.trt[1].lo, hi1 = us.trt[1].hi;
+        auto takes = [&](int t, int j) {
+          if (kSparse) return ((sl.bits[j] >> t) & 1u) != 0u;
+          const int kt = j < ns ? j : lo + (j - ns);
+          return t ? (kt < ns1 || (kt >= lo1 && kt <= hi1)) : (kt < ns0 || (kt >= lo0 && kt <= hi0));
+        };
+        if (nk == 0) {
+          dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
+          continue;
+        }
+        // K_j lives in k[g & 1] (phase (g >> 1) & 1 of its barriers), g = gbase + j; V likewise
+        auto wait_k = [&](int j) {
+          const int g = gbase + j;
+          return wait_bounded(dev::smem_u32(&sm.bar_kfull[g & 1]), (g >> 1) & 1, abort);
+        };
+        auto wait_v = [&](int j) {
+          const int g = gbase + j;
+          return wait_bounded(dev::smem_u32(&sm.bar_vfull[g & 1]), (g >> 1) & 1, abort);
+        };
+        auto next_step = [&](int t, int j) {
+          int q = j + 1;
+          while (q < nk && !takes(t, q)) ++q;
+          return q;
+        };
+        // per tile: cur = the step whose S has been issued and whose P V is next; cnt = steps
+        // of this unit whose P V has been issued
+        int cur0 = next_step(0, -1), cur1 = next_step(1, -1);
+        int cnt0 = 0, cnt1 = 0;
+        int s_issued = 0;
+        // K_j can be waited for at any time up to step j + 2: K_(j+2) reuses the slot of K_j,
+        // which is released at the end of step j - 1.  A block-sparse tile may skip many steps
+        // (the other tile takes them); the S of a step more than two ahead is then deferred
+        // (pend) and issued during the step before it, ahead of that K slot's release.  Dense
+        // masks never skip that far: a tile's steps are contiguous after its first, which is
+        // step 0 or 1.
+        int pend0 = -1, pend1 = -1;
+        auto issue_s_at = [&](int t, int j) {
+          if (!wait_k(j)) return false;
+          dev::tc_fence_after();
+          issue_s(t, (gbase + j) & 1);
+          dev::umma_commit(dev::smem_u32(&sm.bar_s[t]));
+          // the unit's last S product: once it completes, the producer may refill the Q buffers
+          if (++s_issued == s_total) dev::umma_commit(dev::smem_u32(&sm.bar_qempty));
           return true;
-        }
-        return issue_s_at(t, cur);
-      };
-      // one step of tile t at step j: P V, then the S of its next step (or the final commit)
-      auto step = [&](int t, int j, int& cur, int& cnt) {
-        if (cur != j) return true;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_p[t]), cnt & 1, abort)) return false;
-        dev::tc_fence_after();
-        issue_pv(t, j & 1, cnt > 0);
-        ++cnt;
-        const int nxt = next_step(t, j);
-        if (nxt < nk) {
-          if (kSparse && nxt > j + 2) {
-            (t ? pend1 : pend0) = nxt;
-          } else if (!issue_s_at(t, nxt)) {
-            return false;
+        };
+        auto first_s = [&](int t, int cur) {
+          if (cur >= nk) return true;
+          if (kSparse && cur > 1) {
+            (t ? pend1 : pend0) = cur;
+            return true;
           }
-        } else {
-          dev::umma_commit(dev::smem_u32(&sm.bar_o[t]));
-        }
-        cur = nxt;
-        return true;
-      };
-      bool ok = wait_bounded(dev::smem_u32(&sm.bar_q), 0, abort);
-      // first S of each tile, earlier key tile first (the producer loads in step order)
-      if (ok) ok = cur0 <= cur1 ? (first_s(0, cur0) && first_s(1, cur1))
-                                : (first_s(1, cur1) && first_s(0, cur0));
-      // K_0 is released once every S that reads it is issued; a slot is always waited for
-      // before it is handed back, so a copy still landing is never overwritten
-      if (ok && nk > 0) {
-        if ((ok = wait_k(0))) dev::umma_commit(dev::smem_u32(&sm.bar_kempty[0]));
-      }
-      for (int j = 0; ok && j < nk; ++j) {
-        if (!(ok = wait_v(j))) break;
-        if (!(ok = step(0, j, cur0, cnt0) && step(1, j, cur1, cnt1))) break;
-        if constexpr (kSparse) {
-          // deferred S of step j + 1 (K_(j+1) is released below)
-          if (pend0 == j + 1) {
-            if (!(ok = issue_s_at(0, j + 1))) break;
-            pend0 = -1;
+          return issue_s_at(t, cur);
+        };
+        // one step of tile t at step j: P V, then the S of its next step (or the final commit)
+        auto step = [&](int t, int j, int& cur, int& cnt) {
+          if (cur != j) return true;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_p[t]), ptot[t] & 1, abort)) return false;
+          dev::tc_fence_after();
+          issue_pv(t, (gbase + j) & 1, cnt > 0);
+          ++cnt;
+          ++ptot[t];
+          const int nxt = next_step(t, j);
+          if (nxt < nk) {
+            if (kSparse && nxt > j + 2) {
+              (t ? pend1 : pend0) = nxt;
+            } else if (!issue_s_at(t, nxt)) {
+              return false;
+            }
+          } else {
+            dev::umma_commit(dev::smem_u32(&sm.bar_o[t]));
           }
-          if (pend1 == j + 1) {
-            if (!(ok = issue_s_at(1, j + 1))) break;
-            pend1 = -1;
+          cur = nxt;
+          return true;
+        };
+        ok = wait_bounded(dev::smem_u32(&sm.bar_q), q_waits & 1, abort);
+        ++q_waits;
+        // first S of each tile, earlier key tile first (the producer loads in step order)
+        if (ok) ok = cur0 <= cur1 ? (first_s(0, cur0) && first_s(1, cur1))
+                                  : (first_s(1, cur1) && first_s(0, cur0));
+        // K_0 is released once every S that reads it is issued; a slot is always waited for
+        // before it is handed back, so a copy still landing is never overwritten
+        if (ok) {
+          if ((ok = wait_k(0))) dev::umma_commit(dev::smem_u32(&sm.bar_kempty[gbase & 1]));
+        }
+        for (int j = 0; ok && j < nk; ++j) {
+          if (!(ok = wait_v(j))) break;
+          if (!(ok = step(0, j, cur0, cnt0) && step(1, j, cur1, cnt1))) break;
+          if constexpr (kSparse) {
+            // deferred S of step j + 1 (K_(j+1) is released below)
+            if (pend0 == j + 1) {
+              if (!(ok = issue_s_at(0, j + 1))) break;
+              pend0 = -1;
+            }
+            if (pend1 == j + 1) {
+              if (!(ok = issue_s_at(1, j + 1))) break;
+              pend1 = -1;
+            }
+          }
+          // every P V reading V_j and every S reading K_(j+1) is issued by now
+          dev::umma_commit(dev::smem_u32(&sm.bar_vempty[(gbase + j) & 1]));
+          if (j + 1 < nk) {
+            if (!(ok = wait_k(j + 1))) break;
+            dev::umma_commit(dev::smem_u32(&sm.bar_kempty[(gbase + j + 1) & 1]));
           }
         }
-        // every P V reading V_j and every S reading K_(j+1) is issued by now
-        dev::umma_commit(dev::smem_u32(&sm.bar_vempty[j & 1]));
-        if (j + 1 < nk) {
-          if (!(ok = wait_k(j + 1))) break;
-          dev::umma_commit(dev::smem_u32(&sm.bar_kempty[(j + 1) & 1]));
-        }
+        gbase += nk;
+        // every MMA of the unit is issued: the slot may be reused once the softmax warps are done
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
       }
       // drain: every MMA issued above has completed once this commit arrives
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
@@ -490,16 +625,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t t_s = tmem + lane_off + t * 128;
     const uint32_t t_o = tmem + lane_off + 256 + t * 128;
-    const int hq = tile_head(t);        // query head of this tile
-    const int P0 = tile_row0(t) + off;  // key position of the tile's first row
-    const int prow = P0 + row;          // key position of this thread's row
-    // scores in log2 units: c = scale * log2(e), times the Q and K descale factors for E4M3
-    const float c =
-        kFp8 ? p.c * __ldg(p.descale_q + b * p.Hq + hq) * __ldg(p.descale_k + bkv) : p.c;
     const float masked = kNeg ? pos_inf() : neg_inf();
-    float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
-    float l = 0.f;            // running sum of exp2(s*c - m_ref)
-    bool ok = true;
     // O_t *= alpha (per row), in tensor memory; O_t is complete here (the commit for S_t(j)
     // covered PV_t(j-1)) and the next P V has not been issued
     auto rescale_o = [&](float alpha) {
@@ -513,197 +639,203 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         dev::tmem_st32(t_o + cc * 32, o);
       }
     };
-
-    int cnt = 0;  // steps this tile has processed
-    for (int j = 0; j < nk; ++j) {
-      if (!takes_part(t, j)) continue;
-      ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), cnt & 1, abort);
+    bool ok = true;
+    int taken = 0;  // units read from the slots
+    int stot = 0;   // S barrier phases completed for this tile, over all units
+    int otot = 0;   // O barrier phases completed for this tile, over all units
+    while (ok) {
+      const int slot = taken & 1;
+      ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      dev::tc_fence_after();
-      const int kt = step_tile(j);
-      const int key0 = kt * kBN;
+      const Unit& us = sm.unit[slot];
+      if (!us.valid) break;
+      ++taken;
+      const SparseList& sl = lists[slot];
+      const int nk = us.nk;
+      const int tr_ns = us.tr.ns, tr_lo = us.tr.lo;  // step j -> key tile (dense)
+      const TileRange trt = us.trt[t];
+      const MaskSpec mask = us.mask;
+      const int P0 = tile_row0(us, t) + us.off;  // key position of the tile's first row
+      const int prow = P0 + row;                 // key position of this thread's row
+      // scores in log2 units: c = scale * log2(e), times the Q and K descale factors for E4M3
+      const float c = kFp8 ? p.c * __ldg(p.descale_q + us.b * p.Hq + tile_head(us, t)) *
+                                 __ldg(p.descale_k + us.bkv)
+                           : p.c;
+      float m_ref = neg_inf();  // running max (log2 units) used as the exponent reference
+      float l = 0.f;            // running sum of exp2(s*c - m_ref)
+      int cnt = 0;              // steps this tile has processed in this unit
+      for (int j = 0; j < nk; ++j) {
+        const int kt = kSparse ? static_cast<int>(sl.tile[j]) : (j < tr_ns ? j : tr_lo + (j - tr_ns));
+        if (kSparse ? (((sl.bits[j] >> t) & 1u) == 0u) : !in_range(trt, kt)) continue;
+        ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), stot & 1, abort);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        dev::tc_fence_after();
+        const int key0 = kt * kBN;
 
-      // the whole 128-column score row of this thread, one wait
-      uint32_t r[128];
+        // the whole 128-column score row of this thread, one wait
+        uint32_t r[128];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) dev::tmem_ld32(t_s + cc * 32, r + cc * 32);
-      dev::tmem_wait_ld_regs(r);
+        for (int cc = 0; cc < 4; ++cc) dev::tmem_ld32(t_s + cc * 32, r + cc * 32);
+        dev::tmem_wait_ld_regs(r);
 
-      const bool full = tile_is_full(mask, P0, kt);
-      if (!full) {
-        // visible columns of this row inside the tile: (lo <= col <= hi) or col < sk,
-        // as a 128-bit set built with shifts, then one bit test and select per column (no
-        // per-column branches, whatever the compiler knows about hi, lo and sk)
-        int hi, lo, sk;
-        row_cols(mask, prow, key0, hi, lo, sk);
-        uint32_t vis[4];
+        const bool full = tile_is_full(mask, P0, kt);
+        if (!full) {
+          // visible columns of this row inside the tile: (lo <= col <= hi) or col < sk,
+          // as a 128-bit set built with shifts, then one bit test and select per column (no
+          // per-column branches, whatever the compiler knows about hi, lo and sk)
+          int hi, lo, sk;
+          row_cols(mask, prow, key0, hi, lo, sk);
+          uint32_t vis[4];
 #pragma unroll
-        for (int w = 0; w < 4; ++w)
-          vis[w] = row_bits(hi, lo, sk, w);
+          for (int w = 0; w < 4; ++w)
+            vis[w] = row_bits(hi, lo, sk, w);
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          r[e] = ((vis[e >> 5] >> (e & 31)) & 1u) ? r[e] : __float_as_uint(masked);
-      }
+          for (int e = 0; e < 128; ++e)
+            r[e] = ((vis[e >> 5] >> (e & 31)) & 1u) ? r[e] : __float_as_uint(masked);
+        }
 
-      // row max of the raw scores (min when the scale is negative): 3-input max tree
-      auto row_max = [&]() {
-        float a[8];
+        // row max of the raw scores (min when the scale is negative): 3-input max tree
+        auto row_max = [&]() {
+          float a[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r[i]);
+          for (int i = 0; i < 8; ++i) a[i] = __uint_as_float(r[i]);
 #pragma unroll
-        for (int e = 8; e < 120; e += 16) {
+          for (int e = 8; e < 120; e += 16) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              a[i] = kNeg ? dev::min3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]))
+                          : dev::max3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]));
+          }
+          // the loop folded columns 8..119 into a[]; fold 120..127, then reduce a[] to one value
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            a[i] = kNeg ? dev::min3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]))
-                        : dev::max3(a[i], __uint_as_float(r[e + i]), __uint_as_float(r[e + 8 + i]));
-        }
-        // the loop folded columns 8..119 into a[]; fold 120..127, then reduce a[] to one value
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          a[i] = kNeg ? fminf(a[i], __uint_as_float(r[120 + i])) : fmaxf(a[i], __uint_as_float(r[120 + i]));
-        const float mx =
-            kNeg ? dev::min3(dev::min3(a[0], a[1], a[2]), dev::min3(a[3], a[4], a[5]), fminf(a[6], a[7]))
-                 : dev::max3(dev::max3(a[0], a[1], a[2]), dev::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
-        return (mx == masked) ? neg_inf() : mx * c;  // in log2 units
-      };
+            a[i] = kNeg ? fminf(a[i], __uint_as_float(r[120 + i])) : fmaxf(a[i], __uint_as_float(r[120 + i]));
+          const float mx =
+              kNeg ? dev::min3(dev::min3(a[0], a[1], a[2]), dev::min3(a[3], a[4], a[5]), fminf(a[6], a[7]))
+                   : dev::max3(dev::max3(a[0], a[1], a[2]), dev::max3(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+          return (mx == masked) ? neg_inf() : mx * c;  // in log2 units
+        };
 
-      // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t (E4M3: four
-      // codes of kPScaleF8 * P per column over the first 32); the row sum accumulates in 8
-      // independent packed pairs
-      float2 acc[4];
-      auto weights = [&](float m_ref_now) {
-        const float m_use = (m_ref_now == neg_inf()) ? 0.f : m_ref_now;
+        // P = exp2(s*c - m_use) -> bf16 pairs over the first 64 columns of S_t (E4M3: four
+        // codes of kPScaleF8 * P per column over the first 32); the row sum accumulates in 8
+        // independent packed pairs
+        float2 acc[4];
+        auto weights = [&](float m_ref_now) {
+          const float m_use = (m_ref_now == neg_inf()) ? 0.f : m_ref_now;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
+          for (int i = 0; i < 4; ++i) acc[i] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if constexpr (kFp8) {
-            // the exponent carries log2(kPScaleF8), so the weights come out already scaled
-            // for the E4M3 product (the row sum takes the factor back out below)
-            const uint64_t c2 = dev::pack2(c, c);
-            const uint64_t nm2 = dev::pack2(kLog2PScaleF8 - m_use, kLog2PScaleF8 - m_use);
-            uint32_t pk[16];
+          for (int half = 0; half < 2; ++half) {
+            if constexpr (kFp8) {
+              // the exponent carries log2(kPScaleF8), so the weights come out already scaled
+              // for the E4M3 product (the row sum takes the factor back out below)
+              const uint64_t c2 = dev::pack2(c, c);
+              const uint64_t nm2 = dev::pack2(kLog2PScaleF8 - m_use, kLog2PScaleF8 - m_use);
+              uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 64; e += 4) {
-              const int col = half * 64 + e;
-              float2 pr[2];
+              for (int e = 0; e < 64; e += 4) {
+                const int col = half * 64 + e;
+                float2 pr[2];
 #pragma unroll
-              for (int h2 = 0; h2 < 2; ++h2) {
-                const int cc2 = col + 2 * h2;
-                const float2 xx = dev::unpack2(dev::fma2(
-                    dev::pack2(__uint_as_float(r[cc2]), __uint_as_float(r[cc2 + 1])), c2, nm2));
-                pr[h2] = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+                for (int h2 = 0; h2 < 2; ++h2) {
+                  const int cc2 = col + 2 * h2;
+                  const float2 xx = dev::unpack2(dev::fma2(
+                      dev::pack2(__uint_as_float(r[cc2]), __uint_as_float(r[cc2 + 1])), c2, nm2));
+                  pr[h2] = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+                }
+                acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr[0]);
+                acc[((e >> 1) + 1) & 3] = dev::add2(acc[((e >> 1) + 1) & 3], pr[1]);
+                pk[e >> 2] = dev::pack_e4m3x4(pr[0].x, pr[0].y, pr[1].x, pr[1].y);
               }
-              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr[0]);
-              acc[((e >> 1) + 1) & 3] = dev::add2(acc[((e >> 1) + 1) & 3], pr[1]);
-              pk[e >> 2] = dev::pack_e4m3x4(pr[0].x, pr[0].y, pr[1].x, pr[1].y);
-            }
-            dev::tmem_st16(t_s + half * 16, pk);
-          } else {
-            // s * c - m_use two at a time (packed fp32 FMA), 2^x on the multi-function unit
-            const uint64_t c2 = dev::pack2(c, c), nm2 = dev::pack2(-m_use, -m_use);
-            uint32_t pk[32];
+              dev::tmem_st16(t_s + half * 16, pk);
+            } else {
+              // s * c - m_use two at a time (packed fp32 FMA), 2^x on the multi-function unit
+              const uint64_t c2 = dev::pack2(c, c), nm2 = dev::pack2(-m_use, -m_use);
+              uint32_t pk[32];
 #pragma unroll
-            for (int e = 0; e < 64; e += 2) {
-              const int col = half * 64 + e;
-              const float2 xx = dev::unpack2(dev::fma2(
-                  dev::pack2(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), c2, nm2));
-              const float2 pr = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
-              acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr);
-              pk[e >> 1] = dev::pack_bf16x2(pr.x, pr.y);
+              for (int e = 0; e < 64; e += 2) {
+                const int col = half * 64 + e;
+                const float2 xx = dev::unpack2(dev::fma2(
+                    dev::pack2(__uint_as_float(r[col]), __uint_as_float(r[col + 1])), c2, nm2));
+                const float2 pr = make_float2(dev::ex2_approx(xx.x), dev::ex2_approx(xx.y));
+                acc[(e >> 1) & 3] = dev::add2(acc[(e >> 1) & 3], pr);
+                pk[e >> 1] = dev::pack_bf16x2(pr.x, pr.y);
+              }
+              dev::tmem_st32(t_s + half * 32, pk);
             }
-            dev::tmem_st32(t_s + half * 32, pk);
           }
+        };
+
+        const float tmax = row_max();
+        const float m_new = fmaxf(m_ref, tmax);
+        float alpha = 1.f;
+        if (m_new > m_ref + kThreshold) {
+          alpha = dev::ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
+          m_ref = m_new;
         }
-      };
-
-      const float tmax = row_max();
-      const float m_new = fmaxf(m_ref, tmax);
-      float alpha = 1.f;
-      if (m_new > m_ref + kThreshold) {
-        alpha = dev::ex2_approx(m_ref - m_new);  // 0 when m_ref = -inf
-        m_ref = m_new;
+        l *= alpha;
+        if (cnt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o(alpha);
+        weights(m_ref);
+        acc[0] = dev::add2(acc[0], acc[1]);
+        acc[2] = dev::add2(acc[2], acc[3]);
+        acc[0] = dev::add2(acc[0], acc[2]);
+        l += kFp8 ? (acc[0].x + acc[0].y) * (1.f / kPScaleF8) : acc[0].x + acc[0].y;
+        dev::tmem_wait_st();
+        dev::tc_fence_before();
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));
+        ++cnt;
+        ++stot;
       }
-      l *= alpha;
-      if (cnt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) rescale_o(alpha);
-      weights(m_ref);
-      acc[0] = dev::add2(acc[0], acc[1]);
-      acc[2] = dev::add2(acc[2], acc[3]);
-      acc[0] = dev::add2(acc[0], acc[2]);
-      l += kFp8 ? (acc[0].x + acc[0].y) * (1.f / kPScaleF8) : acc[0].x + acc[0].y;
-      dev::tmem_wait_st();
-      dev::tc_fence_before();
-      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[t]));
-      ++cnt;
-    }
 
-    // ---- epilogue: O = O / l in bf16, LSE = ln(sum exp(scale * s)) ----
-    if (ok && cnt > 0) ok = wait_bounded(dev::smem_u32(&sm.bar_o[t]), 0, abort);
-    ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
-      dev::tc_fence_after();
-      const int grow = tile_row0(t) + row;
-      const bool valid = grow < nq;
-      // E4M3: undo the scale of P and apply the V descale factor
-      const float o_mul = kFp8 ? __ldg(p.descale_v + bkv) / kPScaleF8 : 1.f;
-      const float inv_l = l > 0.f ? o_mul / l : 0.f;
-      const size_t orow = kVarlen ? static_cast<size_t>(q_base + grow) * p.Hq + hq
-                                  : static_cast<size_t>(b * p.Hq + hq) * p.Nq + grow;
-      uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
-      // This warp's 32 rows leave as two 32-row x 64-column TMA boxes staged, 128-byte
-      // swizzled, in the tile's Q buffer, which no MMA reads any more (bar_o[t] covered every
-      // MMA of the tile).  A tile without steps never waited for its Q copy, and a box of
-      // packed sequences must not reach past its sequence: those rows use plain stores (a box
-      // wholly past the last row is not stored at all; a dense box is clipped at Nq).
-      const int wrow0 = tile_row0(t) + (warp & 3) * 32;  // first row of this warp's box
-      const bool tma_out = cnt > 0 && wrow0 < nq && (!kVarlen || wrow0 + 31 < nq);
-      const uint32_t box0 = dev::smem_u32(sm.q[t]) + (warp & 3) * 4096;
+      // ---- epilogue: O = O / l in bf16, LSE = ln(sum exp(scale * s)) ----
+      // O_t leaves TMEM before this warpgroup releases its next P (the next unit's first P V
+      // overwrites O_t), so the next unit's first S products may already be running.
+      if (ok && cnt > 0) ok = wait_bounded(dev::smem_u32(&sm.bar_o[t]), otot & 1, abort);
+      if (cnt > 0) ++otot;
+      ok = __all_sync(0xffffffffu, ok);
+      if (ok) {
+        dev::tc_fence_after();
+        // the unit's fields again from its slot (kept out of registers during the steps)
+        const int hq = tile_head(us, t), bkv = us.bkv;
+        const int grow = tile_row0(us, t) + row;
+        const bool valid = grow < us.nq;
+        // E4M3: undo the scale of P and apply the V descale factor
+        const float o_mul = kFp8 ? __ldg(p.descale_v + bkv) / kPScaleF8 : 1.f;
+        const float inv_l = l > 0.f ? o_mul / l : 0.f;
+        const size_t orow = kVarlen ? static_cast<size_t>(us.q_base + grow) * p.Hq + hq
+                                    : static_cast<size_t>(us.b * p.Hq + hq) * p.Nq + grow;
+        uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t o[32];
-        if (cnt > 0) {
-          dev::tmem_ld32(t_o + cc * 32, o);
-          dev::tmem_wait_ld_regs(o);
-        } else {
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          if (cnt > 0) {
+            dev::tmem_ld32(t_o + cc * 32, o);
+            dev::tmem_wait_ld_regs(o);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2)
-          pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
-                                        __uint_as_float(o[e + 1]) * inv_l);
-        if (tma_out) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4) {
-            const int c16 = cc * 4 + v4;  // 16-byte chunk of the 256-byte row
-            const uint32_t a = box0 + (c16 >> 3) * kHalfBytes + lane * 128 +
-                               (static_cast<uint32_t>((c16 & 7) ^ (lane & 7)) << 4);
-            dev::st_shared_v4(a, pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
           }
-        } else if (valid) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
+                                          __uint_as_float(o[e + 1]) * inv_l);
+          if (valid) {
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+        if (valid && p.lse != nullptr) {
+          const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
+          p.lse[orow] =
+              l > 0.f ? (m_use + log2f(l)) * 0.69314718055994531f : neg_inf();
         }
       }
-      if (tma_out) {
-        dev::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          for (int half = 0; half < 2; ++half)
-            dev::tma_store_3d(&tm_o, box0 + half * kHalfBytes, half * 64,
-                              kVarlen ? q_base + wrow0 : wrow0, kVarlen ? hq : b * p.Hq + hq);
-          dev::bulk_commit_group();
-          dev::bulk_wait_group_read0();  // the buffer is free again before the CTA ends
-        }
-        __syncwarp();
-      }
-      if (valid && p.lse != nullptr) {
-        const float m_use = (m_ref == neg_inf()) ? 0.f : m_ref;
-        p.lse[orow] =
-            l > 0.f ? (m_use + log2f(l)) * 0.69314718055994531f : neg_inf();
-      }
+      // this warp is done with the unit slot
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
     }
   }
 
@@ -721,9 +853,8 @@ template <bool kNeg, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v,
-                          const __grid_constant__ CUtensorMap tm_o, const Params p) {
-  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, tm_o, p);
+                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, p);
 }
 
 // bf16 Q, K, V (dense) under a block-sparse layout
@@ -731,9 +862,8 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sparse_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                  const __grid_constant__ CUtensorMap tm_k,
-                                 const __grid_constant__ CUtensorMap tm_v,
-                                 const __grid_constant__ CUtensorMap tm_o, const Params p) {
-  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, tm_o, p);
+                                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, p);
 }
 
 // E4M3 Q, K, V with per-(b, head) descale factors (dense)
@@ -741,9 +871,8 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_o, const Params p) {
-  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, tm_o, p);
+                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
+  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, p);
 }
 
 }  // namespace fwd
