@@ -92,6 +92,15 @@ ATTN_API const char *attn_status_string(int status);
 ATTN_API const char *attn_last_error_detail(void);
 
 /*
+ * The prefill calls (attn_fwd, attn_fwd_block_sparse, attn_fwd_varlen, attn_fwd_fp8) run a
+ * persistent grid whose CTAs take work from a 4-byte counter in device memory that the library
+ * owns: one counter per stream (up to 1024 streams per device; later streams share the counter
+ * of an earlier one, and two streams that share one must not run prefill calls at the same
+ * time).  Calls on one stream are ordered and share its counter.  The counter is back at zero
+ * when a call's kernel ends, also when it ended on ATTN_ERR_DEVICE_TIMEOUT.
+ */
+
+/*
  * attn_fwd - bf16 prefill / full forward.
  *   q, o   bf16 [B][Hq][Nq][d];  k, v  bf16 [B][Hkv][Nk][d];  lse fp32 [B][Hq][Nq] or NULL.
  *   B >= 0, Nq >= 0, Nk >= 0 (B = 0 or Nq = 0: nothing to do; Nk = 0: O = 0, LSE = -inf),

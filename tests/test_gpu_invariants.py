@@ -114,6 +114,37 @@ def test_deterministic():
     assert torch.equal(d1[0], d2[0]) and torch.equal(d1[1], d2[1])
 
 
+def test_prefill_on_concurrent_streams_matches_serial():
+    """The persistent prefill grids take work from one counter per stream: calls queued on two
+    streams at once (so their kernels may overlap) give the same bits as the calls run one
+    after another, and back-to-back calls on one stream see the counter back at zero."""
+    cases = [
+        (rnd(29, 0, (2, 8, 1500, 128)), rnd(29, 1, (2, 2, 1500, 128)), rnd(29, 2, (2, 2, 1500, 128)),
+         dict(mask_kind=CAUSAL)),
+        (rnd(30, 0, (1, 3, 2100, 128)), rnd(30, 1, (1, 1, 2100, 128)), rnd(30, 2, (1, 1, 2100, 128)),
+         dict(mask_kind=SLIDING, window=500, n_sink=2)),
+    ]
+    serial = []
+    for q, k, v, kw in cases:
+        serial.append(A.attn_fwd(q, k, v, **kw))
+        serial.append(A.attn_fwd(q, k, v, **kw))  # same stream, counter reused at once
+    for i in range(0, len(serial), 2):
+        assert torch.equal(serial[i][0], serial[i + 1][0])
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    outs = [[], []]
+    for rep in range(4):
+        for si, (q, k, v, kw) in enumerate(cases):
+            with torch.cuda.stream(streams[si]):
+                outs[si].append(A.attn_fwd(q, k, v, stream=streams[si], **kw))
+    torch.cuda.synchronize()
+    for si in range(2):
+        ref_o, ref_l = serial[2 * si]
+        for o, l in outs[si]:
+            assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    assert A.attn_get_device_error() == 0
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     assert A.attn_get_device_error() == 0
     A.attn_debug_timeout_probe(2_000_000)  # ~1 ms of SM clocks on an mbarrier nobody completes
