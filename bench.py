@@ -597,11 +597,12 @@ def end_to_end(wl, work, scale, unit, steps, flush, world, dist_on):
     """The metric through the public API from pinned host buffers: every step copies its inputs
     host -> device, runs the call and copies its results device -> host.
 
-    Pipelined (the reported value): the copies run on their own streams, two device copies of
+    Pipelined: the copies run on their own streams, two device copies of
     the inputs alternate, so the upload of step i + 1 overlaps the call and the download of step
     i; a call waits for its inputs and for the download of the previous results (the outputs
-    are single-buffered).  The serial figure (each step's upload, call and download one after
-    the other on one stream) is reported beside it.  An L2 flush precedes every call."""
+    are single-buffered).  Serial: each step's upload, call and download one after the other on
+    one stream.  The reported value is the faster of the two; both are kept in the record.  An
+    L2 flush precedes every call."""
     import torch
 
     host_in = [t.cpu().pin_memory() for t in wl.inputs]
@@ -663,10 +664,16 @@ def end_to_end(wl, work, scale, unit, steps, flush, world, dist_on):
     if dist_on:
         dist.barrier()
     ms = total / steps
-    return {"value": round(world * work / (ms * 1e-3) / scale, 3), "unit": unit,
+    # the faster of the two schedules is the end-to-end figure (for a small problem the
+    # pipelined loop's extra stream and event work on the host can cost more than it hides)
+    best = min(ms, serial_ms)
+    return {"value": round(world * work / (best * 1e-3) / scale, 3), "unit": unit,
             "h2d_bytes_per_step": h2d_bytes, "d2h_bytes_per_step": d2h_bytes,
-            "ms_per_step": round(ms, 4), "steps": steps,
+            "ms_per_step": round(best, 4), "steps": steps,
+            "schedule": "pipelined" if ms <= serial_ms else "serial",
             "pipelined": "upload of step i+1 overlaps the call and download of step i",
+            "pipelined_ms_per_step": round(ms, 4),
+            "pipelined_value": round(world * work / (ms * 1e-3) / scale, 3),
             "serial_ms_per_step": round(serial_ms, 4),
             "serial_value": round(world * work / (serial_ms * 1e-3) / scale, 3)}
 
