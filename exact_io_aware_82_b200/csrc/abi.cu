@@ -120,7 +120,7 @@ int current_device(DeviceInfo** out) {
 int configure_fwd(DeviceInfo* info) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!info->fwd_configured) {
-    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*kernels[6])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sm100_kernel<false, false>, fwd::fwd_bf16_sm100_kernel<true, false>,
         fwd::fwd_bf16_sm100_kernel<false, true>,  fwd::fwd_bf16_sm100_kernel<true, true>,
         fwd::fwd_fp8_sm100_kernel<false>,         fwd::fwd_fp8_sm100_kernel<true>};
@@ -129,7 +129,7 @@ int configure_fwd(DeviceInfo* info) {
           kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(fwd::kSmemBytes)));
       if (rc != ATTN_OK) return rc;
     }
-    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
+    void (*sparse_kernels[2])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, fwd::Params) = {
         fwd::fwd_bf16_sparse_sm100_kernel<false>, fwd::fwd_bf16_sparse_sm100_kernel<true>};
     for (auto* kern : sparse_kernels) {
       const int rc = cuda_status(cudaFuncSetAttribute(kern,
@@ -311,6 +311,23 @@ int encode_map_packed(CUtensorMap* map, const void* base, int rows, int heads,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+// TMA map of a prefill output (bf16, d = 128): dense [heads][rows][128] or packed
+// [rows][heads][128], written as boxes of 32 columns x 32 rows x 1 head staged with the 64-byte
+// swizzle (one box per softmax warp and column quarter).
+int encode_map_out(CUtensorMap* map, void* base, int rows, int heads, bool packed) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(fwd::kD), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(heads)};
+  const cuuint64_t strides[2] = {
+      packed ? static_cast<cuuint64_t>(heads) * fwd::kD * 2 : static_cast<cuuint64_t>(fwd::kD) * 2,
+      packed ? static_cast<cuuint64_t>(fwd::kD) * 2 : static_cast<cuuint64_t>(rows) * fwd::kD * 2};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estride[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estride,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
@@ -513,9 +530,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
 
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK || encode_map_out(&to, o, Nq, B * Hq, false) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -540,9 +557,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   p.cu_k = nullptr;
   const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -569,9 +586,9 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
   if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map(&tv, v, Nk, B * Hkv) != ATTN_OK || encode_map_out(&to, o, Nq, B * Hq, false) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -596,9 +613,9 @@ int attn_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, 
   p.mask_ktiles = mask_ktiles;
   const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sparse_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytesSparse, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -626,9 +643,10 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   const FwdSchedule sc = fwd_schedule(num_seqs, Hq, Hkv, max_seqlen_q);
   if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_packed(&tq, q, total_q, Hq) != ATTN_OK || encode_map_packed(&tk, k, total_k, Hkv) != ATTN_OK ||
-      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK)
+      encode_map_packed(&tv, v, total_k, Hkv) != ATTN_OK ||
+      encode_map_out(&to, o, total_q, Hq, true) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = num_seqs;
@@ -651,9 +669,9 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
   p.cu_k = cu_seqlens_k;
   const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<true, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_bf16_sm100_kernel<false, true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 
@@ -679,9 +697,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   const FwdSchedule sc = fwd_schedule(B, Hq, Hkv, Nq);
   if (sc.units > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   if ((rc = configure_fwd(info)) != ATTN_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map_e4m3(&tq, q, Nq, B * Hq) != ATTN_OK || encode_map_e4m3(&tk, k, Nk, B * Hkv) != ATTN_OK ||
-      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK)
+      encode_map_e4m3(&tv, v, Nk, B * Hkv) != ATTN_OK || encode_map_out(&to, o, Nq, B * Hq, false) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   fwd::Params p{};
   p.B = B;
@@ -707,9 +725,9 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
   p.descale_v = descale_v;
   const dim3 grid(static_cast<unsigned>(std::min<long long>(sc.units, info->num_sms)));
   if (scale < 0.f)
-    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<true><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   else
-    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, p);
+    fwd::fwd_fp8_sm100_kernel<false><<<grid, fwd::kThreads, fwd::kSmemBytes, st>>>(tq, tk, tv, to, p);
   return cuda_status(cudaGetLastError());
 }
 

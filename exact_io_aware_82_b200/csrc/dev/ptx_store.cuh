@@ -1,5 +1,5 @@
 // Shared-memory staging and tiled TMA stores (shared -> global), for epilogues that write a
-// tile with the 128-byte swizzle its tensor map declares.
+// tile in the swizzled layout its tensor map declares.
 #pragma once
 
 #include <cstdint>
@@ -38,6 +38,11 @@ __device__ __forceinline__ void bulk_commit_group() {
 // Wait until every bulk group of this thread has finished reading its shared-memory source.
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+// Wait until all but the most recent bulk group of this thread have finished reading.
+__device__ __forceinline__ void bulk_wait_group_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 
 }  // namespace dev

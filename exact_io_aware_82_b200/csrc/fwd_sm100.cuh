@@ -133,18 +133,30 @@ struct __align__(1024) Smem {
   int abort;
 };
 
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + slack to align the base to 1024 B
+// Output staging right after Smem: each softmax warp writes its 32 rows of O as boxes of 32
+// rows x 32 columns (64-byte swizzle, 2 KB), stored by TMA; two boxes per warp alternate (one for
+// block-sparse CTAs, whose step lists take the room).
+constexpr uint32_t kOBoxBytes = 32 * 32 * 2;
+constexpr int kOBoxesDense = 2, kOBoxesSparse = 1;
+constexpr size_t kOStageDense = 8 * kOBoxesDense * kOBoxBytes;
+constexpr size_t kOStageSparse = 8 * kOBoxesSparse * kOBoxBytes;
+
+constexpr size_t kSmemBytes = sizeof(Smem) + kOStageDense + 1024;  // + slack to align to 1024 B
 
 // Block-sparse units list the key tiles they visit (selected for one of their two query tiles
-// and admitted by the base mask) right after Smem, one list per unit slot: tile index and, per
-// entry, which query tiles (bit t) take part.
+// and admitted by the base mask) after the output staging, one list per unit slot: per entry the
+// key tile (low 14 bits) and which query tiles take part (bit 14 + t).
 constexpr int kMaxSparseTiles = 4096;  // key tiles per row of the layout (Nk <= 524288)
 struct SparseList {
-  uint16_t tile[kMaxSparseTiles];
-  uint8_t bits[kMaxSparseTiles];
+  uint16_t e[kMaxSparseTiles];
   int count;
 };
-constexpr size_t kSmemBytesSparse = sizeof(Smem) + 2 * sizeof(SparseList) + 1024;
+__device__ __forceinline__ int sparse_tile(const SparseList& sl, int j) { return sl.e[j] & 0x3fff; }
+__device__ __forceinline__ bool sparse_part(const SparseList& sl, int j, int t) {
+  return ((sl.e[j] >> (14 + t)) & 1u) != 0u;
+}
+constexpr size_t kSmemBytesSparse = sizeof(Smem) + kOStageSparse + 2 * sizeof(SparseList) + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory of a prefill CTA");
 static_assert(kSmemBytesSparse <= 227 * 1024, "shared memory of a block-sparse CTA");
 
 // The readers of a unit slot: the 8 softmax warps and the MMA thread.
@@ -227,7 +239,8 @@ __device__ __forceinline__ bool in_range(const TileRange& r, int u) {
 // write the current unit's output.
 template <bool kNeg, bool kVarlen, bool kFp8, bool kSparse>
 __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtensorMap& tm_k,
-                                          const CUtensorMap& tm_v, const Params& p) {
+                                          const CUtensorMap& tm_v, const CUtensorMap& tm_o,
+                                          const Params& p) {
   static_assert(!kSparse || (!kVarlen && !kFp8), "block-sparse layouts take dense bf16 tensors");
   constexpr int kHalves = kFp8 ? 1 : 2;                          // TMA boxes per tile
   constexpr uint32_t kTile = kFp8 ? kTileBytes / 2 : kTileBytes;  // bytes of one tile
@@ -235,7 +248,10 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                       ~uintptr_t(1023));
-  SparseList* lists = reinterpret_cast<SparseList*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(Smem));
+  constexpr int kOBoxes = kSparse ? kOBoxesSparse : kOBoxesDense;
+  const uint32_t ostage = dev::smem_u32(&sm) + static_cast<uint32_t>(sizeof(Smem));
+  SparseList* lists = reinterpret_cast<SparseList*>(reinterpret_cast<uint8_t*>(&sm) + sizeof(Smem) +
+                                                    kOStageSparse);
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -245,7 +261,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   auto tile_head = [&](const Unit& u, int t) { return pair ? u.h + t : u.h; };
   // key tile of step j, and whether query tile t takes part in it
   auto step_tile = [&](const Unit& u, const SparseList& sl, int j) {
-    return kSparse ? static_cast<int>(sl.tile[j]) : u.tr.tile(j);
+    return kSparse ? sparse_tile(sl, j) : u.tr.tile(j);
   };
 
   // ---- set-up ----
@@ -271,6 +287,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
     dev::tma_prefetch_desc(&tm_q);
     dev::tma_prefetch_desc(&tm_k);
     dev::tma_prefetch_desc(&tm_v);
+    dev::tma_prefetch_desc(&tm_o);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -341,8 +358,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
             const uint32_t sel = __ballot_sync(0xffffffffu, bits != 0u);
             if (bits != 0u) {
               const int pos = base + __popc(sel & ((1u << lane) - 1u));
-              sl.tile[pos] = static_cast<uint16_t>(kt);
-              sl.bits[pos] = static_cast<uint8_t>(bits);
+              sl.e[pos] = static_cast<uint16_t>(kt | (bits << 14));
             }
             base += __popc(sel);
             parts += __reduce_add_sync(0xffffffffu, static_cast<uint32_t>(__popc(bits)));
@@ -505,7 +521,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         const int ns0 = us.trt[0].ns, lo0 = us.trt[0].lo, hi0 = us.trt[0].hi;
         const int ns1 = us.trt[1].ns, lo1 = us.trt[1].lo, hi1 = us.trt[1].hi;
         auto takes = [&](int t, int j) {
-          if (kSparse) return ((sl.bits[j] >> t) & 1u) != 0u;
+          if (kSparse) return sparse_part(sl, j, t);
           const int kt = j < ns ? j : lo + (j - ns);
           return t ? (kt < ns1 || (kt >= lo1 && kt <= hi1)) : (kt < ns0 || (kt >= lo0 && kt <= hi0));
         };
@@ -665,8 +681,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       float l = 0.f;            // running sum of exp2(s*c - m_ref)
       int cnt = 0;              // steps this tile has processed in this unit
       for (int j = 0; j < nk; ++j) {
-        const int kt = kSparse ? static_cast<int>(sl.tile[j]) : (j < tr_ns ? j : tr_lo + (j - tr_ns));
-        if (kSparse ? (((sl.bits[j] >> t) & 1u) == 0u) : !in_range(trt, kt)) continue;
+        const int kt = kSparse ? sparse_tile(sl, j) : (j < tr_ns ? j : tr_lo + (j - tr_ns));
+        if (kSparse ? !sparse_part(sl, j, t) : !in_range(trt, kt)) continue;
         ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), stot & 1, abort);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         dev::tc_fence_after();
@@ -805,6 +821,13 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         const size_t orow = kVarlen ? static_cast<size_t>(us.q_base + grow) * p.Hq + hq
                                     : static_cast<size_t>(us.b * p.Hq + hq) * p.Nq + grow;
         uint4* dst = reinterpret_cast<uint4*>(p.o + orow * kD);
+        // This warp's 32 rows leave as four boxes of 32 rows x 32 columns, staged (64-byte
+        // swizzle: 16-byte chunk c of row r at chunk c ^ ((r >> 1) & 3)) in this warp's boxes and
+        // stored by TMA; a box is rewritten once the store before last from it has read it.  A
+        // box of packed sequences must not reach past its sequence: such rows use plain stores
+        // (a dense box is clipped at Nq by the tensor map).
+        const int wrow0 = tile_row0(us, t) + (warp & 3) * 32;  // first row of this warp's boxes
+        const bool tma_out = wrow0 < us.nq && (!kVarlen || wrow0 + 31 < us.nq);
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
           uint32_t o[32];
@@ -820,7 +843,25 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           for (int e = 0; e < 32; e += 2)
             pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(o[e]) * inv_l,
                                           __uint_as_float(o[e + 1]) * inv_l);
-          if (valid) {
+          if (tma_out) {
+            const uint32_t box = ostage + (warp * kOBoxes + (cc % kOBoxes)) * kOBoxBytes;
+            if (lane == 0) {
+              if (kOBoxes == 2) dev::bulk_wait_group_read1();
+              else dev::bulk_wait_group_read0();
+            }
+            __syncwarp();
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
+                                pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            dev::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              dev::tma_store_3d(&tm_o, box, cc * 32, kVarlen ? us.q_base + wrow0 : wrow0,
+                                kVarlen ? hq : us.b * p.Hq + hq);
+              dev::bulk_commit_group();
+            }
+          } else if (valid) {
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4)
               dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
@@ -840,6 +881,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   }
 
   // ---- teardown ----
+  if (warp < 8 && lane == 0) dev::bulk_wait_group_read0();  // the staged boxes have been read
   dev::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -853,8 +895,9 @@ template <bool kNeg, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, p);
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, kVarlen, false, false>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 // bf16 Q, K, V (dense) under a block-sparse layout
@@ -862,8 +905,9 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_bf16_sparse_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                                  const __grid_constant__ CUtensorMap tm_k,
-                                 const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, p);
+                                 const __grid_constant__ CUtensorMap tm_v,
+                                 const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, false, true>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 // E4M3 Q, K, V with per-(b, head) descale factors (dense)
@@ -871,8 +915,9 @@ template <bool kNeg>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_fp8_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const Params p) {
-  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, p);
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_o, const Params p) {
+  fwd_sm100<kNeg, false, true, false>(tm_q, tm_k, tm_v, tm_o, p);
 }
 
 }  // namespace fwd
