@@ -116,6 +116,8 @@ struct Unit {
   int off;               // keys - queries of the sequence (key position of row i = i + off)
   int nk;                // steps: key tiles the unit visits
   int s_total;           // S products of the unit (steps summed over the query tiles)
+  int tiles;             // bit t: query tile t has rows (without a block-sparse layout, a tile
+                         // with rows takes part in every step of the unit)
   MaskSpec mask;         // mask.Nk is the sequence's key count in variable-length mode
   TileRange tr, trt[2];  // key tiles of the unit and of each query tile
 };
@@ -173,7 +175,7 @@ __device__ __forceinline__ float pos_inf() { return __int_as_float(0x7f800000); 
 
 // Work unit `unit` (0 <= unit < units): heaviest query blocks first, the G heads of a kv head
 // adjacent.  Returns false for a block wholly past its sequence (variable-length mode).
-template <bool kVarlen>
+template <bool kVarlen, bool kSparse>
 __device__ __forceinline__ bool decode_unit(const Params& p, int unit, Unit& u) {
   const bool pair = p.head_pair != 0;
   const int heads_cta = pair ? 2 : 1;            // query heads of one unit
@@ -203,11 +205,18 @@ __device__ __forceinline__ bool decode_unit(const Params& p, int unit, Unit& u) 
   const int last_row = min(u.r0 + rows_cta, u.nq) - 1;
   // key tiles of the whole unit (what the producer loads, in this order) ...
   u.tr = key_tiles(u.mask, u.r0 + u.off, last_row + u.off, kBN);
-  // ... and of each query tile: a (query tile, key tile) pair with no visible entry is skipped
+  // ... and of each query tile.  Under a block-sparse layout a query tile visits only its own
+  // key tiles.  Otherwise a query tile with rows takes part in every step of the unit: its
+  // range differs from the unit's by at most a tile at either end (256 rows of one head under a
+  // causal or window mask), whose entries are all masked and add exact zeros, and keeping both
+  // tiles on every step lets them end together, so the next unit's products start at once
+  // instead of after one tile's extra step.
+  u.tiles = 0;
   for (int t = 0; t < 2; ++t) {
     const int lo_row = pair ? u.r0 : u.r0 + t * kBM, hi_row = min(lo_row + kBM, u.nq) - 1;
+    if (hi_row >= lo_row) u.tiles |= 1 << t;
     u.trt[t] = hi_row < lo_row ? TileRange{0, 0, -1}
-                               : key_tiles(u.mask, lo_row + u.off, hi_row + u.off, kBN);
+               : kSparse ? key_tiles(u.mask, lo_row + u.off, hi_row + u.off, kBN) : u.tr;
   }
   u.nk = u.tr.count();
   return true;
@@ -327,7 +336,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           exhausted = true;
           break;
         }
-        if (decode_unit<kVarlen>(p, f, u)) {
+        if (decode_unit<kVarlen, kSparse>(p, f, u)) {
           u.valid = 1;
           break;
         }
@@ -367,12 +376,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           u.s_total = parts;
           if (lane == 0) sl.count = base;
         } else {
-          int parts = 0;
-          for (int j = lane; j < u.nk; j += 32) {
-            const int kt = u.tr.tile(j);
-            parts += (in_range(u.trt[0], kt) ? 1 : 0) + (in_range(u.trt[1], kt) ? 1 : 0);
-          }
-          u.s_total = static_cast<int>(__reduce_add_sync(0xffffffffu, static_cast<uint32_t>(parts)));
+          u.s_total = u.nk * __popc(u.tiles);
         }
       }
       if (lane == 0) sm.unit[slot] = u;
@@ -516,14 +520,10 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         const SparseList& sl = lists[slot];
         ++taken;
         if (!us.valid) break;
-        const int nk = us.nk, s_total = us.s_total;
-        const int ns = us.tr.ns, lo = us.tr.lo;  // step j -> key tile (dense)
-        const int ns0 = us.trt[0].ns, lo0 = us.trt[0].lo, hi0 = us.trt[0].hi;
-        const int ns1 = us.trt[1].ns, lo1 = us.trt[1].lo, hi1 = us.trt[1].hi;
+        const int nk = us.nk, s_total = us.s_total, tiles = us.tiles;
         auto takes = [&](int t, int j) {
           if (kSparse) return sparse_part(sl, j, t);
-          const int kt = j < ns ? j : lo + (j - ns);
-          return t ? (kt < ns1 || (kt >= lo1 && kt <= hi1)) : (kt < ns0 || (kt >= lo0 && kt <= hi0));
+          return ((tiles >> t) & 1) != 0;
         };
         if (nk == 0) {
           dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
@@ -551,9 +551,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         // K_j can be waited for at any time up to step j + 2: K_(j+2) reuses the slot of K_j,
         // which is released at the end of step j - 1.  A block-sparse tile may skip many steps
         // (the other tile takes them); the S of a step more than two ahead is then deferred
-        // (pend) and issued during the step before it, ahead of that K slot's release.  Dense
-        // masks never skip that far: a tile's steps are contiguous after its first, which is
-        // step 0 or 1.
+        // (pend) and issued during the step before it, ahead of that K slot's release.  Without
+        // a layout a tile with rows takes every step.
         int pend0 = -1, pend1 = -1;
         auto issue_s_at = [&](int t, int j) {
           if (!wait_k(j)) return false;
@@ -669,7 +668,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       const SparseList& sl = lists[slot];
       const int nk = us.nk;
       const int tr_ns = us.tr.ns, tr_lo = us.tr.lo;  // step j -> key tile (dense)
-      const TileRange trt = us.trt[t];
+      const bool mine = ((us.tiles >> t) & 1) != 0;  // this tile has rows
       const MaskSpec mask = us.mask;
       const int P0 = tile_row0(us, t) + us.off;  // key position of the tile's first row
       const int prow = P0 + row;                 // key position of this thread's row
@@ -682,7 +681,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       int cnt = 0;              // steps this tile has processed in this unit
       for (int j = 0; j < nk; ++j) {
         const int kt = kSparse ? sparse_tile(sl, j) : (j < tr_ns ? j : tr_lo + (j - tr_ns));
-        if (kSparse ? !sparse_part(sl, j, t) : !in_range(trt, kt)) continue;
+        if (kSparse ? !sparse_part(sl, j, t) : !mine) continue;
         ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), stot & 1, abort);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         dev::tc_fence_after();
