@@ -108,21 +108,21 @@ MIN_TIMED_MS = 200.0
 # kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
     "full_b1_h1_n256_d64_f32": {"bytes": 260608, "src": "02e210e28044d0c4"},
-    "causal_b4_h16_n2048_d128": {"bytes": 136256000, "src": "db22c40767b52c14"},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 479916032, "src": "db22c40767b52c14"},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 698571520, "src": "db22c40767b52c14"},
-    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1303387888, "src": "db22c40767b52c14"},
-    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 771768064, "src": "db22c40767b52c14"},
-    "fp8_causal_b4_h16_n2048_d128": {"bytes": 54390528, "src": "db22c40767b52c14"},
-    "block_sparse_b1_h32_kv8_n32768_d128": {"bytes": 1000239104, "src": "db22c40767b52c14"},
+    "causal_b4_h16_n2048_d128": {"bytes": 151330048, "src": "e353e585ff2e02b6"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 474978304, "src": "e353e585ff2e02b6"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 692300544, "src": "e353e585ff2e02b6"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293218960, "src": "e353e585ff2e02b6"},
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 769709056, "src": "e353e585ff2e02b6"},
+    "fp8_causal_b4_h16_n2048_d128": {"bytes": 54126848, "src": "e353e585ff2e02b6"},
+    "block_sparse_b1_h32_kv8_n32768_d128": {"bytes": 912254208, "src": "e353e585ff2e02b6"},
     # the backward step's three kernels together (prep + dK/dV + dQ)
-    "bwd_causal_b4_h16_n2048_d128": {"bytes": 1037843968, "src": "0ea6bc652cc64f22"},
+    "bwd_causal_b4_h16_n2048_d128": {"bytes": 1038654976, "src": "7a4bdc98981f1408"},
     # a decode step's two kernels together (split + combine), captured on the 8-sequence
     # cases; the cache is read once per sequence, so the 64-sequence step moves 8x that
-    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1084994200, "src": "08a4fbcfc6e70524"},
-    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1084994200, "src": "08a4fbcfc6e70524"},
-    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1085063864, "src": "08a4fbcfc6e70524"},
-    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1085063864, "src": "08a4fbcfc6e70524"},
+    "decode_b64_h32_kv8_n32768_d128": {"bytes": 8 * 1084886016, "src": "1a9ec2fd52b8d638"},
+    "decode_b8_h32_kv8_n32768_d128": {"bytes": 1084886016, "src": "1a9ec2fd52b8d638"},
+    "paged_decode_b64_h32_kv8_n32768_p16_d128": {"bytes": 8 * 1085015520, "src": "1a9ec2fd52b8d638"},
+    "paged_decode_b8_h32_kv8_n32768_p16_d128": {"bytes": 1085015520, "src": "1a9ec2fd52b8d638"},
 }
 
 # the device sources each kernel family is compiled from (the launch code in abi.cu only sets
