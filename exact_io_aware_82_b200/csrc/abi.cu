@@ -900,7 +900,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   const int nqt = (Nq + bwd::kT - 1) / bwd::kT, nkb = (Nk + bwd::kT - 1) / bwd::kT;
   const long long units_q = static_cast<long long>((nqt + 1) / 2) * B * Hq;  // query-tile pairs
   const long long units_kv = static_cast<long long>(nkb) * B * Hkv;
-  if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   const MaskSpec mask = make_mask(mask_kind, window, n_sink, Nk);
   const BwdLayout L = bwd_layout(B, Hq, Nq, Nk, mask);
   if (static_cast<double>(B) * Hq * static_cast<double>(L.pairs) > 2147483647.0)
@@ -936,6 +936,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   p.ds_off = reinterpret_cast<int*>(dsum + static_cast<size_t>(B) * Hq * p.npad);
   p.ds = reinterpret_cast<__nv_bfloat16*>(static_cast<uint8_t*>(workspace) + L.ds_offset);
   p.ds_pairs = static_cast<long long>(L.pairs);
+  if ((rc = unit_counter(st, &p.unit_counter)) != ATTN_OK) return rc;
   // dS^T blocks as a 3-D tensor (queries, keys, block) for the dQ kernel's TMA loads
   CUtensorMap tds;
   {
@@ -972,8 +973,9 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
       dsum, Nq, p.npad, prow, mask, nkb, p.ds_off);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
-  bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(units_kv), bwd::kThreads, bwd::kSmemKVBytes, st>>>(
-      tq, tk, tv, tdo, tds_out, p);
+  // persistent: one CTA per SM walking the key-block units
+  bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(std::min<long long>(units_kv, info->num_sms)),
+                         bwd::kThreads, bwd::kSmemKVBytes, st>>>(tq, tk, tv, tdo, tds_out, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
       tds, tk, p);

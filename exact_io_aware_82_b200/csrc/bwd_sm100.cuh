@@ -12,7 +12,8 @@
 //
 // Three launches:
 //  1. bwd_prep_kernel: D_i and LSE_i * log2(e) per query row (memory-bound, one warp per row).
-//  2. bwd_dkdv_kernel: one CTA per (b, kv head, 128-key block).  It walks the query tiles that see
+//  2. bwd_dkdv_kernel: one unit per (b, kv head, 128-key block), taken by persistent CTAs (one
+//     per SM) from a counter, lowest key blocks first.  A unit walks the query tiles that see
 //     the block, for each of the G query heads of the group, and keeps dK and dV of its keys in
 //     tensor memory for the whole walk (no atomics; GQA sums in place).  Per step, four tcgen05
 //     MMAs (128 x 128 x 128, bf16 in, fp32 accumulate): S^T = K Q^T and dP^T = V dO^T into TMEM;
@@ -74,6 +75,7 @@ struct Params {
   __nv_bfloat16* ds;
   int* ds_off;         // [num_kblocks + 1], written by the prep kernel
   long long ds_pairs;  // ds_off[num_kblocks]: blocks per (b, query head)
+  unsigned int* unit_counter;  // zero at launch; the dK/dV CTAs take key-block units from it
 };
 
 // Query tiles of one key block: [s0, ns) (the global rows of the local + global mask, when
@@ -290,14 +292,48 @@ struct __align__(1024) SmemKV {
   uint8_t ds_stage[kRowThreads / 32][kDsBoxBytes];  // one box per row warp
   float lse2[2][kT];  // per stage: the query tile's LSE * log2(e) and D, copied with Q and dO
   float dsum[2][kT];
-  uint64_t bar_kv, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_free[2], bar_done;
-  uint64_t bar_drain[2];
+  uint64_t bar_kv, bar_kvempty, bar_qfull[2], bar_qempty[2], bar_s[2], bar_p[2], bar_free[2];
+  uint64_t bar_done, bar_drain[2];
+  uint64_t bar_unit_full[2], bar_unit_empty[2];
+  int unit[2];  // published key-block units (-1: no more)
   uint32_t tmem_base;
   int abort;
 };
 constexpr size_t kSmemKVBytes = sizeof(SmemKV) + 1024;
 static_assert(kSmemKVBytes <= 227 * 1024, "shared memory of the dK/dV kernel");
 
+// The readers of a unit slot: the two MMA threads and the 8 row warps.
+constexpr uint32_t kKVUnitReaders = 10;
+
+// Key block kb of (b, kv head hk) for unit u: lowest blocks first (under a causal mask they have
+// the most query tiles), the (b, kv head) pairs of one block adjacent.
+struct KVUnit {
+  int kb, bk, b, hk, c0, c1;
+  QueryTiles qr;
+  int nqt, nsteps;
+};
+__device__ __forceinline__ KVUnit kv_unit(const Params& p, int u) {
+  KVUnit r;
+  const int nbk = p.B * p.Hkv;
+  r.kb = u / nbk;
+  r.bk = u % nbk;
+  r.b = r.bk / p.Hkv;
+  r.hk = r.bk % p.Hkv;
+  r.c0 = r.kb * kT;
+  r.c1 = min(r.c0 + kT, p.Nk) - 1;
+  r.qr = query_tiles(p.mask, r.c0, r.c1, p.Nk - p.Nq, p.Nq);
+  r.nqt = r.qr.count();
+  r.nsteps = r.nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qr.tile(n % nqt)
+  return r;
+}
+
+// Persistent: one CTA per SM takes key-block units from p.unit_counter (the last taker sets it
+// back to zero).  The producer publishes each unit in one of two slots; the barrier phases, the
+// Q/dO stage ring and the sub-step count run on across units.  A unit's K and V are loaded once
+// the previous unit's last score products have completed (bar_kvempty), while the accumulating
+// products and the row warps finish that unit; its first accumulating product, which overwrites
+// dV and dK in TMEM, waits for the row warps' first weights of the unit, which they release only
+// after reading out the previous unit's dV and dK.
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                     const __grid_constant__ CUtensorMap tm_k,
@@ -308,22 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                           ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
-  // key block kb of (b, hk); lowest blocks first (they have the most query tiles under a
-  // causal mask)
-  const int nbk = p.B * p.Hkv;
-  const int kb = blockIdx.x / nbk;
-  const int bk = blockIdx.x % nbk;
-  const int b = bk / p.Hkv, hk = bk % p.Hkv;
-  const int c0 = kb * kT, c1 = min(c0 + kT, p.Nk) - 1;
   const int off = p.Nk - p.Nq;
-  const QueryTiles qr = query_tiles(p.mask, c0, c1, off, p.Nq);
-  const int nqt = qr.count();
-  const int nsteps = nqt * p.G;  // step n: query head hk*G + n / nqt, query tile qr.tile(n % nqt)
-  const int nsub = 2 * nsteps;
 
   if (tid == 0) {
     dev::mbar_init(dev::smem_u32(&sm.bar_kv), 1);
+    dev::mbar_init(dev::smem_u32(&sm.bar_kvempty), 1);
     for (int s = 0; s < 2; ++s) {
       dev::mbar_init(dev::smem_u32(&sm.bar_qfull[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_qempty[s]), 1);
@@ -331,6 +356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(dev::smem_u32(&sm.bar_p[s]), kRowThreads);
       dev::mbar_init(dev::smem_u32(&sm.bar_free[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_drain[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_full[s]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_empty[s]), kKVUnitReaders);
     }
     dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
     sm.abort = 0;
@@ -352,105 +379,170 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
+  const int units = p.num_kblocks * p.B * p.Hkv;
 
   if (warp == kLoadWarp) {
-    // ================================ TMA producer ================================
-    if (lane == 0 && nsteps > 0) {
-      const uint32_t bkv = dev::smem_u32(&sm.bar_kv);
-      dev::mbar_arrive_expect_tx(bkv, 2 * kTileBytes);
-      for (int half = 0; half < 2; ++half) {
-        dev::tma_load_3d(dev::smem_u32(sm.k) + half * kHalfBytes, &tm_k, bkv, half * 64, c0, bk);
-        dev::tma_load_3d(dev::smem_u32(sm.v) + half * kHalfBytes, &tm_v, bkv, half * 64, c0, bk);
-      }
-      int issued = 0;
-      for (int n = 0; n < nsteps; ++n) {
-        const int s = n & 1;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_qempty[s]), ((n >> 1) & 1) ^ 1, abort)) break;
-        const int hq = hk * p.G + n / nqt;
-        const int r0 = qr.tile(n % nqt) * kT;
-        const uint32_t bq = dev::smem_u32(&sm.bar_qfull[s]);
-        const size_t vrow = static_cast<size_t>(b * p.Hq + hq) * p.npad + r0;
-        dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes + 2 * kT * 4);
-        for (int half = 0; half < 2; ++half) {
-          dev::tma_load_3d(dev::smem_u32(sm.q[s]) + half * kHalfBytes, &tm_q, bq, half * 64, r0,
-                           b * p.Hq + hq);
-          dev::tma_load_3d(dev::smem_u32(sm.dout[s]) + half * kHalfBytes, &tm_do, bq, half * 64,
-                           r0, b * p.Hq + hq);
+    // ============================ unit fetch + TMA producer ============================
+    if (lane == 0) {
+      int published = 0, kv_loads = 0, issued = 0;
+      bool ok = true, exhausted = false;
+      while (ok) {
+        const int slot = published & 1;
+        if (published >= 2 && !wait_bounded(dev::smem_u32(&sm.bar_unit_empty[slot]),
+                                             ((published - 2) >> 1) & 1, abort)) {
+          ok = false;
+          break;
         }
-        bulk_load(dev::smem_u32(sm.lse2[s]), p.lse2 + vrow, kT * 4, bq);
-        bulk_load(dev::smem_u32(sm.dsum[s]), p.dsum + vrow, kT * 4, bq);
-        ++issued;
+        const int f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+        if (f >= units) {
+          if (f == units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+          exhausted = true;
+        }
+        sm.unit[slot] = exhausted ? -1 : f;
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_full[slot]));
+        if (exhausted) break;
+        ++published;
+        const KVUnit u = kv_unit(p, f);
+        if (u.nsteps == 0) continue;
+        // K and V once the previous unit's score products have read them for good
+        if (kv_loads > 0 &&
+            !wait_bounded(dev::smem_u32(&sm.bar_kvempty), (kv_loads - 1) & 1, abort)) {
+          ok = false;
+          break;
+        }
+        const uint32_t bkv = dev::smem_u32(&sm.bar_kv);
+        dev::mbar_arrive_expect_tx(bkv, 2 * kTileBytes);
+        for (int half = 0; half < 2; ++half) {
+          dev::tma_load_3d(dev::smem_u32(sm.k) + half * kHalfBytes, &tm_k, bkv, half * 64, u.c0, u.bk);
+          dev::tma_load_3d(dev::smem_u32(sm.v) + half * kHalfBytes, &tm_v, bkv, half * 64, u.c0, u.bk);
+        }
+        ++kv_loads;
+        for (int n = 0; n < u.nsteps; ++n) {
+          const int g = issued;  // position in the Q/dO stage ring
+          const int s = g & 1;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_qempty[s]), ((g >> 1) & 1) ^ 1, abort)) {
+            ok = false;
+            break;
+          }
+          const int hq = u.hk * p.G + n / u.nqt;
+          const int r0 = u.qr.tile(n % u.nqt) * kT;
+          const uint32_t bq = dev::smem_u32(&sm.bar_qfull[s]);
+          const size_t vrow = static_cast<size_t>(u.b * p.Hq + hq) * p.npad + r0;
+          dev::mbar_arrive_expect_tx(bq, 2 * kTileBytes + 2 * kT * 4);
+          for (int half = 0; half < 2; ++half) {
+            dev::tma_load_3d(dev::smem_u32(sm.q[s]) + half * kHalfBytes, &tm_q, bq, half * 64, r0,
+                             u.b * p.Hq + hq);
+            dev::tma_load_3d(dev::smem_u32(sm.dout[s]) + half * kHalfBytes, &tm_do, bq, half * 64,
+                             r0, u.b * p.Hq + hq);
+          }
+          bulk_load(dev::smem_u32(sm.lse2[s]), p.lse2 + vrow, kT * 4, bq);
+          bulk_load(dev::smem_u32(sm.dsum[s]), p.dsum + vrow, kT * 4, bq);
+          ++issued;
+        }
       }
-      wait_drain(bkv, 0);
+      // a producer that gave up still takes its share of the counter, so that the last taker
+      // resets it
+      if (!exhausted) {
+        while (true) {
+          const int f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+          if (f >= units) {
+            if (f == units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+            break;
+          }
+        }
+      }
+      if (kv_loads > 0) wait_drain(dev::smem_u32(&sm.bar_kv), (kv_loads - 1) & 1);
       for (int s = 0; s < 2; ++s) drain_stage(dev::smem_u32(&sm.bar_qfull[s]), issued, s);
     }
   } else if (warp == kMmaWarp || warp == kGradWarp) {
     // ========================= tcgen05.mma issuers (two threads) ==========================
-    if (lane == 0 && nsteps > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_kk = dev::idesc_bf16_f32(kT, kSub, 0, 0);  // both K-major, N = 64
       constexpr uint32_t idesc_tm = dev::idesc_bf16_f32(kT, kD, 0, 1);    // A in TMEM, B MN-major
       const int role = warp == kMmaWarp ? 0 : 1;
+      // operand descriptors of the two stages: K-major (score products) and MN-major
+      // (accumulating products) views of Q and dO
+      uint64_t dqk[2], dok[2], dqm[2], dom[2];
+      for (int s = 0; s < 2; ++s) {
+        dqk[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), 16, 1024, dev::kSwizzle128B);
+        dok[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), 16, 1024, dev::kSwizzle128B);
+        dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+        dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+      }
+      const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
+      const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
       bool ok = true;
-      if (role == 0) {
-        // S^T = K Q_h^T and dP^T = V dO_h^T for sub-step m (queries 64h .. 64h+63 of its tile)
-        const uint64_t dka = dev::smem_desc(dev::smem_u32(sm.k), 16, 1024, dev::kSwizzle128B);
-        const uint64_t dva = dev::smem_desc(dev::smem_u32(sm.v), 16, 1024, dev::kSwizzle128B);
-        uint64_t dqk[2], dok[2];
-        for (int s = 0; s < 2; ++s) {
-          dqk[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), 16, 1024, dev::kSwizzle128B);
-          dok[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), 16, 1024, dev::kSwizzle128B);
-        }
-        ok = wait_bounded(dev::smem_u32(&sm.bar_kv), 0, abort);
-        for (int m = 0; ok && m < nsub; ++m) {
-          const int n = m >> 1, h = m & 1, s = n & 1;
-          // buffer m & 1 is free once the accumulating MMAs of sub-step m - 2 have completed
-          if (m >= 2 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_free[m & 1]),
-                                            ((m >> 1) - 1) & 1, abort)))
-            break;
-          if (h == 0 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort)))
-            break;
-          dev::tc_fence_after();
-          const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
-          const uint32_t hoff = (h * kSubBytes) >> 4;
-          const uint64_t bq = (s ? dqk[1] : dqk[0]) + hoff, bo = (s ? dok[1] : dok[0]) + hoff;
+      int taken = 0;  // units read from the slots
+      int mg = 0;     // sub-steps of all earlier units (the barrier phases run on)
+      int kv_waits = 0;
+      while (ok) {
+        const int slot = taken & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort)))
+          break;
+        const int f = sm.unit[slot];
+        ++taken;
+        if (f < 0) break;
+        const int nsub = 2 * kv_unit(p, f).nsteps;
+        if (nsub > 0) {
+          if (role == 0) {
+            // S^T = K Q_h^T and dP^T = V dO_h^T for sub-step m (queries 64h .. 64h+63 of its tile)
+            ok = wait_bounded(dev::smem_u32(&sm.bar_kv), kv_waits & 1, abort);
+            ++kv_waits;
+            for (int ml = 0; ok && ml < nsub; ++ml) {
+              const int m = mg + ml;
+              const int n = m >> 1, h = m & 1, s = n & 1;
+              // buffer m & 1 is free once the accumulating MMAs of sub-step m - 2 have completed
+              if (m >= 2 && !(ok = wait_bounded(dev::smem_u32(&sm.bar_free[m & 1]),
+                                                ((m >> 1) - 1) & 1, abort)))
+                break;
+              if (h == 0 &&
+                  !(ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort)))
+                break;
+              dev::tc_fence_after();
+              const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+              const uint32_t hoff = (h * kSubBytes) >> 4;
+              const uint64_t bq = (s ? dqk[1] : dqk[0]) + hoff, bo = (s ? dok[1] : dok[0]) + hoff;
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-            dev::umma_ss(t_st, dka + koff, bq + koff, idesc_kk, ks > 0 ? 1u : 0u);
-          }
+              for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+                dev::umma_ss(t_st, dka + koff, bq + koff, idesc_kk, ks > 0 ? 1u : 0u);
+              }
 #pragma unroll
-          for (int ks = 0; ks < kD / 16; ++ks) {
-            const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
-            dev::umma_ss(t_dpt, dva + koff, bo + koff, idesc_kk, ks > 0 ? 1u : 0u);
-          }
-          dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
-        }
-      } else {
-        // dV += P^T dO_h and dK += dS^T Q_h (K = the 64 queries of the sub-step)
-        uint64_t dqm[2], dom[2];
-        for (int s = 0; s < 2; ++s) {
-          dqm[s] = dev::smem_desc(dev::smem_u32(sm.q[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-          dom[s] = dev::smem_desc(dev::smem_u32(sm.dout[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-        }
-        for (int m = 0; ok && m < nsub; ++m) {
-          const int n = m >> 1, h = m & 1, s = n & 1;
-          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort))) break;
-          dev::tc_fence_after();
-          const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
-          const uint64_t bo = s ? dom[1] : dom[0], bq = s ? dqm[1] : dqm[0];
+              for (int ks = 0; ks < kD / 16; ++ks) {
+                const uint32_t koff = ((ks >> 2) * kHalfBytes + (ks & 3) * 32) >> 4;
+                dev::umma_ss(t_dpt, dva + koff, bo + koff, idesc_kk, ks > 0 ? 1u : 0u);
+              }
+              dev::umma_commit(dev::smem_u32(&sm.bar_s[m & 1]));
+            }
+            // the unit's K and V are read for good once these products complete
+            if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_kvempty));
+          } else {
+            // dV += P^T dO_h and dK += dS^T Q_h (K = the 64 queries of the sub-step)
+            for (int ml = 0; ok && ml < nsub; ++ml) {
+              const int m = mg + ml;
+              const int n = m >> 1, h = m & 1, s = n & 1;
+              if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_p[m & 1]), (m >> 1) & 1, abort))) break;
+              dev::tc_fence_after();
+              const uint32_t t_st = tmem + (m & 1) * kSub, t_dpt = tmem + 128 + (m & 1) * kSub;
+              const uint64_t bo = s ? dom[1] : dom[0], bq = s ? dqm[1] : dqm[0];
 #pragma unroll
-          for (int ks = 0; ks < kSub / 16; ++ks) {
-            const uint32_t acc = (m > 0 || ks > 0) ? 1u : 0u;
-            const uint32_t boff = (h * kSubBytes + ks * 16 * 128) >> 4;
-            dev::umma_ts(tmem + 256, t_st + packed_col(ks), bo + boff, idesc_tm, acc);
-            dev::umma_ts(tmem + 384, t_dpt + packed_col(ks), bq + boff, idesc_tm, acc);
+              for (int ks = 0; ks < kSub / 16; ++ks) {
+                const uint32_t acc = (ml > 0 || ks > 0) ? 1u : 0u;
+                const uint32_t boff = (h * kSubBytes + ks * 16 * 128) >> 4;
+                dev::umma_ts(tmem + 256, t_st + packed_col(ks), bo + boff, idesc_tm, acc);
+                dev::umma_ts(tmem + 384, t_dpt + packed_col(ks), bq + boff, idesc_tm, acc);
+              }
+              dev::umma_commit(dev::smem_u32(&sm.bar_free[m & 1]));
+              if (h == 1) dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));  // stage s read for good
+            }
+            // the accumulators are final once this thread's MMAs have completed (every score MMA
+            // completed before the row warps released the weights these read)
+            if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
           }
-          dev::umma_commit(dev::smem_u32(&sm.bar_free[m & 1]));
-          if (h == 1) dev::umma_commit(dev::smem_u32(&sm.bar_qempty[s]));  // stage s read for good
+          mg += nsub;
         }
-        // the accumulators are final once this thread's MMAs have completed (every score MMA
-        // completed before the row warps released the weights these read)
-        if (ok) dev::umma_commit(dev::smem_u32(&sm.bar_done));
+        // this thread has issued every product of the unit
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
       }
       dev::umma_commit(dev::smem_u32(&sm.bar_drain[role]));
       wait_drain(dev::smem_u32(&sm.bar_drain[role]), 0);
@@ -459,126 +551,148 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ============== row workers: one key each, two warps per key (column halves) ==============
     const int r = (warp & 3) * 32 + lane;  // TMEM lane = key c0 + r
     const int ch = warp >> 2;              // this warp's 32 of the 64 columns of a sub-step
-    const int j = c0 + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const float c = p.c;
-    const long long ds_base = nsteps > 0 ? p.ds_off[kb] : 0;
     bool ok = true;
-    for (int m = 0; m < nsub; ++m) {
-      const int n = m >> 1, h = m & 1, s = n & 1;
-      const int r0 = qr.tile(n % nqt) * kT + h * kSub;  // first query row of the sub-step
-      // the stage's LSE / D vectors came with its Q and dO tiles; the stage cannot be refilled
-      // before this tile's weights are released, so its phase is still this tile's
-      ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort) &&
-           wait_bounded(dev::smem_u32(&sm.bar_s[m & 1]), (m >> 1) & 1, abort);
+    int taken = 0;  // units read from the slots
+    int mg = 0;     // sub-steps of all earlier units
+    int dones = 0;  // units whose accumulators were read
+    while (ok) {
+      const int slot = taken & 1;
+      ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort);
       if (!(ok = __all_sync(0xffffffffu, ok))) break;
-      dev::tc_fence_after();
-      const uint32_t t_st = tmem + lane_off + (m & 1) * kSub + ch * 32;
-      const uint32_t t_dpt = tmem + lane_off + 128 + (m & 1) * kSub + ch * 32;
-      uint32_t sr[32], dr[32];
-      dev::tmem_ld32(t_st, sr);
-      dev::tmem_ld32(t_dpt, dr);
+      const int f = sm.unit[slot];
+      ++taken;
+      if (f < 0) break;
+      const KVUnit u = kv_unit(p, f);
+      const int j = u.c0 + r;
+      const int nsub = 2 * u.nsteps;
+      const long long ds_base = u.nsteps > 0 ? p.ds_off[u.kb] : 0;
+      for (int ml = 0; ml < nsub; ++ml) {
+        const int m = mg + ml;
+        const int nl = ml >> 1, h = m & 1, s = (m >> 1) & 1, n = m >> 1;
+        const int r0 = u.qr.tile(nl % u.nqt) * kT + h * kSub;  // first query row of the sub-step
+        // the stage's LSE / D vectors came with its Q and dO tiles; the stage cannot be refilled
+        // before this tile's weights are released, so its phase is still this tile's
+        ok = wait_bounded(dev::smem_u32(&sm.bar_qfull[s]), (n >> 1) & 1, abort) &&
+             wait_bounded(dev::smem_u32(&sm.bar_s[m & 1]), (m >> 1) & 1, abort);
+        if (!(ok = __all_sync(0xffffffffu, ok))) break;
+        dev::tc_fence_after();
+        const uint32_t t_st = tmem + lane_off + (m & 1) * kSub + ch * 32;
+        const uint32_t t_dpt = tmem + lane_off + 128 + (m & 1) * kSub + ch * 32;
+        uint32_t sr[32], dr[32];
+        dev::tmem_ld32(t_st, sr);
+        dev::tmem_ld32(t_dpt, dr);
 
-      // visible query columns of key j among this warp's 32 (columns past Nq: LSE = +inf):
-      // [lo, hi], and for the local + global mask also the global rows [glo, ghi]
-      const int P0 = r0 + off;
-      uint32_t vis = ~0u;
-      if (!block_visible(p.mask, P0, kSub, c0, kT)) {
-        int lo = -1, hi = kT, glo = 0, ghi = -1;
-        if (j >= p.mask.Nk) {
-          hi = -1;
-        } else if (p.mask.kind == ATTN_MASK_LOCAL_GLOBAL) {
-          if (j >= p.mask.n_sink) {  // a global key is seen by every row
-            lo = clamp_col(static_cast<long long>(j) - p.mask.window - P0);  // p >= j - w
-            hi = clamp_col(static_cast<long long>(j) + p.mask.window - P0);  // p <= j + w
-            glo = clamp_col(-static_cast<long long>(P0));                  // p >= 0
-            ghi = clamp_col(static_cast<long long>(p.mask.n_sink) - 1 - P0);  // p < n_global
+        // visible query columns of key j among this warp's 32 (columns past Nq: LSE = +inf):
+        // [lo, hi], and for the local + global mask also the global rows [glo, ghi]
+        const int P0 = r0 + off;
+        uint32_t vis = ~0u;
+        if (!block_visible(p.mask, P0, kSub, u.c0, kT)) {
+          int lo = -1, hi = kT, glo = 0, ghi = -1;
+          if (j >= p.mask.Nk) {
+            hi = -1;
+          } else if (p.mask.kind == ATTN_MASK_LOCAL_GLOBAL) {
+            if (j >= p.mask.n_sink) {  // a global key is seen by every row
+              lo = clamp_col(static_cast<long long>(j) - p.mask.window - P0);  // p >= j - w
+              hi = clamp_col(static_cast<long long>(j) + p.mask.window - P0);  // p <= j + w
+              glo = clamp_col(-static_cast<long long>(P0));                  // p >= 0
+              ghi = clamp_col(static_cast<long long>(p.mask.n_sink) - 1 - P0);  // p < n_global
+            }
+          } else if (p.mask.kind != ATTN_MASK_FULL) {
+            lo = clamp_col(static_cast<long long>(j) - P0);  // p >= j
+            if (p.mask.kind == ATTN_MASK_SLIDING && j >= p.mask.n_sink)
+              hi = clamp_col(static_cast<long long>(j) + p.mask.window - 1 - P0);  // p < j + w
           }
-        } else if (p.mask.kind != ATTN_MASK_FULL) {
-          lo = clamp_col(static_cast<long long>(j) - P0);  // p >= j
-          if (p.mask.kind == ATTN_MASK_SLIDING && j >= p.mask.n_sink)
-            hi = clamp_col(static_cast<long long>(j) + p.mask.window - 1 - P0);  // p < j + w
+          vis = (cols_upto(hi, ch) & ~cols_upto(lo - 1, ch)) |
+                (cols_upto(ghi, ch) & ~cols_upto(glo - 1, ch));
         }
-        vis = (cols_upto(hi, ch) & ~cols_upto(lo - 1, ch)) |
-              (cols_upto(ghi, ch) & ~cols_upto(glo - 1, ch));
-      }
-      const float4* l2v = reinterpret_cast<const float4*>(sm.lse2[s] + h * kSub + ch * 32);
-      const float4* ddv = reinterpret_cast<const float4*>(sm.dsum[s] + h * kSub + ch * 32);
-      dev::tmem_wait_ld();
+        const float4* l2v = reinterpret_cast<const float4*>(sm.lse2[s] + h * kSub + ch * 32);
+        const float4* ddv = reinterpret_cast<const float4*>(sm.dsum[s] + h * kSub + ch * 32);
+        dev::tmem_wait_ld();
 #pragma unroll
-      for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
-      uint32_t pk[16], dk16[16];
+        for (int e = 0; e < 32; ++e) asm volatile("" : "+r"(sr[e]), "+r"(dr[e]));
+        uint32_t pk[16], dk16[16];
 #pragma unroll
-      for (int e4 = 0; e4 < 8; ++e4) {
-        const float4 l4 = l2v[e4], d4 = ddv[e4];
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 l4 = l2v[e4], d4 = ddv[e4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dvv[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-        for (int e2 = 0; e2 < 4; e2 += 2) {
-          const int e = e4 * 4 + e2;
-          float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -lv[e2]));
-          float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e2 + 1]));
-          p0 = ((vis >> e) & 1u) ? p0 : 0.f;
-          p1 = ((vis >> (e + 1)) & 1u) ? p1 : 0.f;
-          const float d0 = p0 * (__uint_as_float(dr[e]) - dvv[e2]);
-          const float d1 = p1 * (__uint_as_float(dr[e + 1]) - dvv[e2 + 1]);
-          pk[e >> 1] = dev::pack_bf16x2(p0, p1);
-          dk16[e >> 1] = dev::pack_bf16x2(d0, d1);
+          for (int e2 = 0; e2 < 4; e2 += 2) {
+            const int e = e4 * 4 + e2;
+            float p0 = dev::ex2_approx(fmaf(__uint_as_float(sr[e]), c, -lv[e2]));
+            float p1 = dev::ex2_approx(fmaf(__uint_as_float(sr[e + 1]), c, -lv[e2 + 1]));
+            p0 = ((vis >> e) & 1u) ? p0 : 0.f;
+            p1 = ((vis >> (e + 1)) & 1u) ? p1 : 0.f;
+            const float d0 = p0 * (__uint_as_float(dr[e]) - dvv[e2]);
+            const float d1 = p1 * (__uint_as_float(dr[e + 1]) - dvv[e2 + 1]);
+            pk[e >> 1] = dev::pack_bf16x2(p0, p1);
+            dk16[e >> 1] = dev::pack_bf16x2(d0, d1);
+          }
         }
-      }
-      // P^T over S^T and dS^T over dP^T, packed into the first 16 of the 32 columns this warp
-      // has just read (see packed_col)
-      dev::tmem_st16(t_st, pk);
-      dev::tmem_st16(t_dpt, dk16);
-      {
-        // the same bf16 dS^T values into this (key block, query tile) block for the dQ kernel:
-        // rows 32 (warp & 3) .. +31 (keys), columns 64h + 32ch .. +31 (queries), staged in this
-        // warp's box (64-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
-        // once the box's previous store has read it, then one TMA store
-        const int hq = hk * p.G + n / nqt;
-        const long long slot = static_cast<long long>(b * p.Hq + hq) * p.ds_pairs + ds_base + n % nqt;
-        const uint32_t box = dev::smem_u32(sm.ds_stage[warp]);
-        if (m > 0) {
-          if (lane == 0) dev::bulk_wait_group_read0();
+        // P^T over S^T and dS^T over dP^T, packed into the first 16 of the 32 columns this warp
+        // has just read (see packed_col)
+        dev::tmem_st16(t_st, pk);
+        dev::tmem_st16(t_dpt, dk16);
+        {
+          // the same bf16 dS^T values into this (key block, query tile) block for the dQ kernel:
+          // rows 32 (warp & 3) .. +31 (keys), columns 64h + 32ch .. +31 (queries), staged in this
+          // warp's box (64-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ ((r >> 1) & 3))
+          // once the box's previous store has read it, then one TMA store
+          const int hq = u.hk * p.G + nl / u.nqt;
+          const long long slot_ds =
+              static_cast<long long>(u.b * p.Hq + hq) * p.ds_pairs + ds_base + nl % u.nqt;
+          const uint32_t box = dev::smem_u32(sm.ds_stage[warp]);
+          if (m > 0) {
+            if (lane == 0) dev::bulk_wait_group_read0();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
+                              dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
+          dev::fence_proxy_async_smem();
           __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_3d(&tm_ds, box, h * kSub + ch * 32, (warp & 3) * 32,
+                              static_cast<int>(slot_ds));
+            dev::bulk_commit_group();
+          }
         }
-#pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4)
-          dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
-                            dk16[4 * v4], dk16[4 * v4 + 1], dk16[4 * v4 + 2], dk16[4 * v4 + 3]);
-        dev::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          dev::tma_store_3d(&tm_ds, box, h * kSub + ch * 32, (warp & 3) * 32, static_cast<int>(slot));
-          dev::bulk_commit_group();
+        dev::tmem_wait_st();
+        dev::tc_fence_before();
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
+      }
+      mg += nsub;
+
+      // ---- epilogue: dV and scale * dK rows of this unit's keys, bf16, a column half per warp ----
+      // dV and dK leave TMEM before this warp releases the next unit's first weights (whose
+      // accumulating product overwrites them)
+      const bool valid = j < p.Nk;
+      const size_t krow = static_cast<size_t>(u.bk) * p.Nk + j;
+      __nv_bfloat16* dst_v = p.dv + krow * kD;
+      __nv_bfloat16* dst_k = p.dk + krow * kD;
+      if (u.nsteps == 0) {
+        if (valid) {
+          store_zero_row(dst_v, ch);
+          store_zero_row(dst_k, ch);
+        }
+      } else if (ok) {
+        ok = wait_bounded(dev::smem_u32(&sm.bar_done), dones & 1, abort);
+        if ((ok = __all_sync(0xffffffffu, ok))) {
+          dev::tc_fence_after();
+          store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid, ch);
+          store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid, ch);
         }
       }
-      dev::tmem_wait_st();
+      if (u.nsteps > 0) ++dones;
       dev::tc_fence_before();
-      dev::mbar_arrive(dev::smem_u32(&sm.bar_p[m & 1]));
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
     }
-
     // every staged box has been read by its store before the CTA can end
     if (lane == 0) dev::bulk_wait_group_read0();
     __syncwarp();
-
-    // ---- epilogue: dV and scale * dK rows of this CTA's keys, bf16, a column half per warp ----
-    const bool valid = j < p.Nk;
-    const size_t krow = static_cast<size_t>(bk) * p.Nk + j;
-    __nv_bfloat16* dst_v = p.dv + krow * kD;
-    __nv_bfloat16* dst_k = p.dk + krow * kD;
-    if (nsteps == 0) {
-      if (valid) {
-        store_zero_row(dst_v, ch);
-        store_zero_row(dst_k, ch);
-      }
-    } else if (ok) {
-      ok = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
-      if (__all_sync(0xffffffffu, ok)) {
-        dev::tc_fence_after();
-        store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid, ch);
-        store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid, ch);
-      }
-    }
   }
 
   // ---- teardown ----
