@@ -900,7 +900,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   const int nqt = (Nq + bwd::kT - 1) / bwd::kT, nkb = (Nk + bwd::kT - 1) / bwd::kT;
   const long long units_q = static_cast<long long>((nqt + 1) / 2) * B * Hq;  // query-tile pairs
   const long long units_kv = static_cast<long long>(nkb) * B * Hkv;
-  if (units_q > 0x7fffffffLL || units_kv > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
+  if (units_q > 0x7fffffffLL - 4096 || units_kv > 0x7fffffffLL - 4096) return ATTN_ERR_UNSUPPORTED;
   const MaskSpec mask = make_mask(mask_kind, window, n_sink, Nk);
   const BwdLayout L = bwd_layout(B, Hq, Nq, Nk, mask);
   if (static_cast<double>(B) * Hq * static_cast<double>(L.pairs) > 2147483647.0)
@@ -966,6 +966,9 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_UNSUPPORTED;
   }
+  // dQ as boxes of 32 columns x 32 rows staged with the 64-byte swizzle
+  CUtensorMap tdq;
+  if (encode_map_out(&tdq, dq, Nq, B * Hq, false) != ATTN_OK) return ATTN_ERR_UNSUPPORTED;
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
   bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
                                                bwd::kPrepRowsPerBlock),
@@ -977,8 +980,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(std::min<long long>(units_kv, info->num_sms)),
                          bwd::kThreads, bwd::kSmemKVBytes, st>>>(tq, tk, tv, tdo, tds_out, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
-  bwd::bwd_dq_kernel<<<static_cast<unsigned>(units_q), bwd::kThreads, bwd::kSmemQBytes, st>>>(
-      tds, tk, p);
+  bwd::bwd_dq_kernel<<<static_cast<unsigned>(std::min<long long>(units_q, info->num_sms)),
+                       bwd::kThreads, bwd::kSmemQBytes, st>>>(tds, tk, tdq, p);
   return cuda_status(cudaGetLastError());
 }
 

@@ -22,9 +22,10 @@
 //     read from TMEM.
 //     It also writes each (key block, query tile) block of dS^T (bf16, the values its own
 //     dK MMA used) to a workspace slot.
-//  3. bwd_dq_kernel: one CTA per (b, query head, 128-row query tile) computes dQ = scale dS K as
-//     a plain tensor-core product over the dS^T blocks of the tile's key tiles: no recomputation
-//     and no softmax, so it is bound by reading dS (2 bytes per visible pair).
+//  3. bwd_dq_kernel: persistent CTAs take units of (b, query head, two 128-row query tiles) and
+//     compute dQ = scale dS K as a plain tensor-core product over the dS^T blocks of each tile's
+//     key tiles: no recomputation and no softmax, so it is bound by reading dS (2 bytes per
+//     visible pair).
 // Handing dS over through HBM instead of recomputing it (or of atomically adding dQ partials)
 // costs a write and a read of dS but keeps every product on the tensor core exactly once, and
 // the result does not depend on the order in which CTAs finish.
@@ -705,59 +706,87 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// 3. dQ = scale dS K over the dS^T blocks the dK/dV kernel wrote.  One CTA per (b, query head,
+// 3. dQ = scale dS K over the dS^T blocks the dK/dV kernel wrote.  A unit is a (b, query head,
 //    pair of query tiles): tile qt = nqt-1-i (heavy under a causal mask) and tile i (light), so
-//    CTAs carry similar work and each pays its set-up once for two tiles.  dS^T blocks and K
-//    tiles stream through a 3-stage ring (the first tile's blocks, then the second's); one thread
-//    issues the MMAs (A = dS read MN-major from the [keys][queries] block, B = K MN-major) into
-//    one 128-column TMEM accumulator per tile; warps 0-7 store the results.
+//    units carry similar work.  Persistent CTAs (one per SM) take units from a counter.  dS^T
+//    blocks and K tiles stream through a 3-stage ring (a unit's first tile's blocks, then its
+//    second's, the ring running on across units); one thread issues the MMAs (A = dS read
+//    MN-major from the [keys][queries] block, B = K MN-major) into one 128-column TMEM
+//    accumulator per tile, the two accumulator pairs alternating between units so that warps
+//    0-7 store one unit's dQ (staged in shared-memory boxes, stored by TMA) while the next
+//    unit's products run.
 // ------------------------------------------------------------------------------------------
 constexpr int kDqStages = 3;
+constexpr uint32_t kDqBoxBytes = 32 * 32 * 2;  // 32 rows x 32 columns, 64-byte swizzle
 
 struct __align__(1024) SmemQ {
   uint8_t ds[kDqStages][kTileBytes];
   uint8_t k[kDqStages][kTileBytes];
-  uint64_t bar_full[kDqStages], bar_empty[kDqStages], bar_done, bar_drain;
+  uint8_t stage[8][2][kDqBoxBytes];  // two output boxes per store warp, used in turn
+  uint64_t bar_full[kDqStages], bar_empty[kDqStages], bar_drain;
+  uint64_t bar_done[2];     // accumulator pair a: the unit's products completed + flags written
+  uint64_t bar_accfree[2];  // accumulator pair a: read out by the store warps
+  uint64_t bar_unit_full[2], bar_unit_empty[2];
+  int unit[2];              // published units (-1: no more)
+  int any[2];               // per accumulator pair: bit t = some dS block contributed to tile t
   uint32_t tmem_base;
   int abort;
-  int any;  // set by the MMA thread: bit t = some dS block contributed to tile t
 };
 constexpr size_t kSmemQBytes = sizeof(SmemQ) + 1024;
+static_assert(kSmemQBytes <= 227 * 1024, "shared memory of the dQ kernel");
+
+// The readers of a unit slot: the MMA thread and the 8 store warps.
+constexpr uint32_t kQUnitReaders = 9;
 
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_ds,
-                  const __grid_constant__ CUtensorMap tm_k, const Params p) {
+                  const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_dq, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   SmemQ& sm = *reinterpret_cast<SmemQ*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                         ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-
   const int nbh = p.B * p.Hq;
-  const int pi = static_cast<int>(blockIdx.x) / nbh;
-  const int bh = blockIdx.x % nbh;
-  const int b = bh / p.Hq, h = bh % p.Hq;
-  const int bkv = b * p.Hkv + h / p.G;
   const int off = p.Nk - p.Nq;
-  int qts[2] = {p.num_qtiles - 1 - pi, pi};
-  const int ntiles = qts[0] == qts[1] ? 1 : 2;
-  TileRange trs[2];
-  int nks[2] = {0, 0};
-  for (int t = 0; t < ntiles; ++t) {
-    const int r0 = qts[t] * kT, last_row = min(r0 + kT, p.Nq) - 1;
-    trs[t] = key_tiles(p.mask, r0 + off, last_row + off, kT);
-    nks[t] = trs[t].count();
-  }
-  const int nsteps = nks[0] + (ntiles > 1 ? nks[1] : 0);
-  // step jj: tile t = jj < nks[0] ? 0 : 1 and its key tile; a pair outside the key block's
-  // query-tile range has no visible entry and no dS block (slot -1); every role walks the same
-  // list
-  auto step_slot = [&](int jj, int& t, int& kt) -> long long {
-    t = jj < nks[0] ? 0 : 1;
-    kt = t ? trs[1].tile(jj - nks[0]) : trs[0].tile(jj);
+  const int units = ((p.num_qtiles + 1) / 2) * nbh;
+
+  // unit f: (b, h) and its one or two query tiles with their key-tile ranges
+  struct QUnit {
+    int bh, bkv, ntiles, nsteps;
+    int qts[2], nks[2];
+    TileRange trs[2];
+  };
+  auto q_unit = [&](int f) {
+    QUnit u;
+    const int pi = f / nbh;
+    u.bh = f % nbh;
+    const int b = u.bh / p.Hq, h = u.bh % p.Hq;
+    u.bkv = b * p.Hkv + h / p.G;
+    u.qts[0] = p.num_qtiles - 1 - pi;
+    u.qts[1] = pi;
+    u.ntiles = u.qts[0] == u.qts[1] ? 1 : 2;
+    u.nks[0] = u.nks[1] = 0;
+    u.trs[1] = TileRange{0, 0, -1};
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (t >= u.ntiles) break;
+      const int r0 = u.qts[t] * kT, last_row = min(r0 + kT, p.Nq) - 1;
+      u.trs[t] = key_tiles(p.mask, r0 + off, last_row + off, kT);
+      u.nks[t] = u.trs[t].count();
+    }
+    u.nsteps = u.nks[0] + (u.ntiles > 1 ? u.nks[1] : 0);
+    return u;
+  };
+  // step jj of unit u: tile t = jj < nks[0] ? 0 : 1 and its key tile; a pair outside the key
+  // block's query-tile range has no visible entry and no dS block (slot -1); the producer and
+  // the MMA thread walk the same list
+  auto step_slot = [&](const QUnit& u, int jj, int& t, int& kt) -> long long {
+    t = jj < u.nks[0] ? 0 : 1;
+    kt = t ? u.trs[1].tile(jj - u.nks[0]) : u.trs[0].tile(jj);
     const int c0 = kt * kT, c1 = min(c0 + kT, p.Nk) - 1;
-    const int idx = pair_index(query_tiles(p.mask, c0, c1, off, p.Nq), t ? qts[1] : qts[0]);
+    const int idx = pair_index(query_tiles(p.mask, c0, c1, off, p.Nq), t ? u.qts[1] : u.qts[0]);
     if (idx < 0) return -1;
-    return static_cast<long long>(bh) * p.ds_pairs + p.ds_off[kt] + idx;
+    return static_cast<long long>(u.bh) * p.ds_pairs + p.ds_off[kt] + idx;
   };
 
   if (tid == 0) {
@@ -765,18 +794,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(dev::smem_u32(&sm.bar_full[s]), 1);
       dev::mbar_init(dev::smem_u32(&sm.bar_empty[s]), 1);
     }
-    dev::mbar_init(dev::smem_u32(&sm.bar_done), 1);
+    for (int a = 0; a < 2; ++a) {
+      dev::mbar_init(dev::smem_u32(&sm.bar_done[a]), 2);  // the MMA commit and the flags
+      dev::mbar_init(dev::smem_u32(&sm.bar_accfree[a]), 8);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_full[a]), 1);
+      dev::mbar_init(dev::smem_u32(&sm.bar_unit_empty[a]), kQUnitReaders);
+    }
     dev::mbar_init(dev::smem_u32(&sm.bar_drain), 1);
     sm.abort = 0;
-    sm.any = 0;
     dev::fence_barrier_init();
   }
   if (warp == kLoadWarp && lane == 0) {
     dev::tma_prefetch_desc(&tm_ds);
     dev::tma_prefetch_desc(&tm_k);
+    dev::tma_prefetch_desc(&tm_dq);
   }
   if (warp == kMmaWarp) {
-    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 256);
+    dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
     dev::tmem_relinquish();
   }
   dev::tc_fence_before();
@@ -786,25 +820,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort = &sm.abort;
 
   if (warp == kLoadWarp) {
-    // ================================ TMA producer ================================
+    // ============================ unit fetch + TMA producer ============================
     if (lane == 0) {
-      int u = 0;
-      for (int jj = 0; jj < nsteps; ++jj) {
-        int t, kt;
-        const long long slot = step_slot(jj, t, kt);
-        if (slot < 0) continue;
-        const int s = u % kDqStages;
-        if (!wait_bounded(dev::smem_u32(&sm.bar_empty[s]), ((u / kDqStages) & 1) ^ 1, abort))
+      int published = 0, u = 0;  // u: copies started (the stage ring runs on across units)
+      bool ok = true, exhausted = false;
+      while (ok) {
+        const int slot = published & 1;
+        if (published >= 2 && !wait_bounded(dev::smem_u32(&sm.bar_unit_empty[slot]),
+                                             ((published - 2) >> 1) & 1, abort)) {
+          ok = false;
           break;
-        const uint32_t bf = dev::smem_u32(&sm.bar_full[s]);
-        dev::mbar_arrive_expect_tx(bf, 2 * kTileBytes);
-        for (int half = 0; half < 2; ++half) {
-          dev::tma_load_3d(dev::smem_u32(sm.ds[s]) + half * kHalfBytes, &tm_ds, bf, half * 64, 0,
-                           static_cast<int>(slot));
-          dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bf, half * 64,
-                           kt * kT, bkv);
         }
-        ++u;
+        const int f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+        if (f >= units) {
+          if (f == units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+          exhausted = true;
+        }
+        sm.unit[slot] = exhausted ? -1 : f;
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_full[slot]));
+        if (exhausted) break;
+        ++published;
+        const QUnit qu = q_unit(f);
+        for (int jj = 0; jj < qu.nsteps; ++jj) {
+          int t, kt;
+          const long long dslot = step_slot(qu, jj, t, kt);
+          if (dslot < 0) continue;
+          const int s = u % kDqStages;
+          if (!wait_bounded(dev::smem_u32(&sm.bar_empty[s]), ((u / kDqStages) & 1) ^ 1, abort)) {
+            ok = false;
+            break;
+          }
+          const uint32_t bf = dev::smem_u32(&sm.bar_full[s]);
+          dev::mbar_arrive_expect_tx(bf, 2 * kTileBytes);
+          for (int half = 0; half < 2; ++half) {
+            dev::tma_load_3d(dev::smem_u32(sm.ds[s]) + half * kHalfBytes, &tm_ds, bf, half * 64, 0,
+                             static_cast<int>(dslot));
+            dev::tma_load_3d(dev::smem_u32(sm.k[s]) + half * kHalfBytes, &tm_k, bf, half * 64,
+                             kt * kT, qu.bkv);
+          }
+          ++u;
+        }
+      }
+      if (!exhausted) {
+        // a producer that gave up still takes its share of the counter, so that the last taker
+        // resets it
+        while (true) {
+          const int f = static_cast<int>(atomicAdd(p.unit_counter, 1u));
+          if (f >= units) {
+            if (f == units + static_cast<int>(gridDim.x) - 1) atomicExch(p.unit_counter, 0u);
+            break;
+          }
+        }
       }
       // drain: the last copy into each stage has landed
       for (int s = 0; s < kDqStages; ++s) {
@@ -817,53 +883,119 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc = dev::idesc_bf16_f32(kT, kD, 1, 1);  // A and B MN-major
       bool ok = true;
-      int u = 0, used[2] = {0, 0};
-      for (int jj = 0; ok && jj < nsteps; ++jj) {
-        int t, kt;
-        if (step_slot(jj, t, kt) < 0) continue;
-        const int s = u % kDqStages;
-        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_full[s]), (u / kDqStages) & 1, abort))) break;
-        dev::tc_fence_after();
-        const uint64_t da = dev::smem_desc(dev::smem_u32(sm.ds[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-        const uint64_t db = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
-        const int first = t ? used[1] == 0 : used[0] == 0;
+      int u = 0, taken = 0;
+      while (ok) {
+        const int slot = taken & 1;
+        if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort)))
+          break;
+        const int f = sm.unit[slot];
+        const int un = taken++;  // this CTA's unit number: accumulator pair un & 1
+        if (f < 0) break;
+        const QUnit qu = q_unit(f);
+        const int a = un & 1;
+        // the pair's previous unit (two back) has been read out
+        if (un >= 2 &&
+            !(ok = wait_bounded(dev::smem_u32(&sm.bar_accfree[a]), ((un - 2) >> 1) & 1, abort)))
+          break;
+        int used[2] = {0, 0};
+        for (int jj = 0; ok && jj < qu.nsteps; ++jj) {
+          int t, kt;
+          if (step_slot(qu, jj, t, kt) < 0) continue;
+          const int s = u % kDqStages;
+          if (!(ok = wait_bounded(dev::smem_u32(&sm.bar_full[s]), (u / kDqStages) & 1, abort))) break;
+          dev::tc_fence_after();
+          const uint64_t da = dev::smem_desc(dev::smem_u32(sm.ds[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+          const uint64_t db = dev::smem_desc(dev::smem_u32(sm.k[s]), kHalfBytes, 1024, dev::kSwizzle128B);
+          const int first = t ? used[1] == 0 : used[0] == 0;
 #pragma unroll
-        for (int ks = 0; ks < kT / 16; ++ks)  // 16 keys (2 KB of each block) per MMA
-          dev::umma_ss(tmem + t * 128, da + ((ks * 2048) >> 4), db + ((ks * 2048) >> 4), idesc,
-                       (!first || ks > 0) ? 1u : 0u);
-        dev::umma_commit(dev::smem_u32(&sm.bar_empty[s]));
-        if (t) ++used[1]; else ++used[0];
-        ++u;
+          for (int ks = 0; ks < kT / 16; ++ks)  // 16 keys (2 KB of each block) per MMA
+            dev::umma_ss(tmem + a * 256 + t * 128, da + ((ks * 2048) >> 4),
+                         db + ((ks * 2048) >> 4), idesc, (!first || ks > 0) ? 1u : 0u);
+          dev::umma_commit(dev::smem_u32(&sm.bar_empty[s]));
+          if (t) ++used[1]; else ++used[0];
+          ++u;
+        }
+        if (!ok) break;
+        // the products of the unit are done once this commit arrives; the flags follow
+        dev::umma_commit(dev::smem_u32(&sm.bar_done[a]));
+        sm.any[a] = (used[0] > 0 ? 1 : 0) | (used[1] > 0 ? 2 : 0);
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_done[a]));
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
       }
-      if (ok && u > 0) dev::umma_commit(dev::smem_u32(&sm.bar_done));
       dev::umma_commit(dev::smem_u32(&sm.bar_drain));
       wait_drain(dev::smem_u32(&sm.bar_drain), 0);
-      sm.any = ok ? (used[0] > 0 ? 1 : 0) | (used[1] > 0 ? 2 : 0) : 0;
     }
-  }
-  // every MMA has completed (the MMA thread drained them) and sm.any is published
-  __syncthreads();
-  if (warp < 8) {
-    // =================== store: scale * dQ of each tile, a column half per warp ===================
+  } else if (warp < 8) {
+    // ========= store: scale * dQ of each tile, a column half per warp, by TMA boxes =========
     const int r = (warp & 3) * 32 + lane;
     const int ch = warp >> 2;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int flags = sm.any;
-    bool ready = false;
-    if (flags) {
-      ready = wait_bounded(dev::smem_u32(&sm.bar_done), 0, abort);
-      if (ready) dev::tc_fence_after();
-    }
-    for (int t = 0; t < ntiles; ++t) {
-      const int i = qts[t] * kT + r;
-      const bool valid = i < p.Nq;
-      __nv_bfloat16* dst = p.dq + (static_cast<size_t>(bh) * p.Nq + i) * kD;
-      if (!(flags & (1 << t))) {
-        if (valid && !*abort) store_zero_row(dst, ch);
-      } else if (ready) {
-        store_acc_row(tmem + lane_off + t * 128, p.scale, dst, valid, ch);
+    bool ok = true;
+    int taken = 0, nbox = 0;
+    while (ok) {
+      const int slot = taken & 1;
+      ok = wait_bounded(dev::smem_u32(&sm.bar_unit_full[slot]), (taken >> 1) & 1, abort);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      const int f = sm.unit[slot];
+      const int un = taken++;
+      if (f < 0) break;
+      const QUnit qu = q_unit(f);
+      const int a = un & 1;
+      ok = wait_bounded(dev::smem_u32(&sm.bar_done[a]), (un >> 1) & 1, abort);
+      if (!(ok = __all_sync(0xffffffffu, ok))) break;
+      dev::tc_fence_after();
+      const int flags = sm.any[a];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (t >= qu.ntiles) break;
+        const int row0 = (t ? qu.qts[1] : qu.qts[0]) * kT;
+        const int i = row0 + r;
+        const bool valid = i < p.Nq;
+        __nv_bfloat16* dst = p.dq + (static_cast<size_t>(qu.bh) * p.Nq + i) * kD;
+        if (!(flags & (1 << t))) {
+          if (valid) store_zero_row(dst, ch);
+          continue;
+        }
+#pragma unroll 1
+        for (int cc = 2 * ch; cc < 2 * ch + 2; ++cc) {
+          uint32_t acc[32];
+          dev::tmem_ld32(tmem + lane_off + a * 256 + t * 128 + cc * 32, acc);
+          dev::tmem_wait_ld_regs(acc);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2)
+            pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(acc[e]) * p.scale,
+                                          __uint_as_float(acc[e + 1]) * p.scale);
+          // 32 rows x 32 columns through this warp's box (64-byte swizzle: 16-byte chunk c of
+          // row r at chunk c ^ ((r >> 1) & 3)), rewritten once the store before last from it
+          // has read it; rows past Nq are clipped by the tensor map
+          const uint32_t box = dev::smem_u32(sm.stage[warp][nbox & 1]);
+          if (lane == 0) dev::bulk_wait_group_read1();
+          __syncwarp();
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
+                              pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          dev::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            dev::tma_store_3d(&tm_dq, box, cc * 32, row0 + (warp & 3) * 32, qu.bh);
+            dev::bulk_commit_group();
+          }
+          ++nbox;
+        }
+      }
+      // this warp has read the accumulator pair and is done with the unit
+      dev::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_accfree[a]));
+        dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
       }
     }
+    // every staged box has been read by its store before the CTA can end
+    if (lane == 0) dev::bulk_wait_group_read0();
+    __syncwarp();
   }
 
   // ---- teardown ----
@@ -871,7 +1003,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == kMmaWarp) {
     dev::tc_fence_after();
-    dev::tmem_dealloc(tmem, 256);
+    dev::tmem_dealloc(tmem, 512);
   }
 }
 
