@@ -966,9 +966,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_UNSUPPORTED;
   }
-  // dQ as boxes of 32 columns x 32 rows staged with the 64-byte swizzle
-  CUtensorMap tdq;
-  if (encode_map_out(&tdq, dq, Nq, B * Hq, false) != ATTN_OK) return ATTN_ERR_UNSUPPORTED;
+  // dQ, dK and dV as boxes of 32 columns x 32 rows staged with the 64-byte swizzle
+  CUtensorMap tdq, tdk, tdv;
+  if (encode_map_out(&tdq, dq, Nq, B * Hq, false) != ATTN_OK ||
+      encode_map_out(&tdk, dk, Nk, B * Hkv, false) != ATTN_OK ||
+      encode_map_out(&tdv, dv, Nk, B * Hkv, false) != ATTN_OK)
+    return ATTN_ERR_UNSUPPORTED;
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
   bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
                                                bwd::kPrepRowsPerBlock),
@@ -978,7 +981,8 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   // persistent: one CTA per SM walking the key-block units
   bwd::bwd_dkdv_kernel<<<static_cast<unsigned>(std::min<long long>(units_kv, info->num_sms)),
-                         bwd::kThreads, bwd::kSmemKVBytes, st>>>(tq, tk, tv, tdo, tds_out, p);
+                         bwd::kThreads, bwd::kSmemKVBytes, st>>>(tq, tk, tv, tdo, tds_out, tdk,
+                                                                 tdv, p);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;
   bwd::bwd_dq_kernel<<<static_cast<unsigned>(std::min<long long>(units_q, info->num_sms)),
                        bwd::kThreads, bwd::kSmemQBytes, st>>>(tds, tk, tdq, p);

@@ -164,28 +164,6 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
       : "memory");
 }
 
-// Columns [64 ch, 64 ch + 64) of row r of a 128 x 128 fp32 accumulator in TMEM -> bf16 in
-// global memory (times mul).
-__device__ __forceinline__ void store_acc_row(uint32_t t_acc, float mul, __nv_bfloat16* dst,
-                                              bool valid, int ch) {
-#pragma unroll 1
-  for (int cc = 2 * ch; cc < 2 * ch + 2; ++cc) {
-    uint32_t a[32];
-    dev::tmem_ld32(t_acc + cc * 32, a);
-    dev::tmem_wait_ld_regs(a);
-    uint32_t pk[16];
-#pragma unroll
-    for (int e = 0; e < 32; e += 2)
-      pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(a[e]) * mul, __uint_as_float(a[e + 1]) * mul);
-    if (valid) {
-      uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-      for (int v4 = 0; v4 < 4; ++v4)
-        d4[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-    }
-  }
-}
-
 __device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int ch) {
   uint4* d4 = reinterpret_cast<uint4*>(dst + ch * 64);
 #pragma unroll
@@ -340,7 +318,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v,
                     const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_ds, const Params p) {
+                    const __grid_constant__ CUtensorMap tm_ds,
+                    const __grid_constant__ CUtensorMap tm_dk,
+                    const __grid_constant__ CUtensorMap tm_dv, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   SmemKV& sm = *reinterpret_cast<SmemKV*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                           ~uintptr_t(1023));
@@ -370,6 +350,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     dev::tma_prefetch_desc(&tm_v);
     dev::tma_prefetch_desc(&tm_do);
     dev::tma_prefetch_desc(&tm_ds);
+    dev::tma_prefetch_desc(&tm_dk);
+    dev::tma_prefetch_desc(&tm_dv);
   }
   if (warp == kMmaWarp) {
     dev::tmem_alloc(dev::smem_u32(&sm.tmem_base), 512);
@@ -644,10 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const long long slot_ds =
               static_cast<long long>(u.b * p.Hq + hq) * p.ds_pairs + ds_base + nl % u.nqt;
           const uint32_t box = dev::smem_u32(sm.ds_stage[warp]);
-          if (m > 0) {
-            if (lane == 0) dev::bulk_wait_group_read0();
-            __syncwarp();
-          }
+          if (lane == 0) dev::bulk_wait_group_read0();  // the box's previous store has read it
+          __syncwarp();
 #pragma unroll
           for (int v4 = 0; v4 < 4; ++v4)
             dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
@@ -682,8 +662,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_bounded(dev::smem_u32(&sm.bar_done), dones & 1, abort);
         if ((ok = __all_sync(0xffffffffu, ok))) {
           dev::tc_fence_after();
-          store_acc_row(tmem + lane_off + 256, 1.f, dst_v, valid, ch);
-          store_acc_row(tmem + lane_off + 384, p.scale, dst_k, valid, ch);
+          // dV then scale * dK, 32 keys x 32 columns at a time through this warp's box (as the
+          // dS^T blocks), stored by TMA; keys past Nk are clipped by the tensor maps
+#pragma unroll 1
+          for (int w2 = 0; w2 < 4; ++w2) {
+            const int which = w2 >> 1, cc = 2 * ch + (w2 & 1);
+            uint32_t a[32];
+            dev::tmem_ld32(tmem + lane_off + (which ? 384 : 256) + cc * 32, a);
+            dev::tmem_wait_ld_regs(a);
+            const float mul = which ? p.scale : 1.f;
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 32; e += 2)
+              pk[e >> 1] = dev::pack_bf16x2(__uint_as_float(a[e]) * mul, __uint_as_float(a[e + 1]) * mul);
+            const uint32_t box = dev::smem_u32(sm.ds_stage[warp]);
+            if (lane == 0) dev::bulk_wait_group_read0();
+            __syncwarp();
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dev::st_shared_v4(box + lane * 64 + (static_cast<uint32_t>(v4 ^ ((lane >> 1) & 3)) << 4),
+                                pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+            dev::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              dev::tma_store_3d(which ? &tm_dk : &tm_dv, box, cc * 32, u.c0 + (warp & 3) * 32, u.bk);
+              dev::bulk_commit_group();
+            }
+          }
         }
       }
       if (u.nsteps > 0) ++dones;
