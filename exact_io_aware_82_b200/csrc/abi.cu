@@ -973,9 +973,11 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
       encode_map_out(&tdv, dv, Nk, B * Hkv, false) != ATTN_OK)
     return ATTN_ERR_UNSUPPORTED;
   const long long prow = static_cast<long long>(B) * Hq * p.npad;
-  bwd::bwd_prep_kernel<<<static_cast<unsigned>((prow + bwd::kPrepRowsPerBlock - 1) /
-                                               bwd::kPrepRowsPerBlock),
-                         256, 0, st>>>(
+  // one wave (4 blocks of 8 warps per SM at 64 registers a thread), grid-stride over the row groups
+  const long long prep_blocks = std::min<long long>((prow + bwd::kPrepRowsPerBlock - 1) /
+                                                        bwd::kPrepRowsPerBlock,
+                                                    4LL * info->num_sms);
+  bwd::bwd_prep_kernel<<<static_cast<unsigned>(prep_blocks), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, lse2,
       dsum, Nq, p.npad, prow, mask, nkb, p.ds_off);
   if ((rc = cuda_status(cudaGetLastError())) != ATTN_OK) return rc;

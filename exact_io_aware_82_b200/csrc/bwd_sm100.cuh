@@ -179,7 +179,7 @@ __device__ __forceinline__ uint32_t packed_col(int ks) { return ks * 8 + (ks >= 
 // ------------------------------------------------------------------------------------------
 // 1. D_i = dO_i . O_i and LSE_i * log2(e) per (padded) query row
 // ------------------------------------------------------------------------------------------
-constexpr int kPrepRowsPerBlock = 64;  // 8 warps x 8 rows
+constexpr int kPrepRowsPerBlock = 64;  // 8 warps x 8 rows per grid-stride step
 
 __global__ void __launch_bounds__(256)
     bwd_prep_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
@@ -196,47 +196,51 @@ __global__ void __launch_bounds__(256)
     }
     ds_off[num_kblocks] = acc;
   }
-  // a half-warp per row (16 lanes x 16 bytes = one 256-byte row of O and of dO); each warp
-  // takes 8 consecutive padded rows, every load issued before the first use
+  // a half-warp per row (16 lanes x 16 bytes = one 256-byte row of O and of dO); a warp takes
+  // groups of 8 consecutive padded rows, grid-stride (one wave of blocks), every load of a group
+  // issued before the first use
   const int lane = threadIdx.x & 31, sub = lane >> 4, sl = lane & 15;
-  const long long base = static_cast<long long>(blockIdx.x) * kPrepRowsPerBlock +
-                         (threadIdx.x >> 5) * 8;
-  uint4 a[4], g[4];
-  long long src[4];
+  const long long ngroups = (padded_rows + 7) / 8;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long grp = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       grp < ngroups; grp += stride) {
+    uint4 a[4], g[4];
+    long long src[4];
 #pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const long long prow = base + 2 * it + sub;
-    src[it] = -1;
-    if (prow < padded_rows) {
-      const int i = static_cast<int>(prow % npad);
-      if (i < Nq) src[it] = (prow / npad) * Nq + i;
-    }
-    a[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(o + src[it] * kD + sl * 8)
-                         : make_uint4(0u, 0u, 0u, 0u);
-    g[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(dout + src[it] * kD + sl * 8)
-                         : make_uint4(0u, 0u, 0u, 0u);
-  }
-#pragma unroll
-  for (int it = 0; it < 4; ++it) {
-    const uint32_t aw[4] = {a[it].x, a[it].y, a[it].z, a[it].w};
-    const uint32_t gw[4] = {g[it].x, g[it].y, g[it].z, g[it].w};
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(gw[w] << 16), acc);
-      acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(gw[w] & 0xffff0000u), acc);
+    for (int it = 0; it < 4; ++it) {
+      const long long prow = grp * 8 + 2 * it + sub;
+      src[it] = -1;
+      if (prow < padded_rows) {
+        const int i = static_cast<int>(prow % npad);
+        if (i < Nq) src[it] = (prow / npad) * Nq + i;
+      }
+      a[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(o + src[it] * kD + sl * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
+      g[it] = src[it] >= 0 ? *reinterpret_cast<const uint4*>(dout + src[it] * kD + sl * 8)
+                           : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
-    const long long prow = base + 2 * it + sub;
-    if (sl == 0 && prow < padded_rows) {
-      if (src[it] >= 0) {
-        dsum[prow] = acc;
-        const float l = lse[src[it]];
-        lse2[prow] = (l == -pos_inf()) ? pos_inf() : l * kLog2e;
-      } else {  // padding row past Nq
-        dsum[prow] = 0.f;
-        lse2[prow] = pos_inf();
+    for (int it = 0; it < 4; ++it) {
+      const uint32_t aw[4] = {a[it].x, a[it].y, a[it].z, a[it].w};
+      const uint32_t gw[4] = {g[it].x, g[it].y, g[it].z, g[it].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(gw[w] << 16), acc);
+        acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(gw[w] & 0xffff0000u), acc);
+      }
+#pragma unroll
+      for (int sh = 8; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
+      const long long prow = grp * 8 + 2 * it + sub;
+      if (sl == 0 && prow < padded_rows) {
+        if (src[it] >= 0) {
+          dsum[prow] = acc;
+          const float l = lse[src[it]];
+          lse2[prow] = (l == -pos_inf()) ? pos_inf() : l * kLog2e;
+        } else {  // padding row past Nq
+          dsum[prow] = 0.f;
+          lse2[prow] = pos_inf();
+        }
       }
     }
   }
