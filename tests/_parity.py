@@ -17,7 +17,7 @@ from oracle import oracle as O
 
 TOL_BF16 = dict(max_abs=2e-2, mean_abs=2e-3, lse_rel=1e-3)
 TOL_F32 = dict(max_abs=1e-4, mean_abs=1e-5, lse_rel=1e-5)
-# E4M3 forward: the weights 128 * P are rounded to E4M3 (3 mantissa bits) for the P V product.
+# E4M3 forward: the weights 16 * P are rounded to E4M3 (3 mantissa bits) for the P V product.
 # tests/test_tolerance_models.py recomputes the error of exactly that rounding against the
 # oracle and checks that these limits cover it with margin.
 TOL_FP8 = dict(max_abs=0.1, mean_abs=6e-3, lse_rel=1e-3)

@@ -2,7 +2,7 @@
 stand for (scale * E4M3(code), exact in fp64).
 
 Tolerance (derived from the arithmetic; the inputs are exact, so the only rounding beyond
-fp32 accumulation is that of the weights): the kernel rounds 128 * P to E4M3 (3 mantissa bits,
+fp32 accumulation is that of the weights): the kernel rounds 16 * P to E4M3 (3 mantissa bits,
 relative error up to 2^-4) for the P V product and keeps the row sums in fp32.  A numpy model of
 exactly that rounding against the oracle, on causal n = 512 and 2048, full n = 1024 and sliding
 w = 128 + 4 sinks, local + global and Nq != Nk, output rounded to bf16, gives a max error of

@@ -1,7 +1,7 @@
 """Where the E4M3 forward's and the backward's test tolerances come from.
 
 Both GPU paths round an intermediate to a narrow type before a tensor-core product, so they
-cannot meet the bf16 forward's limits: the E4M3 forward rounds the weights 128 * P to E4M3 for
+cannot meet the bf16 forward's limits: the E4M3 forward rounds the weights 16 * P to E4M3 for
 the P V product, and the backward rounds P and dS to bf16 for its four products and computes
 D_i = dO_i . O_i from the bf16 O.  The tests here model exactly those roundings in numpy (fp64
 everywhere else) and compare the model against the fp64 oracle on the inputs the GPU tests use:
@@ -10,7 +10,7 @@ margin.  A model, not a kernel: no code of the CUDA path is imported or run, and
 
 Readings:
 - the kernels' running-max bookkeeping (the E4M3 kernel rescales whenever the max grows by more
-  than one log2 unit) only moves where the E4M3 subnormal range starts, so the model takes P
+  than four log2 units) only moves where the E4M3 subnormal range starts, so the model takes P
   relative to the row's final max; the margin covers the rest (fp32 accumulation of the
   scores and sums, the ex2 approximation, bf16 rounding of the output, which the model does
   include);
@@ -73,7 +73,7 @@ def softmax_weights(S, vis):
 # E4M3 forward
 # ---------------------------------------------------------------------------------------------
 
-P_SCALE_F8 = 128.0  # the weights are scaled by 128 before they are rounded to E4M3
+P_SCALE_F8 = 16.0  # the weights are scaled by 16 before they are rounded to E4M3
 
 FP8_CASES = [  # (B, Hq, Hkv, Nq, Nk, mask, w, s): the shapes tests/test_gpu_fp8.py runs
     (1, 2, 1, 512, 512, CAUSAL, 0, 0),
