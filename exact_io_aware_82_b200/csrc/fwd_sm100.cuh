@@ -119,7 +119,9 @@ struct Unit {
   int nk;                // steps: key tiles the unit visits
   int s_total;           // S products of the unit (steps summed over the query tiles)
   int tiles;             // bit t: query tile t has rows (without a block-sparse layout, a tile
-                         // with rows takes part in every step of the unit)
+                         // with rows takes part in every step of the unit, but see rot)
+  int rot;               // 1: step 0 visits the second tile's extra key tile, which the first
+                         // tile skips; steps 1.. visit the rest of the range in order
   MaskSpec mask;         // mask.Nk is the sequence's key count in variable-length mode
   TileRange tr, trt[2];  // key tiles of the unit and of each query tile
 };
@@ -214,6 +216,7 @@ __device__ __forceinline__ bool decode_unit(const Params& p, int unit, Unit& u) 
   // tiles on every step lets them end together, so the next unit's products start at once
   // instead of after one tile's extra step.
   u.tiles = 0;
+  u.rot = 0;
   for (int t = 0; t < 2; ++t) {
     const int lo_row = pair ? u.r0 : u.r0 + t * kBM, hi_row = min(lo_row + kBM, u.nq) - 1;
     if (hi_row >= lo_row) u.tiles |= 1 << t;
@@ -221,7 +224,19 @@ __device__ __forceinline__ bool decode_unit(const Params& p, int unit, Unit& u) 
                : kSparse ? key_tiles(u.mask, lo_row + u.off, hi_row + u.off, kBN) : u.tr;
   }
   u.nk = u.tr.count();
+  // 256 causal rows of one head: the second tile sees one key tile (its diagonal) beyond the
+  // first tile's range.  That tile goes first, to the second tile alone, while the first tile
+  // starts on the next step: both tiles then end on the same step without a masked step.
+  if (!kSparse && !pair && u.tiles == 3 && u.mask.kind == ATTN_MASK_CAUSAL && u.tr.ns == 0) {
+    const TileRange a = key_tiles(u.mask, u.r0 + u.off, u.r0 + kBM - 1 + u.off, kBN);
+    if (a.ns == 0 && a.lo == u.tr.lo && a.hi + 1 == u.tr.hi) u.rot = 1;
+  }
   return true;
+}
+
+// Key tile of step j of a unit (non-sparse): the range in order, or (rot) its last tile first.
+__device__ __forceinline__ int unit_tile(const TileRange& tr, int rot, int j) {
+  return rot ? (j == 0 ? tr.hi : tr.lo + (j - 1)) : tr.tile(j);
 }
 
 // does a query tile with key-tile range r take part in the step whose key tile is u?
@@ -272,7 +287,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
   auto tile_head = [&](const Unit& u, int t) { return pair ? u.h + t : u.h; };
   // key tile of step j, and whether query tile t takes part in it
   auto step_tile = [&](const Unit& u, const SparseList& sl, int j) {
-    return kSparse ? sparse_tile(sl, j) : u.tr.tile(j);
+    return kSparse ? sparse_tile(sl, j) : unit_tile(u.tr, u.rot, j);
   };
 
   // ---- set-up ----
@@ -378,7 +393,7 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
           u.s_total = parts;
           if (lane == 0) sl.count = base;
         } else {
-          u.s_total = u.nk * __popc(u.tiles);
+          u.s_total = u.nk * __popc(u.tiles) - u.rot;
         }
       }
       if (lane == 0) sm.unit[slot] = u;
@@ -522,10 +537,10 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
         const SparseList& sl = lists[slot];
         ++taken;
         if (!us.valid) break;
-        const int nk = us.nk, s_total = us.s_total, tiles = us.tiles;
+        const int nk = us.nk, s_total = us.s_total, tiles = us.tiles, rot = us.rot;
         auto takes = [&](int t, int j) {
           if (kSparse) return sparse_part(sl, j, t);
-          return ((tiles >> t) & 1) != 0;
+          return ((tiles >> t) & 1) != 0 && !(rot && t == 0 && j == 0);
         };
         if (nk == 0) {
           dev::mbar_arrive(dev::smem_u32(&sm.bar_unit_empty[slot]));
@@ -669,7 +684,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       ++taken;
       const SparseList& sl = lists[slot];
       const int nk = us.nk;
-      const int tr_ns = us.tr.ns, tr_lo = us.tr.lo;  // step j -> key tile (dense)
+      const TileRange utr = us.tr;  // step j -> key tile (dense)
+      const int rot = us.rot;
       const bool mine = ((us.tiles >> t) & 1) != 0;  // this tile has rows
       const MaskSpec mask = us.mask;
       const int P0 = tile_row0(us, t) + us.off;  // key position of the tile's first row
@@ -682,8 +698,8 @@ __device__ __forceinline__ void fwd_sm100(const CUtensorMap& tm_q, const CUtenso
       float l = 0.f;            // running sum of exp2(s*c - m_ref)
       int cnt = 0;              // steps this tile has processed in this unit
       for (int j = 0; j < nk; ++j) {
-        const int kt = kSparse ? sparse_tile(sl, j) : (j < tr_ns ? j : tr_lo + (j - tr_ns));
-        if (kSparse ? !sparse_part(sl, j, t) : !mine) continue;
+        const int kt = kSparse ? sparse_tile(sl, j) : unit_tile(utr, rot, j);
+        if (kSparse ? !sparse_part(sl, j, t) : (!mine || (rot && t == 0 && j == 0))) continue;
         ok = wait_bounded(dev::smem_u32(&sm.bar_s[t]), stot & 1, abort);
         if (!(ok = __all_sync(0xffffffffu, ok))) break;
         dev::tc_fence_after();
