@@ -34,12 +34,14 @@
 // two issuing threads interleave the tiles on the tensor core and lengthen both chains).
 // tcgen05.mma executes in issue order, so S_t(j+1) never overwrites P_t(j) before PV_t(j)
 // has read it, and the commit that signals S_t(j+1) also covers PV_t(j): the softmax may then
-// rescale O_t.  A query tile skips the key tiles none of its rows can see.
+// rescale O_t.  A unit visits only the key tiles some of its rows can see; under a block-sparse
+// layout each query tile takes only its selected tiles, otherwise both tiles take every step
+// (an edge tile one of them cannot see adds exact zeros for it), except that in 256 causal rows
+// of one head the second tile's diagonal tile goes first, to that tile alone.
 #pragma once
 
 #include <cuda.h>
 #include <cuda_bf16.h>
-
 
 #include "common.cuh"
 #include "dev/ptx_f8.cuh"
