@@ -93,10 +93,10 @@ ATTN_API const char *attn_last_error_detail(void);
 
 /*
  * The prefill calls (attn_fwd, attn_fwd_block_sparse, attn_fwd_varlen, attn_fwd_fp8) and
- * attn_bwd run persistent grids whose CTAs take work from a 4-byte counter in device memory that the library
- * owns: one counter per stream (up to 1024 streams per device; later streams share the counter
- * of an earlier one, and two streams that share one must not run prefill calls at the same
- * time).  Calls on one stream are ordered and share its counter; a CUDA graph that captured a
+ * attn_bwd run persistent grids whose CTAs take work from a 4-byte counter in device memory
+ * that the library owns: one counter per stream (up to 1024 streams per device; later streams
+ * share the counter of an earlier one, and two streams that share one must not run these calls
+ * at the same time).  Calls on one stream are ordered and share its counter; a CUDA graph that captured a
  * call keeps the counter of the capturing stream, so two launches of such graphs must not run at
  * the same time.  The counter is back at zero when a call's kernel ends, also when it ended on
  * ATTN_ERR_DEVICE_TIMEOUT.  attn_bwd's dK/dV and dQ kernels use the same counter.
