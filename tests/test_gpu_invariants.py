@@ -145,6 +145,33 @@ def test_prefill_on_concurrent_streams_matches_serial():
     assert A.attn_get_device_error() == 0
 
 
+def test_backward_on_concurrent_streams_matches_serial():
+    """The persistent backward kernels share the per-stream work counter with the prefill: two
+    backward calls queued on two streams at once give the same bits as serial calls."""
+    cases = []
+    for seed, shape_q, shape_kv, kw in ((31, (1, 4, 700, 128), (1, 2, 700, 128), dict(mask_kind=CAUSAL)),
+                                        (32, (2, 2, 500, 128), (2, 1, 500, 128),
+                                         dict(mask_kind=SLIDING, window=200, n_sink=3))):
+        q, k, v = rnd(seed, 0, shape_q), rnd(seed, 1, shape_kv), rnd(seed, 2, shape_kv)
+        do = rnd(seed, 3, shape_q)
+        o, lse = A.attn_fwd(q, k, v, **kw)
+        cases.append((q, k, v, o, lse, do, kw))
+    serial = [A.attn_bwd(q, k, v, o, lse, do, **kw) for q, k, v, o, lse, do, kw in cases]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    torch.cuda.synchronize()
+    outs = [[], []]
+    for rep in range(3):
+        for si, (q, k, v, o, lse, do, kw) in enumerate(cases):
+            with torch.cuda.stream(streams[si]):
+                outs[si].append(A.attn_bwd(q, k, v, o, lse, do, stream=streams[si], **kw))
+    torch.cuda.synchronize()
+    for si in range(2):
+        for got in outs[si]:
+            for x, y in zip(got, serial[si]):
+                assert torch.equal(x, y)
+    assert A.attn_get_device_error() == 0
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     assert A.attn_get_device_error() == 0
     A.attn_debug_timeout_probe(2_000_000)  # ~1 ms of SM clocks on an mbarrier nobody completes
