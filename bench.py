@@ -108,13 +108,13 @@ MIN_TIMED_MS = 200.0
 # kernel family (kernel_sources_hash); reported as null once those sources differ.
 NCU_TRAFFIC = {
     "full_b1_h1_n256_d64_f32": {"bytes": 260608, "src": "02e210e28044d0c4"},
-    "causal_b4_h16_n2048_d128": {"bytes": 151330048, "src": "e353e585ff2e02b6"},
-    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 474978304, "src": "e353e585ff2e02b6"},
-    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 692300544, "src": "e353e585ff2e02b6"},
-    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1293218960, "src": "e353e585ff2e02b6"},
-    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 769709056, "src": "e353e585ff2e02b6"},
-    "fp8_causal_b4_h16_n2048_d128": {"bytes": 54126848, "src": "e353e585ff2e02b6"},
-    "block_sparse_b1_h32_kv8_n32768_d128": {"bytes": 912254208, "src": "e353e585ff2e02b6"},
+    "causal_b4_h16_n2048_d128": {"bytes": 130977024, "src": "e769cf1b4f770bb4"},
+    "gqa_causal_b2_h32_kv8_n8192_d128": {"bytes": 499211008, "src": "e769cf1b4f770bb4"},
+    "sliding_b1_h32_kv8_n32768_w4096_s4_d128": {"bytes": 703764224, "src": "e769cf1b4f770bb4"},
+    "varlen_causal_16seq_32k_h16_d128": {"bytes": 1233493784, "src": "e769cf1b4f770bb4"},
+    "local_global_b1_h32_kv8_n32768_w2048_g4_d128": {"bytes": 758468096, "src": "e769cf1b4f770bb4"},
+    "fp8_causal_b4_h16_n2048_d128": {"bytes": 54257408, "src": "e769cf1b4f770bb4"},
+    "block_sparse_b1_h32_kv8_n32768_d128": {"bytes": 913352960, "src": "e769cf1b4f770bb4"},
     # the backward step's three kernels together (prep + dK/dV + dQ)
     "bwd_causal_b4_h16_n2048_d128": {"bytes": 1037862144, "src": "0f208cebade179e6"},
     # a decode step's two kernels together (split + combine), captured on the 8-sequence
