@@ -47,11 +47,11 @@ int cuda_status(cudaError_t e) {
 }
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
-// Work-unit counters of the persistent prefill kernels, one per stream that launches them: calls
-// on one stream run one after another and can share a counter, calls on different streams may
-// overlap and must not.  A counter is zero between launches (the last CTA of a launch to take
-// from it sets it back).  Past kCounterSlots streams on one device, a stream shares the counter
-// of an earlier one.
+// Work-unit counters of the persistent prefill and backward kernels, one per stream that launches
+// them: calls on one stream run one after another and can share a counter, calls on different
+// streams may overlap and must not.  A counter is zero between launches (the last CTA of a launch
+// to take from it sets it back).  Past kCounterSlots streams on one device, a stream shares the
+// counter of an earlier one.
 constexpr int kCounterSlots = 1024;
 static __device__ unsigned int g_unit_counters[kCounterSlots];
 
