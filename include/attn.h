@@ -99,7 +99,9 @@ ATTN_API const char *attn_last_error_detail(void);
  * at the same time).  Calls on one stream are ordered and share its counter; a CUDA graph that captured a
  * call keeps the counter of the capturing stream, so two launches of such graphs must not run at
  * the same time.  The counter is back at zero when a call's kernel ends, also when it ended on
- * ATTN_ERR_DEVICE_TIMEOUT.  attn_bwd's dK/dV and dQ kernels use the same counter.
+ * ATTN_ERR_DEVICE_TIMEOUT.  attn_bwd's dK/dV and dQ kernels use the same counter.  The first
+ * such call on a device looks the counters' address up (make it before any stream capture) and
+ * keeps it for the life of the process: do not use the library across a device reset.
  */
 
 /*
